@@ -1,0 +1,433 @@
+"""Benchmark of the WorldAttention per-layer HKV + HSA step on B200.
+
+One step = page-level retrieval (hkv_select_pages) + active-cache gather
+(hkv_gather, with the fused 128-row K pooling) + hsa_forward (pooling, block
+selection, Linformer projection and attention, sparse attention with the gated
+merge), on the Wan-1.3B-shaped 480p workload: 12 heads, d = 128, a 4680-query
+chunk, 16 history pages of 12480 tokens resident in HBM, Kp = 4, r = 256.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload I]
+
+Prints one JSON line (rank 0).  N > 1 runs one independent replica per GPU
+(torchrun, NCCL for the barrier and the max-over-ranks timing only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "HSA layer query-tokens/s + eff. TFLOP/s on 1 B200; % tensor/HBM roofline"
+UNIT = "query-tokens/s"
+DEFAULT_WORKLOAD = 1
+
+# DRAM traffic per launch from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
+# keyed by kernel, valid only while the kernel's source file is unchanged (sha256 prefix).
+TRAFFIC = {}
+
+
+def _sha(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            m = json.load(f)
+        return {"hbm_gbs": m["hbm_gbs"], "bf16_tflops": m["bf16_tflops"],
+                "bf16_tflops_sustained": m.get("bf16_tflops_sustained", m["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ work model
+def step_work(shape):
+    """Algorithmic FLOPs and bytes of one step's dense parts (the sparse branch is
+    counted from the selection by exact_pairs)."""
+    H, d, Lq, Lc, r = shape.H, shape.d, shape.Lq, shape.Lc, shape.r
+    L = Lc + Lq
+    return {
+        "proj_flops": H * 4.0 * r * L * d,             # EK and FV: 2 * (2 r L d) per head
+        "lin_attn_flops": H * 4.0 * Lq * r * d,        # Q EK^T and P FV
+        "gather_bytes": 4.0 * Lc * H * d * 2,          # read + write of K and V pages
+        "proj_bytes": 2.0 * L * H * d * 2 + 2.0 * r * L * 2,
+        "pool_bytes": 2.0 * Lq * H * d * 2,            # Q and Kq read once
+        "select_pages_bytes": Lq * H * d * 2.0,        # Q read once
+    }
+
+
+def exact_pairs(shape, sel_bufs):
+    """Selected query-key pairs counted from the selection lists (partial blocks exact)."""
+    import numpy as np
+    H, Lq, Lc = shape.H, shape.Lq, shape.Lc
+    ic = sel_bufs.inter_cnt.cpu().numpy()
+    ii = sel_bufs.inter_idx.cpu().numpy()
+    qc = sel_bufs.intra_cnt.cpu().numpy()
+    qi = sel_bufs.intra_idx.cpu().numpy()
+    kc_size = np.array([min(128, Lc - 128 * j) for j in range(-(-Lc // 128))], dtype=np.float64)
+    kq_size = np.array([min(64, Lq - 64 * j) for j in range(-(-Lq // 64))], dtype=np.float64)
+    pairs = 0.0
+    for h in range(H):
+        for i in range(ic.shape[1]):
+            pairs += min(128, Lq - 128 * i) * kc_size[ii[h, i, :ic[h, i]]].sum()
+        for i in range(qc.shape[1]):
+            pairs += min(64, Lq - 64 * i) * kq_size[qi[h, i, :qc[h, i]]].sum()
+    return pairs, float(ic.sum()) / max(1, ic.size * len(kc_size)), float(qc.sum()) / max(1, qc.size * len(kq_size))
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index=0):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+def oracle_summaries(x, shape):
+    """Page summaries (computed when a page is sealed, outside the step)."""
+    import numpy as np
+    import oracle
+    return np.stack([oracle.page_summary(x.pages_k[p], np.float32) for p in range(shape.NP)])
+
+
+def oracle_step_sample(x, shape, kbar, rows_per_step=256, head=None):
+    """Time the fp64 oracle on a bounded sample of one step and extrapolate to the full step:
+    t_step = t_retrieval + H * (t_head_fixed + t_rows * Lq / rows)."""
+    import numpy as np
+    import oracle
+    h = shape.H // 2 if head is None else head
+    t0 = time.perf_counter()
+    sel, _ = oracle.select_pages(kbar, x.Q, shape.Kp)
+    Kc = oracle.gather_pages(x.pages_k, sel)
+    Vc = oracle.gather_pages(x.pages_v, sel)
+    t_r = time.perf_counter() - t0
+    sl = slice(h, h + 1)
+    Qh, Kch, Vch, Kqh, Vqh = x.Q[:, sl], Kc[:, sl], Vc[:, sl], x.Kq[:, sl], x.Vq[:, sl]
+    t0 = time.perf_counter()
+    selh = oracle.block_select(Qh, Kch, Kqh, x.tau[sl])
+    EK, FV = oracle.linear_projection(x.E, x.F, Kch, Kqh, Vch, Vqh)
+    t_fixed = time.perf_counter() - t0
+    rows = np.linspace(0, shape.Lq - 1, rows_per_step).astype(np.int64)
+    t0 = time.perf_counter()
+    o_s = oracle.sparse_attention(Qh, Kch, Vch, Kqh, Vqh, selh.inter, selh.intra, rows=rows)
+    o_l = oracle.linear_attention(Qh, EK, FV, rows=rows)
+    oracle.gated_merge(o_s, o_l, x.z[sl])
+    t_rows = time.perf_counter() - t0
+    t_step = t_r + shape.H * (t_fixed + t_rows * shape.Lq / len(rows))
+    sample = (f"page retrieval + gather once, then head {h} (tau {float(x.tau[h]):.2f}) alone: block selection, "
+              f"Linformer projection, both branches and merge on {len(rows)} of {shape.Lq} query rows; "
+              f"step time extrapolated as t_retrieval + H*(t_head + t_rows*Lq/rows)")
+    return t_step, sample, t_r + t_fixed + t_rows
+
+
+def blas_threads():
+    try:
+        import threadpoolctl
+        return max([i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()] + [1])
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        backend = os.environ.get("HSA_BENCH_BACKEND", "nccl")
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(value, world, device="cpu"):
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ arms
+def run_reference(args, shape, rank, world):
+    """The oracle as it stands, on the host cores, a bounded sample per step."""
+    if rank != 0:
+        return None
+    import synth
+    x = synth.make_inputs(shape, synth.seed_of(args.workload))
+    kbar = oracle_summaries(x, shape)
+    for _ in range(args.warmup):
+        oracle_step_sample(x, shape, kbar, rows_per_step=64)
+    ts = []
+    sample = ""
+    for _ in range(args.steps):
+        t, sample, _ = oracle_step_sample(x, shape, kbar, rows_per_step=64)
+        ts.append(t)
+    t_step = statistics.mean(ts)
+    value = shape.Lq / t_step
+    cores = blas_threads()
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": workload_config(shape, args),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+                         "cpu": cpu_model()},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def workload_config(shape, args):
+    return {"workload": shape.name, "H": shape.H, "d": shape.d, "Lq": shape.Lq, "Lc": shape.Lc, "L": shape.L,
+            "P_tok": shape.P_tok, "NP": shape.NP, "Kp": shape.Kp, "r": shape.r, "block_inter": 128,
+            "block_intra": 64, "tau": "1.00 -> 0.35 linear across heads", "pages": "host-pinned" if shape.host_pages else "HBM",
+            "l2": "flushed between timed steps (256 MiB write); inputs 1.3 GB > L2",
+            "parallelism": f"replicas x{getattr(args, 'gpus', 1)}"}
+
+
+def run_gpu(args, shape, rank, world, local):
+    import numpy as np
+    import torch
+
+    import synth
+    import hybrid_sparse_attention_hkv_b200 as hsa
+    from synth.device import DeviceStep
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    seed = synth.seed_of(args.workload) + rank  # each replica its own seeded inputs
+    ds = DeviceStep(shape, seed)
+    st = ds.step
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def one_step():
+        ds.run()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        one_step()
+    torch.cuda.synchronize()
+
+    trace = hsa.KernelTrace(max_kernels=16 * args.steps)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    with trace:
+        for k in range(args.steps):
+            flush.zero_()
+            starts[k].record(stream)
+            one_step()
+            ends[k].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier(world)
+    t_steps = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    t_total = sum(t_steps) / 1e3
+    t_max = max_over_ranks(t_total, world, dev if world > 1 and os.environ.get("HSA_BENCH_BACKEND", "nccl") == "nccl" else "cpu")
+    per_kernel = {}
+    launches = 0
+    for name, ms in trace.results():
+        launches += 1
+        d = per_kernel.setdefault(name, {"launches": 0, "ms": 0.0})
+        d["launches"] += 1
+        d["ms"] += ms
+    value = world * shape.Lq * args.steps / t_max
+    ms_per_step = t_max / args.steps * 1e3
+
+    # e2e: host buffers through the public API, copies inside the timed region
+    hQ = ds.Q.cpu().pin_memory()
+    hK = ds.Kq.cpu().pin_memory()
+    hV = ds.Vq.cpu().pin_memory()
+    hout = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
+    e_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for k in range(args.warmup + args.steps):
+        flush.zero_()
+        if k >= args.warmup:
+            e_s[k - args.warmup].record(stream)
+        ds.Q.copy_(hQ, non_blocking=True)
+        ds.Kq.copy_(hK, non_blocking=True)
+        ds.Vq.copy_(hV, non_blocking=True)
+        one_step()
+        hout.copy_(st.out, non_blocking=True)
+        if k >= args.warmup:
+            e_e[k - args.warmup].record(stream)
+    torch.cuda.synchronize()
+    t_e2e = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)) / 1e3, world,
+                           dev if world > 1 and os.environ.get("HSA_BENCH_BACKEND", "nccl") == "nccl" else "cpu")
+    e2e_value = world * shape.Lq * args.steps / t_e2e
+
+    # work and rooflines
+    peaks = load_peaks()
+    pairs, inter_frac, intra_frac = exact_pairs(shape, st.selection)
+    w = step_work(shape)
+    f_sparse = 4.0 * shape.d * pairs
+    f_total = f_sparse + w["proj_flops"] + w["lin_attn_flops"]
+    eff_tflops = f_total / (ms_per_step / 1e3) / 1e12
+    kernel_work = {
+        "sparse_attn_merge": ("tensor", f_sparse),
+        "linear_attn": ("tensor", w["lin_attn_flops"]),
+        "linformer_proj": ("tensor", w["proj_flops"]),
+        "gather": ("hbm", w["gather_bytes"]),
+        "pool": ("hbm", w["pool_bytes"]),
+        "colsum_partial": ("hbm", w["select_pages_bytes"]),
+    }
+    kernels = {}
+    for name, d in per_kernel.items():
+        avg_ms = d["ms"] / d["launches"]
+        entry = {"launches_per_step": d["launches"] / args.steps, "ms_per_launch": avg_ms,
+                 "share": d["ms"] / sum(v["ms"] for v in per_kernel.values())}
+        if name in kernel_work:
+            bound, work = kernel_work[name]
+            if bound == "tensor":
+                ach = work / (avg_ms / 1e3) / 1e12
+                entry.update({"bound": "tensor", "achieved": ach, "unit": "TFLOP/s",
+                              "frac": ach / peaks["bf16_tflops_sustained"]})
+            else:
+                ach = work / (avg_ms / 1e3) / 1e9
+                entry.update({"bound": "hbm", "achieved": ach, "unit": "GB/s", "frac": ach / peaks["hbm_gbs"]})
+        kernels[name] = entry
+    dom = max(kernels, key=lambda k: kernels[k]["share"])
+    de = kernels[dom]
+    bound = de.get("bound", "hbm")
+    peak = peaks["bf16_tflops_sustained"] if bound == "tensor" else peaks["hbm_gbs"]
+    traffic = None
+    tr = TRAFFIC.get(dom)
+    if tr and tr["sha"] == _sha(os.path.join(ROOT, "hybrid_sparse_attention_hkv_b200", "csrc", tr["file"])):
+        traffic = tr["bytes"]
+    roofline = {"kernel": dom, "bound": bound, "achieved": de.get("achieved"), "peak": peak,
+                "unit": "TFLOP/s" if bound == "tensor" else "GB/s", "frac": de.get("frac"), "traffic": traffic,
+                "peak_source": f"{peaks['source']} ({'bf16 sustained' if bound == 'tensor' else 'HBM copy'})"}
+
+    res = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded)",
+        "config": workload_config(shape, args),
+        "eff_tflops": eff_tflops,
+        "selected_fraction": {"inter": inter_frac, "intra": intra_frac},
+        "roofline": roofline,
+        "kernels": kernels,
+        "gpu_launches": launches,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": 3 * shape.Lq * shape.H * shape.d * 2,
+                "d2h_bytes_per_step": shape.Lq * shape.H * shape.d * 4},
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t_step, sample, spent = oracle_step_sample(ds.x, shape, oracle_summaries(ds.x, shape))
+        res["cpu_baseline"] = {"value": shape.Lq / t_step, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                               "sample": sample, "seconds": spent, "cpu": cpu_model()}
+    ds.close()
+    return res if rank == 0 else None
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)
+    import synth
+    shape = synth.SHAPES[args.workload]
+    rank, world, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        res = run_reference(args, shape, rank, world)
+    else:
+        res = run_gpu(args, shape, rank, world, local)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,442 @@
+// C-ABI entry points of the HKV + HSA library: host-side argument checks,
+// workspace layout, per-kernel trace events and the launch sequence of each call.
+// Nothing here allocates, frees or synchronises (hsa_status_read excepted).
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+thread_local char t_detail[512] = "";
+thread_local cudaEvent_t* t_events = nullptr;
+thread_local const char** t_names = nullptr;
+thread_local int t_pairs = 0;
+thread_local int t_count = 0;
+
+hsa_status_t fail(hsa_status_t code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_detail, sizeof(t_detail), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+// Records an event pair around one kernel launch when tracing is on.
+struct TraceScope {
+  cudaStream_t s;
+  int k = -1;
+  TraceScope(const char* name, cudaStream_t s_) : s(s_) {
+    if (t_events && t_count < t_pairs) {
+      k = t_count++;
+      cudaEventRecord(t_events[2 * k], s);
+      if (t_names) t_names[k] = name;
+    }
+  }
+  ~TraceScope() {
+    if (k >= 0) cudaEventRecord(t_events[2 * k + 1], s);
+  }
+};
+
+#define HSA_LAUNCH(name, call)                                                   \
+  do {                                                                           \
+    cudaError_t _e;                                                              \
+    {                                                                            \
+      TraceScope _tr(name, stream);                                              \
+      _e = (call);                                                               \
+    }                                                                            \
+    if (_e != cudaSuccess) return fail(HSA_ERR_CUDA, "%s: %s", name, cudaGetErrorString(_e)); \
+  } while (0)
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// `fn` is the name of the entry point being checked (each entry point defines it).
+#define REQUIRE_PTR(p)                                                                  \
+  do {                                                                                  \
+    if ((p) == nullptr) return fail(HSA_ERR_INVALID_ARG, "%s: " #p " is NULL", fn);     \
+    if (!aligned16(p)) return fail(HSA_ERR_INVALID_ARG, "%s: " #p " is not 16-byte aligned", fn); \
+  } while (0)
+#define OPTIONAL_PTR(p)                                                                 \
+  do {                                                                                  \
+    if ((p) != nullptr && !aligned16(p))                                                \
+      return fail(HSA_ERR_INVALID_ARG, "%s: " #p " is not 16-byte aligned", fn);        \
+  } while (0)
+
+// Workspace layout shared by every entry point (offsets in bytes).
+struct Layout {
+  size_t status = 0, colpart = 0, q128 = 0, q64 = 0, kq64 = 0, kc128 = 0;
+  size_t inter_idx = 0, inter_cnt = 0, intra_idx = 0, intra_cnt = 0;
+  size_t olin = 0, ekhi = 0, eklo = 0, fvhi = 0, fvlo = 0, projpart = 0;
+  size_t pages_end = 0;  // bytes needed by the page (HKV) calls
+  size_t total = 0;
+  int splits = 0;
+};
+
+Layout make_layout(int H, int d, int Lq, long long Lc, int r) {
+  Layout L;
+  size_t off = 256;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  const size_t hd = (size_t)H * d;
+  L.colpart = take((size_t)hsa::kColMaxSplits * hd * 4);
+  L.pages_end = off;
+  const size_t nQ128 = (Lq + 127) / 128, nQ64 = (Lq + 63) / 64, nKc = (size_t)((Lc + 127) / 128);
+  L.q128 = take(nQ128 * hd * 4);
+  L.q64 = take(nQ64 * hd * 4);
+  L.kq64 = take(nQ64 * hd * 4);
+  L.kc128 = take(nKc * hd * 4);
+  L.inter_idx = take((size_t)H * nQ128 * nKc * 4);
+  L.inter_cnt = take((size_t)H * nQ128 * 4);
+  L.intra_idx = take((size_t)H * nQ64 * nQ64 * 4);
+  L.intra_cnt = take((size_t)H * nQ64 * 4);
+  L.olin = take((size_t)Lq * hd * 4);
+  const size_t hrd = (size_t)H * r * d;
+  L.ekhi = take(hrd * 2);
+  L.eklo = take(hrd * 2);
+  L.fvhi = take(hrd * 2);
+  L.fvlo = take(hrd * 2);
+  L.splits = r > 0 ? hsa::proj_splits(H, r, Lc + Lq) : 0;
+  L.projpart = take((size_t)L.splits * 2 * hrd * 4);
+  L.total = off;
+  return L;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+inline int* status_of(void* ws) { return static_cast<int*>(ws); }
+
+hsa_status_t check_heads(const char* fn, int H, int d) {
+  if (H < 1) return fail(HSA_ERR_INVALID_ARG, "%s: H = %d must be >= 1", fn, H);
+  if (d <= 0) return fail(HSA_ERR_INVALID_ARG, "%s: d = %d must be positive", fn, d);
+  if (d != 64 && d != 128) return fail(HSA_ERR_UNSUPPORTED, "%s: d = %d (supported: 64, 128)", fn, d);
+  return HSA_OK;
+}
+
+hsa_status_t check_cfg(const char* fn, const hsa_config_t* c, bool need_rank) {
+  if (!c) return fail(HSA_ERR_INVALID_ARG, "%s: cfg is NULL", fn);
+  hsa_status_t st = check_heads(fn, c->H, c->d);
+  if (st != HSA_OK) return st;
+  if (c->Lq < 1) return fail(HSA_ERR_INVALID_ARG, "%s: Lq = %d must be >= 1", fn, c->Lq);
+  if (c->Lc < 0) return fail(HSA_ERR_INVALID_ARG, "%s: Lc = %d must be >= 0", fn, c->Lc);
+  if (c->block_inter != 128 || c->block_intra != 64)
+    return fail(HSA_ERR_UNSUPPORTED, "%s: block sizes %d/%d (supported: 128/64)", fn, c->block_inter, c->block_intra);
+  if (((long long)c->Lc + c->Lq) % 8 != 0)
+    return fail(HSA_ERR_UNSUPPORTED, "%s: Lc + Lq = %lld must be a multiple of 8", fn, (long long)c->Lc + c->Lq);
+  if ((c->Lc + 127) / 128 > hsa::kMaxSelBlocks || (c->Lq + 63) / 64 > hsa::kMaxSelBlocks)
+    return fail(HSA_ERR_UNSUPPORTED, "%s: more than %d blocks in a selection row", fn, hsa::kMaxSelBlocks);
+  if (!(c->scale >= 0.f) || isinf(c->scale)) return fail(HSA_ERR_INVALID_ARG, "%s: scale must be finite and >= 0", fn);
+  if (need_rank && (c->rank < 64 || c->rank > 1024 || c->rank % 64 != 0))
+    return fail(HSA_ERR_UNSUPPORTED, "%s: rank = %d (supported: multiples of 64 in [64, 1024])", fn, c->rank);
+  return HSA_OK;
+}
+
+inline float scale_of(const hsa_config_t* c) { return c->scale > 0.f ? c->scale : 1.0f / sqrtf((float)c->d); }
+
+hsa_status_t check_ws(const char* fn, const void* ws, size_t ws_bytes, size_t need) {
+  if (!ws) return fail(HSA_ERR_WORKSPACE, "%s: workspace is NULL", fn);
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(HSA_ERR_WORKSPACE, "%s: workspace not 256-byte aligned", fn);
+  if (ws_bytes < need) return fail(HSA_ERR_WORKSPACE, "%s: workspace %zu bytes < %zu needed", fn, ws_bytes, need);
+  return HSA_OK;
+}
+
+hsa_status_t check_sel(const char* fn, const hsa_selection_t& s) {
+  if (!s.inter_idx || !s.inter_cnt || !s.intra_idx || !s.intra_cnt)
+    return fail(HSA_ERR_INVALID_ARG, "%s: selection has a NULL array", fn);
+  if (!aligned16(s.inter_idx) || !aligned16(s.inter_cnt) || !aligned16(s.intra_idx) || !aligned16(s.intra_cnt))
+    return fail(HSA_ERR_INVALID_ARG, "%s: selection arrays must be 16-byte aligned", fn);
+  return HSA_OK;
+}
+
+#define TRY(x)                          \
+  do {                                  \
+    hsa_status_t _s = (x);              \
+    if (_s != HSA_OK) return _s;        \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char* hsa_status_string(hsa_status_t s) {
+  switch (s) {
+    case HSA_OK: return "HSA_OK";
+    case HSA_ERR_INVALID_ARG: return "HSA_ERR_INVALID_ARG";
+    case HSA_ERR_UNSUPPORTED: return "HSA_ERR_UNSUPPORTED";
+    case HSA_ERR_WORKSPACE: return "HSA_ERR_WORKSPACE";
+    case HSA_ERR_CUDA: return "HSA_ERR_CUDA";
+    case HSA_ERR_TIMEOUT: return "HSA_ERR_TIMEOUT";
+    case HSA_ERR_DEVICE: return "HSA_ERR_DEVICE";
+  }
+  return "HSA_ERR_UNKNOWN";
+}
+
+const char* hsa_last_error_detail(void) { return t_detail; }
+
+hsa_status_t hsa_workspace_size(const hsa_config_t* cfg, int NP, int P_tok, size_t* bytes) {
+  (void)NP;
+  (void)P_tok;
+  if (!bytes) return fail(HSA_ERR_INVALID_ARG, "hsa_workspace_size: bytes is NULL");
+  TRY(check_cfg("hsa_workspace_size", cfg, false));
+  *bytes = make_layout(cfg->H, cfg->d, cfg->Lq, cfg->Lc, cfg->rank > 0 ? cfg->rank : 0).total;
+  return HSA_OK;
+}
+
+hsa_status_t hsa_status_clear(void* ws, hsa_stream_t stream) {
+  if (!ws) return fail(HSA_ERR_WORKSPACE, "hsa_status_clear: workspace is NULL");
+  cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int), stream);
+  return e == cudaSuccess ? HSA_OK : fail(HSA_ERR_CUDA, "hsa_status_clear: %s", cudaGetErrorString(e));
+}
+
+hsa_status_t hsa_status_read(const void* ws, hsa_stream_t stream, int* status) {
+  if (!ws || !status) return fail(HSA_ERR_INVALID_ARG, "hsa_status_read: NULL argument");
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e == cudaSuccess) e = cudaMemcpy(status, ws, sizeof(int), cudaMemcpyDeviceToHost);
+  return e == cudaSuccess ? HSA_OK : fail(HSA_ERR_CUDA, "hsa_status_read: %s", cudaGetErrorString(e));
+}
+
+hsa_status_t hsa_trace_begin(void* const* events, int n_pairs, const char** names) {
+  if (events && n_pairs < 0) return fail(HSA_ERR_INVALID_ARG, "hsa_trace_begin: n_pairs < 0");
+  t_events = reinterpret_cast<cudaEvent_t*>(const_cast<void**>(events));
+  t_pairs = events ? n_pairs : 0;
+  t_names = names;
+  t_count = 0;
+  return HSA_OK;
+}
+int hsa_trace_count(void) { return t_count; }
+hsa_status_t hsa_trace_end(void) {
+  t_events = nullptr;
+  t_names = nullptr;
+  t_pairs = 0;
+  return HSA_OK;
+}
+
+// ------------------------------------------------------------------ HKV
+
+hsa_status_t hkv_page_summary(const hsa_bf16* K_page, int P_tok, int H, int d, float* kbar, void* ws,
+                              size_t ws_bytes, hsa_stream_t stream) {
+  const char* fn = __func__;
+  TRY(check_heads(fn, H, d));
+  if (P_tok < 1) return fail(HSA_ERR_INVALID_ARG, "%s: P_tok = %d must be >= 1", fn, P_tok);
+  REQUIRE_PTR(K_page);
+  REQUIRE_PTR(kbar);
+  const Layout L = make_layout(H, d, 1, 0, 0);
+  TRY(check_ws(fn, ws, ws_bytes, L.pages_end));
+  float* part = at<float>(ws, L.colpart);
+  HSA_LAUNCH("colsum_partial", hsa::launch_colsum_partial(K_page, P_tok, H * d, part, stream));
+  HSA_LAUNCH("page_summary_final", hsa::launch_page_summary_final(part, P_tok, H * d, kbar, stream));
+  return HSA_OK;
+}
+
+hsa_status_t hkv_select_prompt(const float* e_cur, const float* e_seg, int n_seg, int dim, const int32_t* seg_begin,
+                               int32_t* seg_out, int32_t* cand_range_out, hsa_stream_t stream) {
+  const char* fn = __func__;
+  if (n_seg < 1 || dim < 1) return fail(HSA_ERR_INVALID_ARG, "%s: n_seg = %d, dim = %d must be >= 1", fn, n_seg, dim);
+  REQUIRE_PTR(e_cur);
+  REQUIRE_PTR(e_seg);
+  REQUIRE_PTR(seg_begin);
+  if (!seg_out || !cand_range_out) return fail(HSA_ERR_INVALID_ARG, "%s: NULL output", fn);
+  HSA_LAUNCH("select_prompt", hsa::launch_select_prompt(e_cur, e_seg, n_seg, dim, seg_begin, seg_out, cand_range_out, stream));
+  return HSA_OK;
+}
+
+hsa_status_t hkv_select_pages(const float* kbar_pages, int NP, const int32_t* cand_range, const hsa_bf16* Q, int Lq,
+                              int H, int d, int Kp, int32_t* sel_out, float* scores_out, void* ws, size_t ws_bytes,
+                              hsa_stream_t stream) {
+  const char* fn = __func__;
+  TRY(check_heads(fn, H, d));
+  if (NP < 1 || Lq < 1) return fail(HSA_ERR_INVALID_ARG, "%s: NP = %d, Lq = %d must be >= 1", fn, NP, Lq);
+  if (Kp < 1 || Kp > NP || Kp > 64) return fail(HSA_ERR_INVALID_ARG, "%s: Kp = %d must be in [1, min(NP, 64)]", fn, Kp);
+  if ((size_t)H * d * 4 + (size_t)NP * 8 > 200 * 1024)
+    return fail(HSA_ERR_UNSUPPORTED, "%s: H*d*4 + NP*8 bytes exceed the shared-memory budget", fn);
+  REQUIRE_PTR(kbar_pages);
+  REQUIRE_PTR(Q);
+  if (!sel_out) return fail(HSA_ERR_INVALID_ARG, "%s: sel_out is NULL", fn);
+  const Layout L = make_layout(H, d, 1, 0, 0);
+  TRY(check_ws(fn, ws, ws_bytes, L.pages_end));
+  float* part = at<float>(ws, L.colpart);
+  HSA_LAUNCH("colsum_partial", hsa::launch_colsum_partial(Q, Lq, H * d, part, stream));
+  HSA_LAUNCH("select_pages_final", hsa::launch_select_pages_final(part, Lq, H * d, kbar_pages, NP, cand_range, Kp,
+                                                                  sel_out, scores_out, status_of(ws), stream));
+  return HSA_OK;
+}
+
+hsa_status_t hkv_gather(const hsa_bf16* const* page_k, const hsa_bf16* const* page_v, int NP, const int32_t* sel,
+                        int Kp, int P_tok, int H, int d, hsa_bf16* Kc, hsa_bf16* Vc, float* kbar128, void* ws,
+                        size_t ws_bytes, hsa_stream_t stream) {
+  const char* fn = __func__;
+  TRY(check_heads(fn, H, d));
+  if (NP < 1 || P_tok < 1) return fail(HSA_ERR_INVALID_ARG, "%s: NP = %d, P_tok = %d must be >= 1", fn, NP, P_tok);
+  if (Kp < 1 || Kp > NP) return fail(HSA_ERR_INVALID_ARG, "%s: Kp = %d must be in [1, NP]", fn, Kp);
+  if (!page_k || !page_v || !sel) return fail(HSA_ERR_INVALID_ARG, "%s: NULL page table or selection", fn);
+  REQUIRE_PTR(Kc);
+  REQUIRE_PTR(Vc);
+  OPTIONAL_PTR(kbar128);
+  TRY(check_ws(fn, ws, ws_bytes, 256));
+  HSA_LAUNCH("gather", hsa::launch_gather(reinterpret_cast<const uint16_t* const*>(page_k),
+                                          reinterpret_cast<const uint16_t* const*>(page_v), NP, sel, Kp, P_tok, H, d,
+                                          Kc, Vc, kbar128, status_of(ws), stream));
+  return HSA_OK;
+}
+
+// ------------------------------------------------------------------ HSA
+
+static hsa_status_t run_block_select(const hsa_config_t* cfg, const Layout& L, const hsa_bf16* Q, const hsa_bf16* Kc,
+                                     const hsa_bf16* Kq, const float* kbar128, const float* tau,
+                                     const hsa_selection_t& sel, void* ws, hsa_stream_t stream) {
+  float* q128 = at<float>(ws, L.q128);
+  float* q64 = at<float>(ws, L.q64);
+  float* kq64 = at<float>(ws, L.kq64);
+  float* kc128 = kbar128 ? const_cast<float*>(kbar128) : at<float>(ws, L.kc128);
+  HSA_LAUNCH("pool", hsa::launch_pool(Q, Kq, Kc, cfg->H, cfg->d, cfg->Lq, cfg->Lc, q128, q64, kq64,
+                                      kbar128 ? nullptr : kc128, stream));
+  HSA_LAUNCH("block_select", hsa::launch_block_select(q128, kc128, q64, kq64, tau, cfg->H, cfg->d, cfg->Lq, cfg->Lc,
+                                                      scale_of(cfg), sel.inter_idx, sel.inter_cnt, sel.intra_idx,
+                                                      sel.intra_cnt, stream));
+  return HSA_OK;
+}
+
+static hsa::AttnArgs attn_args(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc, const hsa_bf16* Vc,
+                               const hsa_bf16* Kq, const hsa_bf16* Vq) {
+  hsa::AttnArgs a;
+  memset(&a, 0, sizeof(a));
+  a.Q = Q; a.Kc = Kc; a.Vc = Vc; a.Kq = Kq; a.Vq = Vq;
+  a.H = cfg->H; a.d = cfg->d; a.Lq = cfg->Lq; a.Lc = cfg->Lc;
+  a.scale = scale_of(cfg);
+  a.r = cfg->rank;
+  return a;
+}
+
+static hsa_status_t run_linear(const hsa_config_t* cfg, const Layout& L, const hsa_bf16* Q, const hsa_bf16* Kc,
+                               const hsa_bf16* Vc, const hsa_bf16* Kq, const hsa_bf16* Vq, const hsa_bf16* E,
+                               const hsa_bf16* F, long long ef_head_stride, float* o_lin, void* ws,
+                               hsa_stream_t stream) {
+  float* part = at<float>(ws, L.projpart);
+  uint16_t* ekhi = at<uint16_t>(ws, L.ekhi);
+  uint16_t* eklo = at<uint16_t>(ws, L.eklo);
+  uint16_t* fvhi = at<uint16_t>(ws, L.fvhi);
+  uint16_t* fvlo = at<uint16_t>(ws, L.fvlo);
+  HSA_LAUNCH("linformer_proj", hsa::launch_proj(E, F, ef_head_stride, Kc, Kq, Vc, Vq, cfg->H, cfg->d, cfg->rank,
+                                                cfg->Lc, cfg->Lq, L.splits, part, stream));
+  HSA_LAUNCH("linformer_reduce", hsa::launch_proj_reduce(part, L.splits, cfg->H, cfg->d, cfg->rank, ekhi, eklo, fvhi,
+                                                         fvlo, stream));
+  hsa::AttnArgs a = attn_args(cfg, Q, Kc, Vc, Kq, Vq);
+  a.EKhi = ekhi; a.EKlo = eklo; a.FVhi = fvhi; a.FVlo = fvlo;
+  a.out_f32 = o_lin;
+  HSA_LAUNCH("linear_attn", hsa::launch_linear_attn(a, stream));
+  return HSA_OK;
+}
+
+static hsa_status_t check_tensors(const char* fn, const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc,
+                                  const hsa_bf16* Vc, const hsa_bf16* Kq, const hsa_bf16* Vq, bool needV) {
+  REQUIRE_PTR(Q);
+  REQUIRE_PTR(Kq);
+  if (needV) REQUIRE_PTR(Vq);
+  if (cfg->Lc > 0) {
+    REQUIRE_PTR(Kc);
+    if (needV) REQUIRE_PTR(Vc);
+  }
+  return HSA_OK;
+}
+
+hsa_status_t hsa_block_select(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc, const hsa_bf16* Kq,
+                              const float* kbar128, const float* tau, hsa_selection_t sel, void* ws, size_t ws_bytes,
+                              hsa_stream_t stream) {
+  const char* fn = __func__;
+  TRY(check_cfg(fn, cfg, false));
+  TRY(check_tensors(fn, cfg, Q, Kc, nullptr, Kq, nullptr, false));
+  OPTIONAL_PTR(kbar128);
+  if (!tau) return fail(HSA_ERR_INVALID_ARG, "%s: tau is NULL", fn);
+  TRY(check_sel(fn, sel));
+  const Layout L = make_layout(cfg->H, cfg->d, cfg->Lq, cfg->Lc, 0);
+  TRY(check_ws(fn, ws, ws_bytes, L.inter_idx));
+  return run_block_select(cfg, L, Q, Kc, Kq, kbar128, tau, sel, ws, stream);
+}
+
+hsa_status_t hsa_sparse_attn(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc, const hsa_bf16* Vc,
+                             const hsa_bf16* Kq, const hsa_bf16* Vq, hsa_selection_t sel, float* o_sparse, void* ws,
+                             size_t ws_bytes, hsa_stream_t stream) {
+  const char* fn = __func__;
+  (void)ws;
+  (void)ws_bytes;
+  TRY(check_cfg(fn, cfg, false));
+  TRY(check_tensors(fn, cfg, Q, Kc, Vc, Kq, Vq, true));
+  TRY(check_sel(fn, sel));
+  REQUIRE_PTR(o_sparse);
+  hsa::AttnArgs a = attn_args(cfg, Q, Kc, Vc, Kq, Vq);
+  a.inter_idx = sel.inter_idx; a.inter_cnt = sel.inter_cnt; a.intra_idx = sel.intra_idx; a.intra_cnt = sel.intra_cnt;
+  a.out_f32 = o_sparse;
+  a.status = ws ? status_of(ws) : nullptr;
+  HSA_LAUNCH("sparse_attn", hsa::launch_sparse_attn(a, stream));
+  return HSA_OK;
+}
+
+hsa_status_t hsa_linear_attn(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc, const hsa_bf16* Vc,
+                             const hsa_bf16* Kq, const hsa_bf16* Vq, const hsa_bf16* E, const hsa_bf16* F,
+                             long long ef_head_stride, float* o_linear, void* ws, size_t ws_bytes,
+                             hsa_stream_t stream) {
+  const char* fn = __func__;
+  TRY(check_cfg(fn, cfg, true));
+  TRY(check_tensors(fn, cfg, Q, Kc, Vc, Kq, Vq, true));
+  REQUIRE_PTR(E);
+  REQUIRE_PTR(F);
+  REQUIRE_PTR(o_linear);
+  if (ef_head_stride < 0 || ef_head_stride % 8 != 0)
+    return fail(HSA_ERR_INVALID_ARG, "%s: ef_head_stride must be >= 0 and a multiple of 8", fn);
+  const Layout L = make_layout(cfg->H, cfg->d, cfg->Lq, cfg->Lc, cfg->rank);
+  TRY(check_ws(fn, ws, ws_bytes, L.total));
+  return run_linear(cfg, L, Q, Kc, Vc, Kq, Vq, E, F, ef_head_stride, o_linear, ws, stream);
+}
+
+hsa_status_t hsa_forward(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc, const hsa_bf16* Vc,
+                         const hsa_bf16* Kq, const hsa_bf16* Vq, const float* kbar128, const float* tau,
+                         const float* gate_logit, const hsa_bf16* E, const hsa_bf16* F, long long ef_head_stride,
+                         void* out, int out_is_bf16, const hsa_selection_t* sel_out, void* ws, size_t ws_bytes,
+                         hsa_stream_t stream) {
+  const char* fn = __func__;
+  TRY(check_cfg(fn, cfg, true));
+  TRY(check_tensors(fn, cfg, Q, Kc, Vc, Kq, Vq, true));
+  OPTIONAL_PTR(kbar128);
+  if (!tau || !gate_logit) return fail(HSA_ERR_INVALID_ARG, "%s: tau / gate_logit is NULL", fn);
+  REQUIRE_PTR(E);
+  REQUIRE_PTR(F);
+  REQUIRE_PTR(out);
+  if (ef_head_stride < 0 || ef_head_stride % 8 != 0)
+    return fail(HSA_ERR_INVALID_ARG, "%s: ef_head_stride must be >= 0 and a multiple of 8", fn);
+  if (sel_out) TRY(check_sel(fn, *sel_out));
+  const Layout L = make_layout(cfg->H, cfg->d, cfg->Lq, cfg->Lc, cfg->rank);
+  TRY(check_ws(fn, ws, ws_bytes, L.total));
+
+  hsa_selection_t sel;
+  if (sel_out) {
+    sel = *sel_out;
+  } else {
+    sel.inter_idx = at<int32_t>(ws, L.inter_idx);
+    sel.inter_cnt = at<int32_t>(ws, L.inter_cnt);
+    sel.intra_idx = at<int32_t>(ws, L.intra_idx);
+    sel.intra_cnt = at<int32_t>(ws, L.intra_cnt);
+  }
+  TRY(run_block_select(cfg, L, Q, Kc, Kq, kbar128, tau, sel, ws, stream));
+  // linear branch first: its output is the merge input of the sparse kernel
+  float* o_lin = out_is_bf16 ? at<float>(ws, L.olin) : static_cast<float*>(out);
+  TRY(run_linear(cfg, L, Q, Kc, Vc, Kq, Vq, E, F, ef_head_stride, o_lin, ws, stream));
+  hsa::AttnArgs a = attn_args(cfg, Q, Kc, Vc, Kq, Vq);
+  a.inter_idx = sel.inter_idx; a.inter_cnt = sel.inter_cnt; a.intra_idx = sel.intra_idx; a.intra_cnt = sel.intra_cnt;
+  a.o_lin = o_lin;
+  a.gate_logit = gate_logit;
+  a.status = status_of(ws);
+  if (out_is_bf16) a.out_bf16 = static_cast<uint16_t*>(out);
+  else a.out_f32 = static_cast<float*>(out);
+  HSA_LAUNCH("sparse_attn_merge", hsa::launch_sparse_attn(a, stream));
+  return HSA_OK;
+}
+
+}  // extern "C"

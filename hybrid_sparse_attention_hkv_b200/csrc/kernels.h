@@ -1,0 +1,76 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the kernels.
+// Every launcher enqueues on `stream` and returns cudaGetLastError().
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace hsa {
+
+// ---------------------------------------------------------------- hkv.cu
+constexpr int kColMaxSplits = 296;  // 2 CTAs per SM for the column-sum partial pass
+
+int colsum_splits(long long n);  // number of row splits used for n rows
+cudaError_t launch_colsum_partial(const uint16_t* X, long long n, int C, float* part, cudaStream_t s);
+cudaError_t launch_page_summary_final(const float* part, long long n, int C, float* kbar, cudaStream_t s);
+cudaError_t launch_select_pages_final(const float* part, long long Lq, int C, const float* kbar_pages, int NP,
+                                      const int32_t* cand_range, int Kp, int32_t* sel_out, float* scores_out,
+                                      int* status, cudaStream_t s);
+cudaError_t launch_select_prompt(const float* e_cur, const float* e_seg, int n_seg, int dim,
+                                 const int32_t* seg_begin, int32_t* seg_out, int32_t* cand_range_out,
+                                 cudaStream_t s);
+cudaError_t launch_gather(const uint16_t* const* page_k, const uint16_t* const* page_v, int NP,
+                          const int32_t* sel, int Kp, long long P_tok, int H, int d, uint16_t* Kc,
+                          uint16_t* Vc, float* kbar128, int* status, cudaStream_t s);
+
+// ---------------------------------------------------------------- select.cu
+constexpr int kMaxSelBlocks = 8192;  // blocks per selection row (inter: ceil(Lc/128), intra: ceil(Lq/64))
+
+cudaError_t launch_pool(const uint16_t* Q, const uint16_t* Kq, const uint16_t* Kc, int H, int d, int Lq,
+                        long long Lc, float* q128, float* q64, float* kq64, float* kc128, cudaStream_t s);
+cudaError_t launch_block_select(const float* q128, const float* kc128, const float* q64, const float* kq64,
+                                const float* tau, int H, int d, int Lq, long long Lc, float scale,
+                                int32_t* inter_idx, int32_t* inter_cnt, int32_t* intra_idx, int32_t* intra_cnt,
+                                cudaStream_t s);
+
+// ---------------------------------------------------------------- attn.cu
+struct AttnArgs {
+  const uint16_t* Q;
+  const uint16_t* Kc;
+  const uint16_t* Vc;
+  const uint16_t* Kq;
+  const uint16_t* Vq;
+  int H, d, Lq;
+  long long Lc;
+  float scale;
+  // sparse branch
+  const int32_t* inter_idx;
+  const int32_t* inter_cnt;
+  const int32_t* intra_idx;
+  const int32_t* intra_cnt;
+  // linear branch: split-bf16 projections, [H][r][d]
+  const uint16_t* EKhi;
+  const uint16_t* EKlo;
+  const uint16_t* FVhi;
+  const uint16_t* FVlo;
+  int r;
+  // output [Lq, H, d]: fp32 (out_f32) or bf16 (out_bf16)
+  float* out_f32;
+  uint16_t* out_bf16;
+  // gated merge (sparse kernel only): out = g*o_sparse + (1-g)*o_lin, g = sigmoid(gate_logit[h])
+  const float* o_lin;
+  const float* gate_logit;
+  int* status;  // workspace status word (may be NULL)
+};
+cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t s);
+cudaError_t launch_linear_attn(const AttnArgs& a, cudaStream_t s);
+
+// ---------------------------------------------------------------- proj.cu
+int proj_splits(int H, int r, long long L);
+cudaError_t launch_proj(const uint16_t* E, const uint16_t* F, long long ef_head_stride, const uint16_t* Kc,
+                        const uint16_t* Kq, const uint16_t* Vc, const uint16_t* Vq, int H, int d, int r,
+                        long long Lc, int Lq, int splits, float* part, cudaStream_t s);
+cudaError_t launch_proj_reduce(const float* part, int splits, int H, int d, int r, uint16_t* EKhi,
+                               uint16_t* EKlo, uint16_t* FVhi, uint16_t* FVlo, cudaStream_t s);
+
+}  // namespace hsa

@@ -1,0 +1,63 @@
+"""One per-layer HKV + HSA step over a page store, through the C ABI.
+
+``HkvHsaStep`` owns the device buffers of a step (selected page ids, the
+contiguous active cache, block selections, workspace, output) and issues the
+C-ABI calls in the order of the method's overall architecture (WorldAttention
+project page, figure "Overall architecture of WorldAttention"): optional
+prompt-level Top-1, page-level top-Kp retrieval, gather, HSA forward.  All
+arithmetic happens in the library's kernels.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (SelectionBuffers, hkv_gather, hkv_page_summary, hkv_select_pages, hkv_select_prompt,
+               hsa_forward, hsa_workspace_size, make_config)
+
+
+def page_pointers(pages: torch.Tensor) -> torch.Tensor:
+    """Device int64 tensor of the base addresses of pages[p] for a [NP, P_tok, H, d] store
+    (device memory or page-locked host memory)."""
+    NP = pages.shape[0]
+    stride = pages.stride(0) * pages.element_size()
+    base = pages.data_ptr()
+    return torch.tensor([base + p * stride for p in range(NP)], dtype=torch.int64, device="cuda")
+
+
+class HkvHsaStep:
+    def __init__(self, H, d, Lq, P_tok, NP, Kp, rank, page_k_ptrs, page_v_ptrs, out_dtype=torch.float32,
+                 scale=0.0, device="cuda"):
+        self.H, self.d, self.Lq, self.P_tok, self.NP, self.Kp, self.rank = H, d, Lq, P_tok, NP, Kp, rank
+        self.Lc = Kp * P_tok
+        self.cfg = make_config(H, d, Lq, self.Lc, rank, scale)
+        dev = torch.device(device)
+        self.page_k_ptrs, self.page_v_ptrs = page_k_ptrs, page_v_ptrs
+        self.kbar_pages = torch.zeros(NP, H, d, dtype=torch.float32, device=dev)
+        self.sel = torch.zeros(Kp, dtype=torch.int32, device=dev)
+        self.scores = torch.zeros(NP, dtype=torch.float32, device=dev)
+        self.cand_range = torch.zeros(2, dtype=torch.int32, device=dev)
+        self.seg = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.Kc = torch.empty(self.Lc, H, d, dtype=torch.bfloat16, device=dev)
+        self.Vc = torch.empty(self.Lc, H, d, dtype=torch.bfloat16, device=dev)
+        self.kbar128 = torch.zeros(-(-self.Lc // 128), H, d, dtype=torch.float32, device=dev)
+        self.selection = SelectionBuffers.empty(self.cfg, dev)
+        self.ws = torch.zeros(hsa_workspace_size(self.cfg, NP, P_tok), dtype=torch.uint8, device=dev)
+        self.out = torch.empty(Lq, H, d, dtype=out_dtype, device=dev)
+
+    def seal_pages(self, pages_k: torch.Tensor):
+        """Page summaries (mean key per head) of every page, computed once."""
+        for p in range(self.NP):
+            hkv_page_summary(pages_k[p], self.kbar_pages[p], self.ws)
+
+    def __call__(self, Q, Kq, Vq, tau, gate_logit, E, F, e_cur=None, e_seg=None, seg_begin=None,
+                 ef_head_stride=0):
+        cand = None
+        if e_cur is not None:
+            hkv_select_prompt(e_cur, e_seg, seg_begin, self.seg, self.cand_range)
+            cand = self.cand_range
+        hkv_select_pages(self.kbar_pages, Q, self.Kp, self.sel, self.ws, self.scores, cand)
+        hkv_gather(self.page_k_ptrs, self.page_v_ptrs, self.sel, self.Kp, self.P_tok, self.H, self.d,
+                   self.Kc, self.Vc, self.ws, self.kbar128)
+        hsa_forward(self.cfg, Q, self.Kc, self.Vc, Kq, Vq, tau, gate_logit, E, F, self.out, self.ws,
+                    self.kbar128, self.selection, ef_head_stride)
+        return self.out

@@ -1,0 +1,220 @@
+/*
+ * hsa.h -- C ABI of the WorldAttention per-layer attention step on NVIDIA B200
+ * (sm_100a): Hierarchical KV Cache (HKV) retrieval + Hybrid Sparse Attention
+ * (HSA).
+ *
+ * Method sources (cited by short name below):
+ *   [NEWS] "WorldAttention pairs hierarchical KV caching with hybrid sparse
+ *          attention to reach 22 FPS on a single H100 and 0.9472 subject
+ *          consistency on VBench-Long" (English news summary of the paper):
+ *          HKV paragraph, HSA paragraph, kernel paragraph, open-questions
+ *          paragraph.
+ *   [PROJ] WorldAttention project page, Method figures ("Overall architecture
+ *          of WorldAttention"; "three-tier hierarchical KV cache with
+ *          prompt-level and page-level retrieval").
+ *
+ * Conventions shared by every entry point
+ *   - bf16 tensors are passed as hsa_bf16 (the 16-bit pattern).  Token-major
+ *     tensors are [tokens, H, d], row stride H*d elements, densely packed.
+ *     A history page is K_p, V_p in [P_tok, H, d].
+ *   - Every pointer argument is a DEVICE pointer (or, where stated, a pointer
+ *     to page-locked host memory mapped into the device address space), 16-byte
+ *     aligned.  The caller owns all memory: the library never allocates, frees
+ *     or synchronises (hsa_status_read is the one documented exception).
+ *   - All work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream).
+ *   - Arguments are validated on the host before anything is launched; a
+ *     failed check returns HSA_ERR_INVALID_ARG / HSA_ERR_UNSUPPORTED /
+ *     HSA_ERR_WORKSPACE and launches nothing.  hsa_last_error_detail() then
+ *     describes the check (thread-local text).
+ *   - A launch failure returns HSA_ERR_CUDA.  Conditions only the device can
+ *     see (for example a candidate page range shorter than Kp, or a bounded
+ *     device wait that ran out) are written as an hsa_status_t code into the
+ *     status word at the start of the workspace; read it with hsa_status_read
+ *     after the stream has reached the call.
+ *   - Workspace: one caller-allocated device buffer of hsa_workspace_size()
+ *     bytes (256-byte aligned) serves every entry point of a configuration.
+ *     Calls that share a workspace must be ordered on one stream.
+ *   - Supported shapes: d in {64, 128}; H >= 1; block_inter = 128;
+ *     block_intra = 64; rank a multiple of 64 in [64, 1024]; (Lc + Lq) a
+ *     multiple of 8; Lq >= 1.  Lc may be 0 (no retrieved history) and need not
+ *     be a multiple of 128 (a partial last inter block is the mean of its rows).
+ */
+#ifndef HSA_H_
+#define HSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t hsa_bf16;                  /* bfloat16 bit pattern */
+typedef struct CUstream_st* hsa_stream_t;   /* == cudaStream_t */
+
+typedef enum {
+  HSA_OK = 0,
+  HSA_ERR_INVALID_ARG = 1,   /* null / misaligned pointer, bad size */
+  HSA_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. d = 96) */
+  HSA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than hsa_workspace_size() */
+  HSA_ERR_CUDA = 4,          /* a CUDA launch or API call failed */
+  HSA_ERR_TIMEOUT = 5,       /* (device status) a bounded device wait ran out */
+  HSA_ERR_DEVICE = 6         /* (device status) a device-side check failed */
+} hsa_status_t;
+
+/* Human-readable name of a status code (static storage). */
+const char* hsa_status_string(hsa_status_t s);
+
+/* Text of the last failing host-side check on this thread ("" if none). */
+const char* hsa_last_error_detail(void);
+
+/* Shape of one HSA call.  [NEWS] HSA paragraph: Binter = 128 against the cached
+ * KV, Bintra = 64 inside the current chunk, Linformer rank r. */
+typedef struct {
+  int H;             /* heads */
+  int d;             /* head dim: 64 or 128 */
+  int Lq;            /* queries (= chunk tokens = chunk keys) */
+  int Lc;            /* cached (retrieved) KV tokens */
+  int block_inter;   /* must be 128 */
+  int block_intra;   /* must be 64 */
+  int rank;          /* Linformer r */
+  float scale;       /* softmax scale; 0 means 1/sqrt(d) */
+} hsa_config_t;
+
+/* Per-head block selections (device buffers, written by hsa_block_select).
+ * nQ128 = ceil(Lq/128), nKc = ceil(Lc/128), nQ64 = ceil(Lq/64), nKq = ceil(Lq/64).
+ * Row (h, i) of inter_idx holds inter_cnt[h*nQ128+i] ascending block ids of Kc,
+ * the rest of the row is unspecified; likewise for intra. */
+typedef struct {
+  int32_t* inter_idx;   /* [H][nQ128][nKc] */
+  int32_t* inter_cnt;   /* [H][nQ128]      */
+  int32_t* intra_idx;   /* [H][nQ64][nKq]  */
+  int32_t* intra_cnt;   /* [H][nQ64]       */
+} hsa_selection_t;
+
+/* Bytes of workspace every entry point below needs for `cfg` with NP history
+ * pages of P_tok tokens (NP, P_tok may be 0 when only hsa_* calls are used).
+ * The size includes the 256-byte status header. */
+hsa_status_t hsa_workspace_size(const hsa_config_t* cfg, int NP, int P_tok, size_t* bytes);
+
+/* Clear the device status word of `ws` (enqueued on `stream`). */
+hsa_status_t hsa_status_clear(void* ws, hsa_stream_t stream);
+
+/* Synchronise `stream`, then copy the device status word of `ws` into *status
+ * (an hsa_status_t value).  The only call that synchronises. */
+hsa_status_t hsa_status_read(const void* ws, hsa_stream_t stream, int* status);
+
+/* ---------------------------------------------------------------- HKV ---- */
+
+/* Page descriptor ([NEWS] HKV paragraph; reading: the mean key of the page per
+ * head, computed once when the page is sealed):
+ *   kbar[h*d + c] = (1/P_tok) * sum_t K_page[t, h, c]            (fp32 out)
+ * K_page: [P_tok, H, d] bf16 (device or mapped pinned host).  kbar: [H*d] fp32.
+ * Deterministic (fixed reduction order).  Uses the workspace. */
+hsa_status_t hkv_page_summary(const hsa_bf16* K_page, int P_tok, int H, int d, float* kbar,
+                              void* ws, size_t ws_bytes, hsa_stream_t stream);
+
+/* Stage 1, prompt-level retrieval ([NEWS] HKV and open-questions paragraphs:
+ * Top-1): s* = argmax_s cos(e_cur, e_seg[s]) (ties -> lowest s); then
+ *   seg_out[0] = s*,  cand_range_out = { seg_begin[s*], seg_begin[s*+1] }.
+ * e_cur: [dim] fp32; e_seg: [n_seg, dim] fp32; seg_begin: [n_seg+1] int32
+ * (segment s owns pages [seg_begin[s], seg_begin[s+1])).  All device. */
+hsa_status_t hkv_select_prompt(const float* e_cur, const float* e_seg, int n_seg, int dim,
+                               const int32_t* seg_begin, int32_t* seg_out, int32_t* cand_range_out,
+                               hsa_stream_t stream);
+
+/* Stage 2, page-level retrieval ([NEWS] HKV paragraph, Table 5: Kp = 4):
+ *   qbar[h] = mean_t Q[t, h, :];   s_p = sum_h qbar[h] . kbar_pages[p, h, :]
+ * keeps the Kp candidates with the largest s_p (ties -> lower p) and writes
+ * them to sel_out[0..Kp) in ascending page order.
+ * kbar_pages: [NP, H, d] fp32 (from hkv_page_summary).  cand_range: device
+ * int32[2] {first, end} or NULL for all NP pages; a range with fewer than Kp
+ * pages sets HSA_ERR_DEVICE in the workspace status and writes -1s.
+ * scores_out: optional [NP] fp32 (entries outside the range are -inf).
+ * Q: [Lq, H, d] bf16.  Uses the workspace. */
+hsa_status_t hkv_select_pages(const float* kbar_pages, int NP, const int32_t* cand_range,
+                              const hsa_bf16* Q, int Lq, int H, int d, int Kp,
+                              int32_t* sel_out, float* scores_out,
+                              void* ws, size_t ws_bytes, hsa_stream_t stream);
+
+/* Active-cache assembly ([NEWS] HKV and kernel paragraphs: KV-cache
+ * reorganisation into contiguous memory): for i < Kp,
+ *   Kc[i*P_tok + t] = page_k[sel[i]][t],  Vc[i*P_tok + t] = page_v[sel[i]][t]
+ * (bitwise copies).  page_k/page_v: device arrays of NP page pointers; a page
+ * may live in device memory or in mapped page-locked host memory (the lower
+ * tier), read directly by the copy kernel.  sel: device int32[Kp], values
+ * checked on the device (out of range -> HSA_ERR_DEVICE status, row skipped).
+ * Kc, Vc: [Kp*P_tok, H, d] bf16.  kbar128 (optional): [ceil(Lc/128), H, d]
+ * fp32 block means of Kc, fused into the copy (pass it to hsa_block_select). */
+hsa_status_t hkv_gather(const hsa_bf16* const* page_k, const hsa_bf16* const* page_v, int NP,
+                        const int32_t* sel, int Kp, int P_tok, int H, int d,
+                        hsa_bf16* Kc, hsa_bf16* Vc, float* kbar128,
+                        void* ws, size_t ws_bytes, hsa_stream_t stream);
+
+/* ---------------------------------------------------------------- HSA ---- */
+
+/* Head-adaptive block selection ([NEWS] HSA paragraph).  Pools Q and Kc into
+ * 128-row block means and Q and Kq into 64-row block means (a partial block is
+ * the mean of its real rows), scores S = qbar . kbar * scale per head, softmaxes
+ * each row, ranks blocks by mass (ties -> lower index) and keeps the shortest
+ * prefix whose cumulative mass is >= tau[h] (tau >= 1 keeps all; at least one
+ * block).  The inter map (128-query blocks x Kc blocks) and the intra map
+ * (64-query blocks x Kq blocks) are thresholded separately.
+ * Q, Kq: [Lq, H, d]; Kc: [Lc, H, d] bf16; kbar128: optional fp32 block means of
+ * Kc from hkv_gather (NULL -> pooled here); tau: [H] fp32.
+ * Masses are accumulated in fp64; scores are fp32. */
+hsa_status_t hsa_block_select(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc,
+                              const hsa_bf16* Kq, const float* kbar128, const float* tau,
+                              hsa_selection_t sel, void* ws, size_t ws_bytes, hsa_stream_t stream);
+
+/* Sparse branch ([NEWS] HSA paragraph): for query t of head h, exact softmax
+ * attention over the tokens of the Kc blocks sel.inter(h, t/128) together with
+ * the Kq blocks sel.intra(h, t/64), one joint softmax, no causal mask:
+ *   o_sparse[t, h, :] = sum_k softmax_k(q_t . k * scale) v_k        (fp32 out)
+ * Q, Kq, Vq: [Lq, H, d]; Kc, Vc: [Lc, H, d] bf16; o_sparse: [Lq, H, d] fp32. */
+hsa_status_t hsa_sparse_attn(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc,
+                             const hsa_bf16* Vc, const hsa_bf16* Kq, const hsa_bf16* Vq,
+                             hsa_selection_t sel, float* o_sparse,
+                             void* ws, size_t ws_bytes, hsa_stream_t stream);
+
+/* Linear branch ([NEWS] HSA paragraph, Linformer-style low rank):
+ *   EK_h = E_h [Kc; Kq]_h,  FV_h = F_h [Vc; Vq]_h   (E_h, F_h: [r, L], L = Lc+Lq)
+ *   o_linear[t, h, :] = softmax_j(q_t . EK_h[j] * scale) FV_h        (fp32 out)
+ * E, F: bf16 [r, L] row-major; head h reads E + h*ef_head_stride (0 = one
+ * matrix shared by all heads).  EK/FV are accumulated in fp32 and applied with
+ * split-bf16 (hi + lo) operands.  Uses the workspace. */
+hsa_status_t hsa_linear_attn(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc,
+                             const hsa_bf16* Vc, const hsa_bf16* Kq, const hsa_bf16* Vq,
+                             const hsa_bf16* E, const hsa_bf16* F, long long ef_head_stride,
+                             float* o_linear, void* ws, size_t ws_bytes, hsa_stream_t stream);
+
+/* Whole HSA step ([PROJ] overall architecture): block selection, linear branch,
+ * sparse branch and the gated merge ([NEWS] HSA paragraph, learned gates;
+ * reading: one sigmoid gate per head)
+ *   g_h = 1 / (1 + exp(-gate_logit[h]));  out = g_h * o_sparse + (1 - g_h) * o_linear
+ * kbar128: optional Kc block means from hkv_gather (NULL -> pooled here).
+ * gate_logit may be +-inf (g exactly 1 or 0).  out: [Lq, H, d], fp32 when
+ * out_is_bf16 == 0, else bf16.  sel_out: optional; when given, the selection
+ * is written there (otherwise kept in the workspace).  Uses the workspace. */
+hsa_status_t hsa_forward(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc,
+                         const hsa_bf16* Vc, const hsa_bf16* Kq, const hsa_bf16* Vq,
+                         const float* kbar128, const float* tau, const float* gate_logit,
+                         const hsa_bf16* E, const hsa_bf16* F, long long ef_head_stride,
+                         void* out, int out_is_bf16, const hsa_selection_t* sel_out,
+                         void* ws, size_t ws_bytes, hsa_stream_t stream);
+
+/* Optional per-kernel timing hook (tracing).  When `events` is non-NULL, the
+ * next entry-point calls on this thread record events[2*k] before and
+ * events[2*k+1] after their k-th kernel launch, for k < n_pairs, and store the
+ * kernel's name pointer in names[k] (may be NULL).  hsa_trace_count() returns
+ * how many pairs were recorded since the last hsa_trace_begin(). */
+hsa_status_t hsa_trace_begin(void* const* events, int n_pairs, const char** names);
+int hsa_trace_count(void);
+hsa_status_t hsa_trace_end(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HSA_H_ */

@@ -140,6 +140,8 @@ def block_probs(qbar, kbar, scale, dtype=np.float64) -> np.ndarray:
     """Block attention mass: per head, row i of softmax_j(qbar_i . kbar_j * scale).
     qbar: [nQ, H, d], kbar: [nK, H, d] -> [H, nQ, nK] (float64)."""
     s = _as(np.einsum("ihc,jhc->hij", np.asarray(qbar, np.float64), np.asarray(kbar, np.float64)) * scale, dtype)
+    if s.shape[2] == 0:  # no retrieved history: an empty map, nothing to keep
+        return s
     s = s - s.max(axis=2, keepdims=True)
     e = np.exp(s)
     return e / e.sum(axis=2, keepdims=True)

@@ -1,0 +1,277 @@
+"""GPU parity of every step of the path against the fp64 oracle, on shapes the
+oracle finishes in seconds that still span several tiles and a ragged tail, plus
+edge cases and the invariants the method fixes.  All calls go through the C ABI."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from hsa_testlib import (DeviceStep, assert_close, bits_of, check_pages, check_selection, errors,
+                         selection_lists, to_dev)
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import hybrid_sparse_attention_hkv_b200 as hsa
+    from hybrid_sparse_attention_hkv_b200 import SelectionBuffers, make_config
+
+# several 128-query tiles, a ragged query tail, pages not a multiple of 128 tokens
+SMALL = [
+    synth.StepShape("h3_d128_lq296_p200", H=3, d=128, frames=1, F_tok=296, page_frames=1, page_tok=200,
+                    NP=6, Kp=3, r=128),
+    synth.StepShape("h2_d64_lq200_p136", H=2, d=64, frames=1, F_tok=200, page_frames=1, page_tok=136,
+                    NP=5, Kp=2, r=64),
+    synth.StepShape("h4_d128_lq520_p384_biased", H=4, d=128, frames=2, F_tok=260, page_frames=1, page_tok=384,
+                    NP=8, Kp=2, r=192, n_biased=2),
+]
+
+
+def _ids(s):
+    return s.name
+
+
+@pytest.fixture(scope="module", params=SMALL, ids=_ids)
+def small(request):
+    ds = DeviceStep(request.param, 77)
+    ds.run()
+    torch.cuda.synchronize()
+    yield ds
+    ds.close()
+
+
+def test_page_summaries(small):
+    x = small.x
+    ref = np.stack([oracle.page_summary(x.pages_k[p]) for p in range(small.shape.NP)])
+    got = small.step.kbar_pages.cpu().numpy().astype(np.float64)
+    np.testing.assert_allclose(got, ref, rtol=1e-5, atol=1e-6)
+
+
+def test_page_selection(small):
+    x, st = small.x, small.step
+    kbar = st.kbar_pages.cpu().numpy()
+    sel_ref, scores_ref = oracle.select_pages(kbar, x.Q, small.shape.Kp)
+    scores = st.scores.cpu().numpy()
+    np.testing.assert_allclose(scores, scores_ref, rtol=1e-5, atol=1e-5 * np.abs(scores_ref).max())
+    check_pages(st.sel.cpu().numpy(), sel_ref, scores_ref, small.shape.Kp)
+    assert np.all(np.diff(st.sel.cpu().numpy()) > 0)
+    if x.biased:
+        assert set(x.biased) <= set(st.sel.cpu().numpy().tolist())
+
+
+def test_gather_bitwise_and_fused_pooling(small):
+    x, st = small.x, small.step
+    sel = st.sel.cpu().numpy()
+    assert np.array_equal(bits_of(st.Kc), oracle.gather_pages(x.pages_k, sel))
+    assert np.array_equal(bits_of(st.Vc), oracle.gather_pages(x.pages_v, sel))
+    ref = oracle.block_means(bits_of(st.Kc), 128)
+    np.testing.assert_allclose(st.kbar128.cpu().numpy(), ref, rtol=1e-5, atol=1e-6)
+
+
+def test_block_selection(small):
+    x, st = small.x, small.step
+    Kc = bits_of(st.Kc)
+    ref = oracle.block_select(x.Q, Kc, x.Kq, x.tau, dtype=np.float32)
+    sb = st.selection
+    gi = selection_lists(sb.inter_idx.cpu().numpy(), sb.inter_cnt.cpu().numpy())
+    gq = selection_lists(sb.intra_idx.cpu().numpy(), sb.intra_cnt.cpu().numpy())
+    n1, e1 = check_selection(gi, ref.inter, ref.p_inter, x.tau, "inter")
+    n2, e2 = check_selection(gq, ref.intra, ref.p_intra, x.tau, "intra")
+    assert e1 + e2 <= max(1, (n1 + n2) // 100)
+
+
+def test_forward_output(small):
+    x, st = small.x, small.step
+    Kc, Vc = bits_of(st.Kc), bits_of(st.Vc)
+    sb = st.selection
+    sel = oracle.Selection(selection_lists(sb.inter_idx.cpu().numpy(), sb.inter_cnt.cpu().numpy()),
+                           selection_lists(sb.intra_idx.cpu().numpy(), sb.intra_cnt.cpu().numpy()), None, None)
+    ref = oracle.hsa_step(x.Q, Kc, Vc, x.Kq, x.Vq, x.tau, x.z, x.E, x.F, selection=sel)
+    assert_close(st.out.cpu().numpy(), ref["out"], "hsa_forward out")
+
+
+def test_branches_standalone(small):
+    x, st = small.x, small.step
+    cfg = st.cfg
+    Kc, Vc = bits_of(st.Kc), bits_of(st.Vc)
+    o_s = torch.empty_like(st.out)
+    o_l = torch.empty_like(st.out)
+    hsa.hsa_sparse_attn(cfg, small.Q, st.Kc, st.Vc, small.Kq, small.Vq, st.selection, o_s, st.ws)
+    hsa.hsa_linear_attn(cfg, small.Q, st.Kc, st.Vc, small.Kq, small.Vq, small.E, small.F, o_l, st.ws)
+    torch.cuda.synchronize()
+    sb = st.selection
+    inter = selection_lists(sb.inter_idx.cpu().numpy(), sb.inter_cnt.cpu().numpy())
+    intra = selection_lists(sb.intra_idx.cpu().numpy(), sb.intra_cnt.cpu().numpy())
+    ref_s = oracle.sparse_attention(x.Q, Kc, Vc, x.Kq, x.Vq, inter, intra)
+    assert_close(o_s.cpu().numpy(), ref_s, "sparse branch")
+    EK, FV = oracle.linear_projection(x.E, x.F, Kc, x.Kq, Vc, x.Vq)
+    ref_l = oracle.linear_attention(x.Q, EK, FV)
+    assert_close(o_l.cpu().numpy(), ref_l, "linear branch")
+    # the gates isolate each branch exactly (same kernels, g = 1 or 0 in the merge)
+    H = small.shape.H
+    for z, want in ((float("inf"), o_s), (float("-inf"), o_l)):
+        zz = torch.full((H,), z, dtype=torch.float32, device="cuda")
+        out = torch.empty_like(st.out)
+        hsa.hsa_forward(cfg, small.Q, st.Kc, st.Vc, small.Kq, small.Vq, small.tau, zz, small.E, small.F, out, st.ws,
+                        st.kbar128)
+        torch.cuda.synchronize()
+        assert torch.equal(out, want), z
+
+
+def test_deterministic(small):
+    first = small.step.out.clone()
+    small.run()
+    torch.cuda.synchronize()
+    assert torch.equal(first, small.step.out)
+
+
+def test_bf16_output(small):
+    st = small.step
+    out = torch.empty(st.out.shape, dtype=torch.bfloat16, device="cuda")
+    hsa.hsa_forward(st.cfg, small.Q, st.Kc, st.Vc, small.Kq, small.Vq, small.tau, small.z, small.E, small.F, out,
+                    st.ws, st.kbar128)
+    torch.cuda.synchronize()
+    assert torch.equal(out, st.out.to(torch.bfloat16))
+
+
+# ----------------------------------------------------------------- invariants on the GPU path
+
+def _sdpa64(q, k, v, scale):
+    tq = torch.from_numpy(q).permute(1, 0, 2)
+    tk = torch.from_numpy(k).permute(1, 0, 2)
+    tv = torch.from_numpy(v).permute(1, 0, 2)
+    return torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, scale=scale).permute(1, 0, 2).numpy()
+
+
+def test_tau_one_is_dense_attention():
+    shape = SMALL[0]
+    ds = DeviceStep(shape, 5)
+    H = shape.H
+    ones = torch.ones(H, dtype=torch.float32, device="cuda")
+    inf = torch.full((H,), float("inf"), dtype=torch.float32, device="cuda")
+    out = ds.run(tau=ones, z=inf).cpu().numpy()
+    st = ds.step
+    assert np.all(st.selection.inter_cnt.cpu().numpy() == -(-st.Lc // 128))
+    K = np.concatenate([oracle.widen(bits_of(st.Kc)), oracle.widen(ds.x.Kq)])
+    V = np.concatenate([oracle.widen(bits_of(st.Vc)), oracle.widen(ds.x.Vq)])
+    ref = _sdpa64(oracle.widen(ds.x.Q), K, V, 1 / math.sqrt(shape.d))
+    assert_close(out, ref, "tau = 1 vs dense attention")
+
+
+def test_tau_zero_keeps_one_block_per_row():
+    shape = SMALL[0]
+    ds = DeviceStep(shape, 6)
+    zeros = torch.zeros(shape.H, dtype=torch.float32, device="cuda")
+    ds.run(tau=zeros)
+    torch.cuda.synchronize()
+    assert np.all(ds.step.selection.inter_cnt.cpu().numpy() == 1)
+    assert np.all(ds.step.selection.intra_cnt.cpu().numpy() == 1)
+
+
+def test_linear_identity_is_dense_attention():
+    H, d, Lq, Lc = 2, 128, 256, 256
+    L = Lq + Lc
+    x = synth.make_inputs(synth.StepShape("id", H=H, d=d, frames=1, F_tok=Lq, page_frames=1, page_tok=Lc,
+                                          NP=1, Kp=1, r=L), 9)
+    I = synth.f32_to_bf16(np.eye(L, dtype=np.float32))
+    cfg = make_config(H, d, Lq, Lc, L)
+    ws = hsa.workspace(cfg)
+    out = torch.empty(Lq, H, d, dtype=torch.float32, device="cuda")
+    Kc, Vc = to_dev(x.pages_k[0]), to_dev(x.pages_v[0])
+    hsa.hsa_linear_attn(cfg, to_dev(x.Q), Kc, Vc, to_dev(x.Kq), to_dev(x.Vq), to_dev(I), to_dev(I), out, ws)
+    torch.cuda.synchronize()
+    K = np.concatenate([oracle.widen(x.pages_k[0]), oracle.widen(x.Kq)])
+    V = np.concatenate([oracle.widen(x.pages_v[0]), oracle.widen(x.Vq)])
+    assert_close(out.cpu().numpy(), _sdpa64(oracle.widen(x.Q), K, V, 1 / math.sqrt(d)), "E = F = I")
+
+
+def test_per_head_projection_matrices():
+    shape = SMALL[1]
+    x = synth.make_inputs(shape, 12)
+    H, r, L = shape.H, shape.r, shape.L
+    E = synth.normal_bf16((H, r, L), 12, 901, sigma=1 / math.sqrt(r))
+    F = synth.normal_bf16((H, r, L), 12, 902, sigma=1 / math.sqrt(r))
+    Kc = oracle.gather_pages(x.pages_k, [0, 1])
+    Vc = oracle.gather_pages(x.pages_v, [0, 1])
+    cfg = make_config(H, shape.d, shape.Lq, shape.Lc, r)
+    ws = hsa.workspace(cfg)
+    out = torch.empty(shape.Lq, H, shape.d, dtype=torch.float32, device="cuda")
+    hsa.hsa_linear_attn(cfg, to_dev(x.Q), to_dev(Kc), to_dev(Vc), to_dev(x.Kq), to_dev(x.Vq), to_dev(E), to_dev(F),
+                        out, ws, ef_head_stride=r * L)
+    torch.cuda.synchronize()
+    EK, FV = oracle.linear_projection(E, F, Kc, x.Kq, Vc, x.Vq)
+    assert_close(out.cpu().numpy(), oracle.linear_attention(x.Q, EK, FV), "per-head E, F")
+
+
+@pytest.mark.parametrize("Lq,d,H", [(8, 64, 1), (64, 128, 2), (136, 128, 3)])
+def test_no_history(Lq, d, H):
+    """Lc = 0: no retrieved pages; the sparse branch runs over the chunk's own blocks."""
+    shape = synth.StepShape("nohist", H=H, d=d, frames=1, F_tok=Lq, page_frames=1, page_tok=8, NP=1, Kp=1, r=64)
+    x = synth.make_inputs(shape, 21)
+    E = x.E[:, shape.page_tok:].copy()  # columns of the chunk only
+    F = x.F[:, shape.page_tok:].copy()
+    cfg = make_config(H, d, Lq, 0, 64)
+    ws = hsa.workspace(cfg)
+    sel = SelectionBuffers.empty(cfg)
+    out = torch.empty(Lq, H, d, dtype=torch.float32, device="cuda")
+    hsa.hsa_forward(cfg, to_dev(x.Q), None, None, to_dev(x.Kq), to_dev(x.Vq), torch.from_numpy(x.tau).cuda(),
+                    torch.from_numpy(x.z).cuda(), to_dev(E), to_dev(F), out, ws, sel=sel)
+    torch.cuda.synchronize()
+    assert np.all(sel.inter_cnt.cpu().numpy() == 0)
+    empty = np.zeros((0, H, d), dtype=np.uint16)
+    ref = oracle.hsa_step(x.Q, empty, empty, x.Kq, x.Vq, x.tau, x.z, E, F)
+    gq = selection_lists(sel.intra_idx.cpu().numpy(), sel.intra_cnt.cpu().numpy())
+    check_selection(gq, ref["selection"].intra, ref["selection"].p_intra, x.tau, "intra")
+    ref = oracle.hsa_step(x.Q, empty, empty, x.Kq, x.Vq, x.tau, x.z, E, F,
+                          selection=oracle.Selection([[np.zeros(0, np.int64)] * -(-Lq // 128)] * H, gq, None, None))
+    assert_close(out.cpu().numpy(), ref["out"], "Lc = 0")
+
+
+# ----------------------------------------------------------------- device-side status and argument checks
+
+def test_device_status_short_candidate_range():
+    shape = SMALL[0]
+    ds = DeviceStep(shape, 3)
+    st = ds.step
+    hsa.hsa_status_clear(st.ws)
+    rng = torch.tensor([2, 3], dtype=torch.int32, device="cuda")  # one page < Kp = 3
+    hsa.hkv_select_pages(st.kbar_pages, ds.Q, shape.Kp, st.sel, st.ws, st.scores, rng)
+    assert hsa.hsa_status_read(st.ws) == 6  # HSA_ERR_DEVICE
+    assert np.all(st.sel.cpu().numpy() == -1)
+    hsa.hsa_status_clear(st.ws)
+    assert hsa.hsa_status_read(st.ws) == 0
+
+
+def test_device_status_bad_page_id():
+    shape = SMALL[0]
+    ds = DeviceStep(shape, 4)
+    st = ds.step
+    hsa.hsa_status_clear(st.ws)
+    bad = torch.tensor([0, 99, 1], dtype=torch.int32, device="cuda")
+    hsa.hkv_gather(st.page_k_ptrs, st.page_v_ptrs, bad, shape.Kp, shape.P_tok, shape.H, shape.d, st.Kc, st.Vc,
+                   st.ws, st.kbar128)
+    assert hsa.hsa_status_read(st.ws) == 6
+    # rows of valid slots were still copied
+    assert np.array_equal(bits_of(st.Kc)[:shape.P_tok], ds.x.pages_k[0])
+
+
+def test_invalid_arguments_launch_nothing():
+    cfg = make_config(2, 128, 256, 256, 64)
+    ws = hsa.workspace(cfg)
+    Q = torch.zeros(256, 2, 128, dtype=torch.bfloat16, device="cuda")
+    out = torch.zeros(256, 2, 128, dtype=torch.float32, device="cuda")
+    tau = torch.ones(2, device="cuda")
+    E = torch.zeros(64, 512, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(hsa.HsaError) as e:  # misaligned pointer
+        hsa.hsa_forward(cfg, Q[:, :, 1:], Q, Q, Q, Q, tau, tau, E, E, out, ws)
+    assert e.value.code == 1
+    with pytest.raises(hsa.HsaError) as e:  # workspace too small
+        hsa.hsa_forward(cfg, Q, Q, Q, Q, Q, tau, tau, E, E, out, ws[:1024])
+    assert e.value.code == 3
+    with pytest.raises(hsa.HsaError) as e:  # unsupported head dim
+        hsa.hsa_forward(make_config(2, 96, 256, 256, 64), Q, Q, Q, Q, Q, tau, tau, E, E, out, ws)
+    assert e.value.code == 2
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(out) == 0

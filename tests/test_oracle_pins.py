@@ -388,3 +388,16 @@ def test_biased_workload_retrieves_the_planted_pages():
             cand = range(int(x.seg_begin[s]), int(x.seg_begin[s + 1]))
         sel, _ = oracle.select_pages(kbar, x.Q, shape.Kp, cand)
         assert set(x.biased) <= set(sel.tolist()), (i, x.biased, sel)
+
+
+def test_no_history_reduces_to_chunk_attention():
+    """Lc = 0: the inter map is empty and, with tau = 1, the sparse branch is dense
+    attention over the chunk's own keys (library routine)."""
+    Q, _, _, Kq, Vq = _tiny(111, Lq=40, Lc=8, d=16)
+    H, d = Q.shape[1], Q.shape[2]
+    empty = np.zeros((0, H, d), dtype=np.uint16)
+    sel = oracle.block_select(Q, empty, Kq, np.ones(H), None, 16, 8, dtype=np.float64)
+    assert all(len(b) == 0 for rows in sel.inter for b in rows)
+    o = oracle.sparse_attention(Q, empty, empty, Kq, Vq, sel.inter, sel.intra, None, 16, 8)
+    ref = sdpa(oracle.widen(Q), oracle.widen(Kq), oracle.widen(Vq), 1 / math.sqrt(d))
+    np.testing.assert_allclose(o, ref, rtol=1e-11, atol=1e-12)
