@@ -1,0 +1,108 @@
+"""Host-side logic on CPU: the seeded generator, the workload table, and the
+multi-process (replica) plumbing of bench.py with gloo ranks (world size 2)."""
+import json
+import multiprocessing as mp
+import os
+import socket
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def test_generator_is_seeded_and_counter_based():
+    a = synth.normal_bf16((1000,), 7, 3)
+    b = synth.normal_bf16((1000,), 7, 3)
+    c = synth.normal_bf16((1000,), 8, 3)
+    assert np.array_equal(a, b) and not np.array_equal(a, c)
+    # any sub-range of a stream can be drawn on its own
+    tail = synth.normal_bf16((400,), 7, 3, start=600)
+    assert np.array_equal(tail, a[600:])
+    x = synth.bf16_to_f32(synth.normal_bf16((200000,), 1, 1))
+    assert abs(x.mean()) < 0.01 and abs(x.std() - 1) < 0.01
+
+
+def test_bf16_rounding_is_nearest_even():
+    v = np.array([1.0, 1.00390625, 1.01171875, -2.5, 3.0e-3], dtype=np.float32)  # halfway cases at 1+2^-8
+    bits = synth.f32_to_bf16(v)
+    back = synth.bf16_to_f32(bits)
+    assert back[0] == 1.0 and back[1] == 1.0 and back[2] == 1.015625 and back[3] == -2.5
+
+
+def test_workload_table():
+    s = synth.SHAPES
+    assert (s[0].H, s[0].d, s[0].Lq, s[0].P_tok, s[0].NP, s[0].Kp, s[0].r) == (2, 64, 256, 256, 8, 2, 64)
+    assert (s[1].H, s[1].Lq, s[1].P_tok, s[1].Lc, s[1].L, s[1].r) == (12, 4680, 12480, 49920, 54600, 256)
+    assert (s[2].H, s[2].Lq, s[2].Lc) == (40, 4680, 49920)
+    assert (s[3].H, s[3].Lq, s[3].P_tok, s[3].Lc, s[3].r, s[3].NP) == (40, 10800, 28800, 115200, 512, 12)
+    assert s[4].host_pages and s[4].NP == 48 and s[4].n_segments == 9
+    for sh in s:
+        assert sh.L % 8 == 0 and sh.r % 64 == 0
+    assert synth.segment_bounds(48, 9).tolist() == [0, 5, 10, 16, 21, 26, 32, 37, 42, 48]
+    t = synth.tau_schedule(12)
+    assert t[0] == 1.0 and abs(t[-1] - 0.35) < 1e-7 and np.all(np.diff(t) < 0)
+
+
+def test_biased_pages_and_segment_choice():
+    x = synth.make_inputs(synth.SHAPES[4].replace(F_tok=32, page_tok=0), 1004)
+    lo, hi = x.seg_begin[x.s_star], x.seg_begin[x.s_star + 1]
+    assert len(set(x.biased)) == 3 and all(lo <= c < hi for c in x.biased)
+    cos = x.e_seg @ x.e_cur / (np.linalg.norm(x.e_seg, axis=1) * np.linalg.norm(x.e_cur))
+    assert int(np.argmax(cos)) == x.s_star
+
+
+def _rank_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank), HSA_BENCH_BACKEND="gloo")
+    sys.path.insert(0, ROOT)
+    import torch.distributed as dist
+
+    import bench
+    r, w, _ = bench.dist_setup(world)
+    m = bench.max_over_ranks(10.0 * (r + 1), w)
+    bench.barrier(w)
+    q.put((r, w, m))
+    dist.destroy_process_group()
+
+
+def test_replica_timing_is_max_over_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = free_port()
+    procs = [ctx.Process(target=_rank_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert out == [(0, 2, 20.0), (1, 2, 20.0)]
+
+
+def test_reference_arm_two_ranks_prints_one_line():
+    """torchrun with 2 gloo ranks: rank 0 alone runs the oracle arm and prints one JSON line."""
+    port = free_port()
+    env = dict(os.environ, HSA_BENCH_BACKEND="gloo", OMP_NUM_THREADS="2")
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
+           "--impl", "reference", "--workload", "0", "--gpus", "2", "--steps", "1", "--warmup", "3"]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=600, env=env, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-3000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    res = json.loads(lines[0])
+    assert res["impl"] == "reference" and res["unit"] == "query-tokens/s" and res["value"] > 0
+    assert res["cpu_baseline"]["kind"] == "oracle" and res["e2e"]["h2d_bytes_per_step"] == 0
