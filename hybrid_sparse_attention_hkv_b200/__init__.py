@@ -22,7 +22,7 @@ HSA_STATUS = {0: "HSA_OK", 1: "HSA_ERR_INVALID_ARG", 2: "HSA_ERR_UNSUPPORTED", 3
 
 EXPORTED = [
     "hsa_status_string", "hsa_last_error_detail", "hsa_workspace_size", "hsa_status_clear", "hsa_status_read",
-    "hkv_page_summary", "hkv_select_prompt", "hkv_select_pages", "hkv_gather",
+    "hkv_page_summary", "hkv_select_prompt", "hkv_select_pages", "hkv_select_pages_noalloc", "hkv_gather",
     "hsa_block_select", "hsa_sparse_attn", "hsa_linear_attn", "hsa_forward",
     "hsa_trace_begin", "hsa_trace_count", "hsa_trace_end",
 ]
@@ -67,6 +67,7 @@ def load_library(path: str = LIB_PATH):
         "hkv_page_summary": (I, [P, I, I, I, P, P, S, P]),
         "hkv_select_prompt": (I, [P, P, I, I, P, P, P, P]),
         "hkv_select_pages": (I, [P, I, P, P, I, I, I, I, P, P, P, S, P]),
+        "hkv_select_pages_noalloc": (I, [P, I, P, P, I, I, I, I, P, P, P, P]),
         "hkv_gather": (I, [P, P, I, P, I, I, I, I, P, P, P, P, S, P]),
         "hsa_block_select": (I, [CP, P, P, P, P, P, _Selection, P, S, P]),
         "hsa_sparse_attn": (I, [CP, P, P, P, P, P, _Selection, P, P, S, P]),
@@ -164,6 +165,16 @@ def hkv_select_pages(kbar_pages, Q, Kp, sel_out, ws, scores_out=None, cand_range
     Lq, H, d = Q.shape
     _check(load_library().hkv_select_pages(_p(kbar_pages), NP, _p(cand_range), _p(Q), Lq, H, d, Kp, _p(sel_out),
                                            _p(scores_out), _p(ws), ws.numel(), _stream(stream)), "hkv_select_pages")
+
+
+def hkv_select_pages_noalloc(kbar_pages, Q, Kp, sel_out, scores_out=None, cand_range=None, status_out=None,
+                             stream=None):
+    """hkv_select_pages without a workspace (scratch in a static device array)."""
+    NP = kbar_pages.shape[0]
+    Lq, H, d = Q.shape
+    _check(load_library().hkv_select_pages_noalloc(_p(kbar_pages), NP, _p(cand_range), _p(Q), Lq, H, d, Kp,
+                                                   _p(sel_out), _p(scores_out), _p(status_out), _stream(stream)),
+           "hkv_select_pages_noalloc")
 
 
 def hkv_gather(page_k_ptrs, page_v_ptrs, sel, Kp, P_tok, H, d, Kc, Vc, ws, kbar128=None, stream=None):

@@ -164,6 +164,16 @@ hsa_status_t check_sel(const char* fn, const hsa_selection_t& s) {
 
 }  // namespace
 
+namespace hsa {
+hsa_status_t api_fail(hsa_status_t code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_detail, sizeof(t_detail), fmt, ap);
+  va_end(ap);
+  return code;
+}
+}  // namespace hsa
+
 extern "C" {
 
 const char* hsa_status_string(hsa_status_t s) {

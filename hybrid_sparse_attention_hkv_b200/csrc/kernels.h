@@ -5,7 +5,13 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/hsa.h"
+
 namespace hsa {
+
+// ---------------------------------------------------------------- api.cu
+// Record the text returned by hsa_last_error_detail() and return `code`.
+hsa_status_t api_fail(hsa_status_t code, const char* fmt, ...);
 
 // ---------------------------------------------------------------- hkv.cu
 constexpr int kColMaxSplits = 296;  // 2 CTAs per SM for the column-sum partial pass

@@ -152,6 +152,28 @@ hsa_status_t hkv_gather(const hsa_bf16* const* page_k, const hsa_bf16* const* pa
                         hsa_bf16* Kc, hsa_bf16* Vc, float* kbar128,
                         void* ws, size_t ws_bytes, hsa_stream_t stream);
 
+/* Allocation-free variant of hkv_select_pages.  The paper has no counterpart:
+ * this exists for callers that may not allocate device memory at all -- a host
+ * framework that owns every device buffer and passes a plugin only the tensors
+ * of the call, a runtime whose memory plan is fixed before it serves, or a loop
+ * where an allocation could stall the device -- and so cannot provide the
+ * workspace hkv_select_pages uses for its column-sum partials.
+ * Same inputs, outputs and results as hkv_select_pages; the scratch lives in a
+ * static device array of 8 MiB inside the library (held by every GPU that loads
+ * the library until the process exits), so 256 + 296 * H * d * 4 bytes must fit:
+ * H * d <= 7084, else HSA_ERR_UNSUPPORTED.  Calls no allocator.
+ * status_out: optional device int32 that receives the device status
+ * (HSA_ERR_DEVICE for a candidate range shorter than Kp); cleared by the call.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it: make that
+ * first call before any stream capture.  Every call on a device shares the
+ * array: calls whose kernels could overlap on the GPU race and must be ordered
+ * (one stream, or events). */
+hsa_status_t hkv_select_pages_noalloc(const float* kbar_pages, int NP, const int32_t* cand_range,
+                                      const hsa_bf16* Q, int Lq, int H, int d, int Kp,
+                                      int32_t* sel_out, float* scores_out, int32_t* status_out,
+                                      hsa_stream_t stream);
+
 /* ---------------------------------------------------------------- HSA ---- */
 
 /* Head-adaptive block selection ([NEWS] HSA paragraph).  Pools Q and Kc into
