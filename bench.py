@@ -32,7 +32,13 @@ DEFAULT_WORKLOAD = 1
 
 # DRAM traffic per launch from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
 # keyed by kernel, valid only while the kernel's source file is unchanged (sha256 prefix).
-TRAFFIC = {}
+TRAFFIC = {
+    # profiles/sparse_attn_mma_sync_wan1.3b_480p.md
+    "sparse_attn_merge": {"file": "attn.cu", "sha": "32b35d7d723278fc", "bytes": 306676480 + 18457856},
+    # profiles/gather_and_projection_hbm_wan1.3b_480p.md
+    "gather": {"file": "hkv.cu", "sha": "577b859a6a30a103", "bytes": 306822656 + 249974016},
+    "linformer_proj": {"file": "proj.cu", "sha": "2f89ba706af1053b", "bytes": 395510016 + 25282816},
+}
 
 
 def _sha(path):
@@ -87,7 +93,7 @@ def exact_pairs(shape, sel_bufs):
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    """nvidia-smi clock / throttle-reason samples; mark() brackets the timed region."""
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -96,33 +102,46 @@ class ClockSampler:
         self.index = index
         self.proc = None
         self.lines = []
+        self.err = ""
+        self.marks = []
 
-    def start(self):
+    def start(self, wait_s=5.0):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-        except (OSError, FileNotFoundError):
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
+        except OSError as e:
+            self.err = str(e)
             self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+        t0 = time.time()
+        while not self.lines and time.time() - t0 < wait_s and self.proc.poll() is None:
+            time.sleep(0.02)
 
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
+    def mark(self):
+        self.marks.append(len(self.lines))
+
     def stop(self):
         if not self.proc:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [f"nvidia-smi unavailable: {self.err}"]}
         self.proc.terminate()
         try:
-            self.proc.wait(timeout=5)
+            _, err = self.proc.communicate(timeout=5)
+            self.err = (err or "").strip()[:200]
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.t.join(timeout=2)
+        lo, hi = (self.marks + [0, len(self.lines)])[:2] if len(self.marks) >= 2 else (0, len(self.lines))
+        window = self.lines[lo:max(hi, lo + 1)] or self.lines[-1:]
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in window:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
@@ -134,8 +153,11 @@ class ClockSampler:
             for n, v in zip(names, f[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        out = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+               "samples": len(sm)}
+        if not sm and self.err:
+            out["error"] = self.err
+        return out
 
 
 # ------------------------------------------------------------------ CPU oracle timing
@@ -146,34 +168,32 @@ def oracle_summaries(x, shape):
     return np.stack([oracle.page_summary(x.pages_k[p], np.float32) for p in range(shape.NP)])
 
 
-def oracle_step_sample(x, shape, kbar, rows_per_step=256, head=None):
-    """Time the fp64 oracle on a bounded sample of one step and extrapolate to the full step:
-    t_step = t_retrieval + H * (t_head_fixed + t_rows * Lq / rows)."""
+def oracle_step_sample(x, shape, kbar, heads=None, rows_per_step=None):
+    """Time the fp64 oracle on one step, or on a bounded sample of it: page retrieval +
+    gather, then the HSA of the given heads on the given number of query rows; the
+    step time is extrapolated as t_retrieval + H/len(heads) * t_heads * Lq/rows."""
     import numpy as np
     import oracle
-    h = shape.H // 2 if head is None else head
+    heads = list(range(shape.H)) if heads is None else list(heads)
+    nrows = shape.Lq if rows_per_step is None else min(rows_per_step, shape.Lq)
+    rows = None if nrows == shape.Lq else np.linspace(0, shape.Lq - 1, nrows).astype(np.int64)
     t0 = time.perf_counter()
     sel, _ = oracle.select_pages(kbar, x.Q, shape.Kp)
     Kc = oracle.gather_pages(x.pages_k, sel)
     Vc = oracle.gather_pages(x.pages_v, sel)
     t_r = time.perf_counter() - t0
-    sl = slice(h, h + 1)
-    Qh, Kch, Vch, Kqh, Vqh = x.Q[:, sl], Kc[:, sl], Vc[:, sl], x.Kq[:, sl], x.Vq[:, sl]
     t0 = time.perf_counter()
-    selh = oracle.block_select(Qh, Kch, Kqh, x.tau[sl])
-    EK, FV = oracle.linear_projection(x.E, x.F, Kch, Kqh, Vch, Vqh)
-    t_fixed = time.perf_counter() - t0
-    rows = np.linspace(0, shape.Lq - 1, rows_per_step).astype(np.int64)
-    t0 = time.perf_counter()
-    o_s = oracle.sparse_attention(Qh, Kch, Vch, Kqh, Vqh, selh.inter, selh.intra, rows=rows)
-    o_l = oracle.linear_attention(Qh, EK, FV, rows=rows)
-    oracle.gated_merge(o_s, o_l, x.z[sl])
-    t_rows = time.perf_counter() - t0
-    t_step = t_r + shape.H * (t_fixed + t_rows * shape.Lq / len(rows))
-    sample = (f"page retrieval + gather once, then head {h} (tau {float(x.tau[h]):.2f}) alone: block selection, "
-              f"Linformer projection, both branches and merge on {len(rows)} of {shape.Lq} query rows; "
-              f"step time extrapolated as t_retrieval + H*(t_head + t_rows*Lq/rows)")
-    return t_step, sample, t_r + t_fixed + t_rows
+    hs = np.array(heads)
+    oracle.hsa_step(x.Q[:, hs], Kc[:, hs], Vc[:, hs], x.Kq[:, hs], x.Vq[:, hs], x.tau[hs], x.z[hs], x.E, x.F,
+                    rows=rows)
+    t_h = time.perf_counter() - t0
+    t_step = t_r + t_h * (shape.H / len(heads)) * (shape.Lq / nrows)
+    if len(heads) == shape.H and nrows == shape.Lq:
+        sample = "the whole step: page retrieval, gather, block selection, both branches and merge, all heads and rows"
+    else:
+        sample = (f"page retrieval + gather, then HSA of heads {heads} on {nrows} of {shape.Lq} query rows; step time "
+                  f"extrapolated as t_retrieval + (H/heads) * t_heads * (Lq/rows)")
+    return t_step, sample, t_r + t_h
 
 
 def blas_threads():
@@ -236,12 +256,13 @@ def run_reference(args, shape, rank, world):
     import synth
     x = synth.make_inputs(shape, synth.seed_of(args.workload))
     kbar = oracle_summaries(x, shape)
-    for _ in range(args.warmup):
-        oracle_step_sample(x, shape, kbar, rows_per_step=64)
+    # each step: one head (rotating), all query rows, so that --steps K stays within minutes
+    for k in range(args.warmup):
+        oracle_step_sample(x, shape, kbar, heads=[k % shape.H])
     ts = []
     sample = ""
-    for _ in range(args.steps):
-        t, sample, _ = oracle_step_sample(x, shape, kbar, rows_per_step=64)
+    for k in range(args.steps):
+        t, sample, _ = oracle_step_sample(x, shape, kbar, heads=[k % shape.H])
         ts.append(t)
     t_step = statistics.mean(ts)
     value = shape.Lq / t_step
@@ -293,9 +314,10 @@ def run_gpu(args, shape, rank, world, local):
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     clocks = ClockSampler(local)
+    clocks.start()
     barrier(world)
     torch.cuda.synchronize()
-    clocks.start()
+    clocks.mark()
     with trace:
         for k in range(args.steps):
             flush.zero_()
@@ -303,6 +325,7 @@ def run_gpu(args, shape, rank, world, local):
             one_step()
             ends[k].record(stream)
     torch.cuda.synchronize()
+    clocks.mark()
     clk = clocks.stop()
     barrier(world)
     t_steps = [s.elapsed_time(e) for s, e in zip(starts, ends)]
@@ -408,7 +431,7 @@ def run_gpu(args, shape, rank, world, local):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD)
