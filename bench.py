@@ -31,19 +31,29 @@ UNIT = "query-tokens/s"
 DEFAULT_WORKLOAD = 1
 
 # DRAM traffic per launch from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
-# keyed by kernel, valid only while the kernel's source file is unchanged (sha256 prefix).
+# keyed by kernel; valid only while that kernel's section of its source file (from its
+# section marker to the next one) is unchanged (sha256 prefix of the section).
 TRAFFIC = {
     # profiles/sparse_attn_mma_sync_wan1.3b_480p.md
-    "sparse_attn_merge": {"file": "attn.cu", "sha": "32b35d7d723278fc", "bytes": 306676480 + 18457856},
+    "attention_merge": {"file": "attn_tc.cu", "sha": "none yet", "bytes": None},
     # profiles/gather_and_projection_hbm_wan1.3b_480p.md
     "gather": {"file": "hkv.cu", "sha": "577b859a6a30a103", "bytes": 306822656 + 249974016},
     "linformer_proj": {"file": "proj.cu", "sha": "2f89ba706af1053b", "bytes": 395510016 + 25282816},
 }
 
 
-def _sha(path):
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+SECTION_MARK = "// ------------------------------------------------------------------ "
+
+
+def section_sha(path, section):
+    """sha256 prefix of the text from the `section` marker line to the next marker (or the end)."""
+    with open(path) as f:
+        text = f.read()
+    start = text.find(SECTION_MARK + section)
+    if start < 0:
+        return None
+    nxt = text.find(SECTION_MARK, start + len(SECTION_MARK))
+    return hashlib.sha256(text[start:nxt if nxt >= 0 else len(text)].encode()).hexdigest()[:16]
 
 
 def load_peaks():
@@ -256,13 +266,15 @@ def run_reference(args, shape, rank, world):
     import synth
     x = synth.make_inputs(shape, synth.seed_of(args.workload))
     kbar = oracle_summaries(x, shape)
-    # each step: one head (rotating), all query rows, so that --steps K stays within minutes
+    # each step: one head (rotating) on a row sample sized so that K + W steps stay
+    # within a few minutes (all rows for up to ~50 steps, fewer rows beyond)
+    rows = max(64, shape.Lq // max(1, (args.steps + args.warmup) // 50))
     for k in range(args.warmup):
-        oracle_step_sample(x, shape, kbar, heads=[k % shape.H])
+        oracle_step_sample(x, shape, kbar, heads=[k % shape.H], rows_per_step=rows)
     ts = []
     sample = ""
     for k in range(args.steps):
-        t, sample, _ = oracle_step_sample(x, shape, kbar, heads=[k % shape.H])
+        t, sample, _ = oracle_step_sample(x, shape, kbar, heads=[k % shape.H], rows_per_step=rows)
         ts.append(t)
     t_step = statistics.mean(ts)
     value = shape.Lq / t_step
@@ -372,8 +384,9 @@ def run_gpu(args, shape, rank, world, local):
     f_total = f_sparse + w["proj_flops"] + w["lin_attn_flops"]
     eff_tflops = f_total / (ms_per_step / 1e3) / 1e12
     kernel_work = {
-        "sparse_attn_merge": ("tensor", f_sparse),
-        "linear_attn": ("tensor", w["lin_attn_flops"]),
+        # the fused attention kernel: selected-block FLOPs of the sparse branch plus the
+        # useful FLOPs of the linear branch (the split-precision extra products not counted)
+        "attention_merge": ("tensor", f_sparse + w["lin_attn_flops"]),
         "linformer_proj": ("tensor", w["proj_flops"]),
         "gather": ("hbm", w["gather_bytes"]),
         "pool": ("hbm", w["pool_bytes"]),
@@ -400,7 +413,8 @@ def run_gpu(args, shape, rank, world, local):
     peak = peaks["bf16_tflops_sustained"] if bound == "tensor" else peaks["hbm_gbs"]
     traffic = None
     tr = TRAFFIC.get(dom)
-    if tr and tr["sha"] == _sha(os.path.join(ROOT, "hybrid_sparse_attention_hkv_b200", "csrc", tr["file"])):
+    if tr and tr["sha"] == section_sha(os.path.join(ROOT, "hybrid_sparse_attention_hkv_b200", "csrc", tr["file"]),
+                                       tr["section"]):
         traffic = tr["bytes"]
     roofline = {"kernel": dom, "bound": bound, "achieved": de.get("achieved"), "peak": peak,
                 "unit": "TFLOP/s" if bound == "tensor" else "GB/s", "frac": de.get("frac"), "traffic": traffic,

@@ -70,7 +70,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 struct Layout {
   size_t status = 0, colpart = 0, q128 = 0, q64 = 0, kq64 = 0, kc128 = 0;
   size_t inter_idx = 0, inter_cnt = 0, intra_idx = 0, intra_cnt = 0;
-  size_t olin = 0, ekhi = 0, eklo = 0, fvhi = 0, fvlo = 0, projpart = 0;
+  size_t ekhi = 0, eklo = 0, fvhi = 0, fvlo = 0, projpart = 0;
   size_t pages_end = 0;  // bytes needed by the page (HKV) calls
   size_t total = 0;
   int splits = 0;
@@ -96,13 +96,12 @@ Layout make_layout(int H, int d, int Lq, long long Lc, int r) {
   L.inter_cnt = take((size_t)H * nQ128 * 4);
   L.intra_idx = take((size_t)H * nQ64 * nQ64 * 4);
   L.intra_cnt = take((size_t)H * nQ64 * 4);
-  L.olin = take((size_t)Lq * hd * 4);
   const size_t hrd = (size_t)H * r * d;
   L.ekhi = take(hrd * 2);
   L.eklo = take(hrd * 2);
   L.fvhi = take(hrd * 2);
   L.fvlo = take(hrd * 2);
-  L.splits = r > 0 ? hsa::proj_splits(H, r, Lc + Lq) : 0;
+  L.splits = r > 0 ? hsa::proj_tc_splits(H, r, Lc, Lq) : 0;
   L.projpart = take((size_t)L.splits * 2 * hrd * 4);
   L.total = off;
   return L;
@@ -129,8 +128,8 @@ hsa_status_t check_cfg(const char* fn, const hsa_config_t* c, bool need_rank) {
   if (c->Lc < 0) return fail(HSA_ERR_INVALID_ARG, "%s: Lc = %d must be >= 0", fn, c->Lc);
   if (c->block_inter != 128 || c->block_intra != 64)
     return fail(HSA_ERR_UNSUPPORTED, "%s: block sizes %d/%d (supported: 128/64)", fn, c->block_inter, c->block_intra);
-  if (((long long)c->Lc + c->Lq) % 8 != 0)
-    return fail(HSA_ERR_UNSUPPORTED, "%s: Lc + Lq = %lld must be a multiple of 8", fn, (long long)c->Lc + c->Lq);
+  if (c->Lc % 8 != 0 || c->Lq % 8 != 0)
+    return fail(HSA_ERR_UNSUPPORTED, "%s: Lc = %d and Lq = %d must be multiples of 8", fn, c->Lc, c->Lq);
   if ((c->Lc + 127) / 128 > hsa::kMaxSelBlocks || (c->Lq + 63) / 64 > hsa::kMaxSelBlocks)
     return fail(HSA_ERR_UNSUPPORTED, "%s: more than %d blocks in a selection row", fn, hsa::kMaxSelBlocks);
   if (!(c->scale >= 0.f) || isinf(c->scale)) return fail(HSA_ERR_INVALID_ARG, "%s: scale must be finite and >= 0", fn);
@@ -265,8 +264,8 @@ hsa_status_t hkv_select_pages(const float* kbar_pages, int NP, const int32_t* ca
   TRY(check_heads(fn, H, d));
   if (NP < 1 || Lq < 1) return fail(HSA_ERR_INVALID_ARG, "%s: NP = %d, Lq = %d must be >= 1", fn, NP, Lq);
   if (Kp < 1 || Kp > NP || Kp > 64) return fail(HSA_ERR_INVALID_ARG, "%s: Kp = %d must be in [1, min(NP, 64)]", fn, Kp);
-  if ((size_t)H * d * 4 + (size_t)NP * 8 > 200 * 1024)
-    return fail(HSA_ERR_UNSUPPORTED, "%s: H*d*4 + NP*8 bytes exceed the shared-memory budget", fn);
+  if ((size_t)H * d * 8 + (size_t)NP * 8 > 200 * 1024)
+    return fail(HSA_ERR_UNSUPPORTED, "%s: H*d*8 + NP*8 bytes exceed the shared-memory budget", fn);
   REQUIRE_PTR(kbar_pages);
   REQUIRE_PTR(Q);
   if (!sel_out) return fail(HSA_ERR_INVALID_ARG, "%s: sel_out is NULL", fn);
@@ -325,23 +324,21 @@ static hsa::AttnArgs attn_args(const hsa_config_t* cfg, const hsa_bf16* Q, const
   return a;
 }
 
-static hsa_status_t run_linear(const hsa_config_t* cfg, const Layout& L, const hsa_bf16* Q, const hsa_bf16* Kc,
-                               const hsa_bf16* Vc, const hsa_bf16* Kq, const hsa_bf16* Vq, const hsa_bf16* E,
-                               const hsa_bf16* F, long long ef_head_stride, float* o_lin, void* ws,
-                               hsa_stream_t stream) {
+// Linformer projection (EK, FV as split-bf16 pairs in the workspace); sets the
+// linear-branch fields of `a`.
+static hsa_status_t run_projection(const hsa_config_t* cfg, const Layout& L, const hsa_bf16* Kc, const hsa_bf16* Vc,
+                                   const hsa_bf16* Kq, const hsa_bf16* Vq, const hsa_bf16* E, const hsa_bf16* F,
+                                   long long ef_head_stride, void* ws, hsa::AttnArgs& a, hsa_stream_t stream) {
   float* part = at<float>(ws, L.projpart);
   uint16_t* ekhi = at<uint16_t>(ws, L.ekhi);
   uint16_t* eklo = at<uint16_t>(ws, L.eklo);
   uint16_t* fvhi = at<uint16_t>(ws, L.fvhi);
   uint16_t* fvlo = at<uint16_t>(ws, L.fvlo);
-  HSA_LAUNCH("linformer_proj", hsa::launch_proj(E, F, ef_head_stride, Kc, Kq, Vc, Vq, cfg->H, cfg->d, cfg->rank,
-                                                cfg->Lc, cfg->Lq, L.splits, part, stream));
+  HSA_LAUNCH("linformer_proj", hsa::launch_proj_tc(E, F, ef_head_stride, Kc, Kq, Vc, Vq, cfg->H, cfg->d, cfg->rank,
+                                                   cfg->Lc, cfg->Lq, L.splits, part, status_of(ws), stream));
   HSA_LAUNCH("linformer_reduce", hsa::launch_proj_reduce(part, L.splits, cfg->H, cfg->d, cfg->rank, ekhi, eklo, fvhi,
                                                          fvlo, stream));
-  hsa::AttnArgs a = attn_args(cfg, Q, Kc, Vc, Kq, Vq);
   a.EKhi = ekhi; a.EKlo = eklo; a.FVhi = fvhi; a.FVlo = fvlo;
-  a.out_f32 = o_lin;
-  HSA_LAUNCH("linear_attn", hsa::launch_linear_attn(a, stream));
   return HSA_OK;
 }
 
@@ -385,7 +382,7 @@ hsa_status_t hsa_sparse_attn(const hsa_config_t* cfg, const hsa_bf16* Q, const h
   a.inter_idx = sel.inter_idx; a.inter_cnt = sel.inter_cnt; a.intra_idx = sel.intra_idx; a.intra_cnt = sel.intra_cnt;
   a.out_f32 = o_sparse;
   a.status = ws ? status_of(ws) : nullptr;
-  HSA_LAUNCH("sparse_attn", hsa::launch_sparse_attn(a, stream));
+  HSA_LAUNCH("attention", hsa::launch_attn_tc(a, stream));
   return HSA_OK;
 }
 
@@ -399,11 +396,16 @@ hsa_status_t hsa_linear_attn(const hsa_config_t* cfg, const hsa_bf16* Q, const h
   REQUIRE_PTR(E);
   REQUIRE_PTR(F);
   REQUIRE_PTR(o_linear);
-  if (ef_head_stride < 0 || ef_head_stride % 8 != 0)
-    return fail(HSA_ERR_INVALID_ARG, "%s: ef_head_stride must be >= 0 and a multiple of 8", fn);
+  if (ef_head_stride != 0 && ef_head_stride != (long long)cfg->rank * (cfg->Lc + cfg->Lq))
+    return fail(HSA_ERR_UNSUPPORTED, "%s: ef_head_stride must be 0 (shared) or r * (Lc + Lq) (stacked per head)", fn);
   const Layout L = make_layout(cfg->H, cfg->d, cfg->Lq, cfg->Lc, cfg->rank);
   TRY(check_ws(fn, ws, ws_bytes, L.total));
-  return run_linear(cfg, L, Q, Kc, Vc, Kq, Vq, E, F, ef_head_stride, o_linear, ws, stream);
+  hsa::AttnArgs a = attn_args(cfg, Q, Kc, Vc, Kq, Vq);
+  TRY(run_projection(cfg, L, Kc, Vc, Kq, Vq, E, F, ef_head_stride, ws, a, stream));
+  a.out_f32 = o_linear;
+  a.status = status_of(ws);
+  HSA_LAUNCH("attention", hsa::launch_attn_tc(a, stream));
+  return HSA_OK;
 }
 
 hsa_status_t hsa_forward(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc, const hsa_bf16* Vc,
@@ -419,8 +421,8 @@ hsa_status_t hsa_forward(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_b
   REQUIRE_PTR(E);
   REQUIRE_PTR(F);
   REQUIRE_PTR(out);
-  if (ef_head_stride < 0 || ef_head_stride % 8 != 0)
-    return fail(HSA_ERR_INVALID_ARG, "%s: ef_head_stride must be >= 0 and a multiple of 8", fn);
+  if (ef_head_stride != 0 && ef_head_stride != (long long)cfg->rank * (cfg->Lc + cfg->Lq))
+    return fail(HSA_ERR_UNSUPPORTED, "%s: ef_head_stride must be 0 (shared) or r * (Lc + Lq) (stacked per head)", fn);
   if (sel_out) TRY(check_sel(fn, *sel_out));
   const Layout L = make_layout(cfg->H, cfg->d, cfg->Lq, cfg->Lc, cfg->rank);
   TRY(check_ws(fn, ws, ws_bytes, L.total));
@@ -435,17 +437,14 @@ hsa_status_t hsa_forward(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_b
     sel.intra_cnt = at<int32_t>(ws, L.intra_cnt);
   }
   TRY(run_block_select(cfg, L, Q, Kc, Kq, kbar128, tau, sel, ws, stream));
-  // linear branch first: its output is the merge input of the sparse kernel
-  float* o_lin = out_is_bf16 ? at<float>(ws, L.olin) : static_cast<float*>(out);
-  TRY(run_linear(cfg, L, Q, Kc, Vc, Kq, Vq, E, F, ef_head_stride, o_lin, ws, stream));
   hsa::AttnArgs a = attn_args(cfg, Q, Kc, Vc, Kq, Vq);
+  TRY(run_projection(cfg, L, Kc, Vc, Kq, Vq, E, F, ef_head_stride, ws, a, stream));
   a.inter_idx = sel.inter_idx; a.inter_cnt = sel.inter_cnt; a.intra_idx = sel.intra_idx; a.intra_cnt = sel.intra_cnt;
-  a.o_lin = o_lin;
   a.gate_logit = gate_logit;
   a.status = status_of(ws);
   if (out_is_bf16) a.out_bf16 = static_cast<uint16_t*>(out);
   else a.out_f32 = static_cast<float*>(out);
-  HSA_LAUNCH("sparse_attn_merge", hsa::launch_sparse_attn(a, stream));
+  HSA_LAUNCH("attention_merge", hsa::launch_attn_tc(a, stream));
   return HSA_OK;
 }
 

@@ -1,0 +1,594 @@
+// HSA attention on the 5th-generation tensor cores (tcgen05 + TMEM + TMA): the
+// block-sparse branch, the Linformer branch and their gated merge in one kernel
+// ("WorldAttention pairs hierarchical KV caching with hybrid sparse attention..."
+// news summary, HSA paragraph: exact attention over each head's kept blocks, a
+// low-rank linear global branch, learned gates merging the two).
+//
+// One CTA per (head, 128-query tile).  Its key tiles, in order:
+//   linear tiles  64 rows of EK / FV (split bf16 hi + lo), r / 64 of them;
+//   cached tiles  one 128-row tile per kept inter block of the cached KV;
+//   chunk tiles   the union of the two 64-query halves' kept 64-row intra blocks,
+//                 each tagged with the halves that use it.
+// 7 warps:
+//   warp 0      TMA producer of the Q tile (once) and of each key tile's K part
+//               (K, or EK_hi + EK_lo) into a 3-slot ring of 128-byte-swizzled
+//               buffers (a slot frees when its S MMA ends);
+//   warp 6      TMA producer of the V parts (V, or FV_hi + FV_lo) into a 2-slot
+//               ring (a slot frees when its P.V MMA ends);
+//   warp 1      MMA issuer (lane 0): S_j = Q K_j^T (+ Q EK_lo^T) into one of two
+//               TMEM S buffers, then O += P_j V_j with P_j read from TMEM (written
+//               over S_j; for linear tiles P_hi FV_hi + P_lo FV_hi + P_hi FV_lo
+//               into a second accumulator O_l);
+//   warps 2-5   softmax, one TMEM lane (= query row) per thread, one running
+//               max / sum per branch: exp2, row sums, P as packed bf16 back into
+//               TMEM; the running max is raised (and that O rescaled in TMEM) only
+//               when it grows by more than 2^8; finally o_s = O_s / l_s,
+//               o_l = O_l / l_l, out = g o_s + (1 - g) o_l, stored.
+// The tensor core computes S_{j+1} while the softmax warps work on S_j.
+// Every wait is bounded (HSA_ERR_TIMEOUT in the workspace status on expiry).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace hsa {
+using namespace sm100;
+
+namespace {
+
+constexpr int kTcThreads = 224;  // 7 warps
+constexpr int kKStages = 3;      // K ring: a slot frees as soon as its S MMA completes
+constexpr int kVStages = 2;      // V ring: a slot frees when its P.V MMA completes
+constexpr int kRegionBytes = 128 * 128;  // one [128 rows x 64 bf16] swizzled region
+
+struct TcMaps {
+  CUtensorMap q, kc, vc, kq, vq, ekhi, eklo, fvhi, fvlo;
+};
+
+// Key-tile code: (first row << 4) | (type << 2) | half-mask.
+constexpr int kTileCached = 0;  // 128 rows of Kc / Vc
+constexpr int kTileChunk = 1;   // 64 rows of Kq / Vq
+constexpr int kTileLinear = 2;  // 64 rows of EK / FV (hi + lo)
+
+template <int D>
+struct TcLayout {
+  static constexpr int kQBytes = (D / 64) * kRegionBytes;
+  static constexpr int kKVBytes = (D / 64) * kRegionBytes;  // one 128-row K or V tile
+  static constexpr int kBytes = kQBytes + (kKStages + kVStages) * kKVBytes;
+};
+
+__device__ __forceinline__ int tc_tile_code(long long start, int type, int mask) {
+  return (int)(start << 4) | (type << 2) | mask;
+}
+__device__ __forceinline__ int tile_type(int code) { return (code >> 2) & 3; }
+__device__ __forceinline__ int tile_start(int code) { return code >> 4; }
+__device__ __forceinline__ int tile_rows(int code) { return tile_type(code) == kTileCached ? 128 : 64; }
+
+// ------------------------------------------------------------------ kernel
+// Online-softmax step of one query row over one key tile of ROWS columns held in
+// sr[] (raw scores): update the running max m (raised only when it grows by more
+// than 2^8, returning the factor alpha for O), write P = 2^(s*sl2 - m) as packed
+// bf16 pairs over the first ROWS/2 columns of the S buffer, and fold the row sum
+// into l.  MASKED: only the first `valid` keys exist.
+template <int ROWS, bool MASKED>
+__device__ __forceinline__ void softmax_tile(const uint32_t (&sr)[128], int valid, float sl2, float& m, float& l,
+                                             float& alpha, bool& rescale, uint32_t tS) {
+  float pm[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) pm[q] = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < ROWS; ++k)
+    if (!MASKED || k < valid) pm[k & 7] = fmaxf(pm[k & 7], __uint_as_float(sr[k]));
+  const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+  const float mn = mx * sl2;
+  if (mn > m + 8.f) {
+    if (m != -INFINITY) {
+      alpha = ex2_approx(m - mn);
+      rescale = true;
+    }
+    m = mn;
+  }
+  const float2 a2 = make_float2(sl2, sl2), b2 = make_float2(-m, -m);
+  float2 acc[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int c = 0; c < ROWS / 32; ++c) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int i = c * 32 + 2 * k;
+      const float2 t = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), a2, b2);
+      float p0, p1;
+      if (!MASKED && (k & 3) == 3) {  // every 4th pair on the FMA pipe, the rest on the SFU
+        const float2 e = ex2_poly2(t);
+        p0 = e.x;
+        p1 = e.y;
+      } else {
+        p0 = ex2_approx(t.x);
+        p1 = ex2_approx(t.y);
+      }
+      if (MASKED) {
+        if (i >= valid) p0 = 0.f;
+        if (i + 1 >= valid) p1 = 0.f;
+      }
+      acc[k & 3] = __fadd2_rn(acc[k & 3], make_float2(p0, p1));
+      pk[k] = pack_bf16x2(p0, p1);
+    }
+    tmem_st16(tS + c * 16, pk);  // P (bf16 pairs) over the first half of S
+  }
+  const float2 s01 = __fadd2_rn(acc[0], acc[1]), s23 = __fadd2_rn(acc[2], acc[3]);
+  const float2 st = __fadd2_rn(s01, s23);
+  l = l * alpha + (st.x + st.y);
+}
+
+// Linear-branch variant over 64 projected rows (no masking): P is written as two
+// bf16 parts, hi = bf16(p) over columns [0, 32) and lo = bf16(p - hi) over
+// [32, 64) of the S buffer, so that P.FV keeps about 16 significant bits.
+__device__ __forceinline__ void softmax_tile_split(const uint32_t (&sr)[64], float sl2, float& m, float& l,
+                                                   float& alpha, bool& rescale, uint32_t tS) {
+  float pm[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) pm[q] = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < 64; ++k) pm[k & 7] = fmaxf(pm[k & 7], __uint_as_float(sr[k]));
+  const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
+  const float mn = mx * sl2;
+  if (mn > m + 8.f) {
+    if (m != -INFINITY) {
+      alpha = ex2_approx(m - mn);
+      rescale = true;
+    }
+    m = mn;
+  }
+  const float2 a2 = make_float2(sl2, sl2), b2 = make_float2(-m, -m);
+  float2 acc[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    uint32_t hi[16], lo[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int i = c * 32 + 2 * k;
+      const float2 t = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), a2, b2);
+      const float p0 = ex2_approx(t.x), p1 = ex2_approx(t.y);
+      acc[k & 3] = __fadd2_rn(acc[k & 3], make_float2(p0, p1));
+      __nv_bfloat16 h0, l0, h1, l1;
+      split_bf16(p0, h0, l0);
+      split_bf16(p1, h1, l1);
+      hi[k] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+      lo[k] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+    }
+    tmem_st16(tS + c * 16, hi);
+    tmem_st16(tS + 32 + c * 16, lo);
+  }
+  const float2 s01 = __fadd2_rn(acc[0], acc[1]), s23 = __fadd2_rn(acc[2], acc[3]);
+  const float2 st = __fadd2_rn(s01, s23);
+  l = l * alpha + (st.x + st.y);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    sparse_attn_tc_kernel(const __grid_constant__ TcMaps maps, const AttnArgs a, int nQ128, int nKc, int nQ64,
+                          int nKq) {
+  using Lay = TcLayout<D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem =
+      reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* sQ = smem;
+  unsigned char* sK = smem + Lay::kQBytes;                    // [kKStages] K tiles
+  unsigned char* sV = sK + kKStages * Lay::kKVBytes;          // [kVStages] V tiles
+  int* tiles = reinterpret_cast<int*>(smem + Lay::kBytes);  // [r/64 + nKc + nKq]
+  int* flags = tiles + (a.EKhi ? a.r / 64 : 0) + nKc + nKq; // [nKq]
+  __shared__ __align__(8) uint64_t bar_q, bar_k_full[kKStages], bar_k_empty[kKStages], bar_v_full[kVStages],
+      bar_v_empty[kVStages], bar_s_full[2], bar_p_full[2], bar_o_done;
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_ntiles;
+
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int qb = blockIdx.x % nQ128, h = blockIdx.x / nQ128;
+  const int q0 = qb * 128;
+  int* status = a.status;
+
+  if (warp == 0) {
+    tmem_alloc(&s_tmem, 512);
+    tmem_relinquish();
+  }
+  if (tid == 32) {
+    mbar_init(&bar_q, 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(&bar_k_full[s], 1);
+      mbar_init(&bar_k_empty[s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(&bar_v_full[s], 1);
+      mbar_init(&bar_v_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bar_s_full[b], 1);
+      mbar_init(&bar_p_full[b], 128);
+    }
+    mbar_init(&bar_o_done, 1);
+    fence_barrier_init();
+  }
+
+  // ---- key-tile list (linear tiles, cached tiles, chunk tiles).  Selection counts
+  // and ids come from caller buffers: counts are clamped, out-of-range ids skipped.
+  const bool do_lin = a.EKhi != nullptr;
+  const bool do_sparse = a.inter_cnt != nullptr;
+  const int n_lin = do_lin ? a.r / 64 : 0;
+  const int n_inter = do_sparse ? min(max(a.inter_cnt[(long long)h * nQ128 + qb], 0), nKc) : 0;
+  for (int t = tid; t < n_lin; t += kTcThreads) tiles[t] = tc_tile_code((long long)t * 64, kTileLinear, 3);
+  if (do_sparse) {
+    const int32_t* ilist = a.inter_idx + ((long long)h * nQ128 + qb) * nKc;
+    for (int m = tid; m < n_inter; m += kTcThreads) {
+      const long long j = ilist[m];
+      const bool ok = j >= 0 && j < nKc;
+      if (!ok) set_status(status, HSA_ERR_DEVICE);
+      tiles[n_lin + m] = ok ? tc_tile_code(j * 128, kTileCached, 3) : tc_tile_code(0, kTileCached, 0);
+    }
+    for (int j = tid; j < nKq; j += kTcThreads) flags[j] = 0;
+  }
+  __syncthreads();
+  if (do_sparse) {
+    for (int half = 0; half < 2; ++half) {
+      const int i64 = 2 * qb + half;
+      if (i64 < nQ64) {
+        const int cnt = min(max(a.intra_cnt[(long long)h * nQ64 + i64], 0), nKq);
+        const int32_t* lst = a.intra_idx + ((long long)h * nQ64 + i64) * nKq;
+        for (int m = tid; m < cnt; m += kTcThreads) {
+          const int j = lst[m];
+          if (j >= 0 && j < nKq) atomicOr(&flags[j], 1 << half);
+          else set_status(status, HSA_ERR_DEVICE);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    int base = n_lin + n_inter;
+    if (do_sparse) {
+      for (int b = 0; b < nKq; b += 32) {
+        const int j = b + lane;
+        const int f = j < nKq ? flags[j] : 0;
+        const unsigned bal = __ballot_sync(0xffffffffu, f != 0);
+        if (f) tiles[base + __popc(bal & ((1u << lane) - 1u))] = tc_tile_code((long long)j * 64, kTileChunk, f);
+        base += __popc(bal);
+      }
+    }
+    if (lane == 0) s_ntiles = base;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const int T = s_ntiles;
+  if (T == 0 && tid == 0) set_status(status, HSA_ERR_DEVICE);  // no key tile: selection buffers were empty
+  const uint32_t tmem = s_tmem;
+  const uint32_t tOs = tmem + 256, tOl = tmem + 256 + D;
+  constexpr int kHalfSlot = (D / 64) * 64 * 128;  // 64 rows x D bf16: hi part / lo part of a slot
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ Q + K producer
+    if (lane == 0) {
+      prefetch_tensormap(&maps.q);
+      mbar_arrive_expect_tx(&bar_q, Lay::kQBytes);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) tma_load_2d(sQ + c * kRegionBytes, &maps.q, &bar_q, h * D + c * 64, q0);
+    }
+    for (int j = 0; j < T; ++j) {
+      const int s = j % kKStages;
+      if (!mbar_wait(&bar_k_empty[s], ((j / kKStages) & 1) ^ 1, status)) break;
+      if (lane == 0) {
+        const int code = tiles[j];
+        const int type = tile_type(code);
+        const int rows = tile_rows(code);
+        unsigned char* dK = sK + s * Lay::kKVBytes;
+        mbar_arrive_expect_tx(&bar_k_full[s], type == kTileLinear ? 2 * kHalfSlot : (D / 64) * rows * 128);
+        if (type == kTileLinear) {
+          const int y = h * a.r + tile_start(code);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_2d(dK + c * 64 * 128, &maps.ekhi, &bar_k_full[s], c * 64, y);
+            tma_load_2d(dK + kHalfSlot + c * 64 * 128, &maps.eklo, &bar_k_full[s], c * 64, y);
+          }
+        } else {
+          const CUtensorMap* mk = type == kTileChunk ? &maps.kq : &maps.kc;
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_2d(dK + c * rows * 128, mk, &bar_k_full[s], h * D + c * 64, tile_start(code));
+        }
+      }
+      __syncwarp();
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------ V producer
+    for (int j = 0; j < T; ++j) {
+      const int s = j % kVStages;
+      if (!mbar_wait(&bar_v_empty[s], ((j / kVStages) & 1) ^ 1, status)) break;
+      if (lane == 0) {
+        const int code = tiles[j];
+        const int type = tile_type(code);
+        const int rows = tile_rows(code);
+        unsigned char* dV = sV + s * Lay::kKVBytes;
+        mbar_arrive_expect_tx(&bar_v_full[s], type == kTileLinear ? 2 * kHalfSlot : (D / 64) * rows * 128);
+        if (type == kTileLinear) {
+          const int y = h * a.r + tile_start(code);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_2d(dV + c * 64 * 128, &maps.fvhi, &bar_v_full[s], c * 64, y);
+            tma_load_2d(dV + kHalfSlot + c * 64 * 128, &maps.fvlo, &bar_v_full[s], c * 64, y);
+          }
+        } else {
+          const CUtensorMap* mv = type == kTileChunk ? &maps.vq : &maps.vc;
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_2d(dV + c * rows * 128, mv, &bar_v_full[s], h * D + c * 64, tile_start(code));
+        }
+      }
+      __syncwarp();
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    bool ok = mbar_wait(&bar_q, 0, status);
+    tc_fence_after();
+    const uint32_t q_base = smem_u32(sQ);
+    auto issue_s = [&](int j) -> bool {
+      const int s = j % kKStages;
+      if (!mbar_wait(&bar_k_full[s], (j / kKStages) & 1, status)) return false;
+      tc_fence_after();
+      if (lane == 0) {
+        const int code = tiles[j];
+        const int rows = tile_rows(code);
+        const uint32_t idesc = idesc_bf16(128, rows, false, false);
+        const uint32_t k_base = smem_u32(sK + s * Lay::kKVBytes);
+        const uint32_t tS = tmem + (j & 1) * 128;
+        const int parts = tile_type(code) == kTileLinear ? 2 : 1;  // EK_hi then EK_lo
+        for (int part = 0; part < parts; ++part) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t qa = q_base + (kk / 4) * kRegionBytes + (kk % 4) * 32;
+            const uint32_t ka = k_base + part * kHalfSlot + (kk / 4) * (rows * 128) + (kk % 4) * 32;
+            mma_ss(tS, sdesc_sw128(qa, 16, 1024), sdesc_sw128(ka, 16, 1024), idesc,
+                   (part > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        mma_commit(&bar_k_empty[s]);
+        mma_commit(&bar_s_full[j & 1]);
+      }
+      __syncwarp();
+      return true;
+    };
+    if (ok && T > 0) ok = issue_s(0);
+    for (int j = 0; ok && j < T; ++j) {
+      if (j + 1 < T && !issue_s(j + 1)) break;
+      if (!mbar_wait(&bar_p_full[j & 1], (j >> 1) & 1, status)) break;
+      const int sv = j % kVStages;
+      if (!mbar_wait(&bar_v_full[sv], (j / kVStages) & 1, status)) break;
+      tc_fence_after();
+      if (lane == 0) {
+        const int code = tiles[j];
+        const int rows = tile_rows(code);
+        const uint32_t idesc = idesc_bf16(128, D, false, true);
+        const uint32_t v_base = smem_u32(sV + sv * Lay::kKVBytes);
+        const uint32_t tP = tmem + (j & 1) * 128;
+        if (tile_type(code) == kTileLinear) {
+          // O_l += P_hi FV_hi + P_lo FV_hi + P_hi FV_lo; first linear tile initialises O_l
+          const bool first = j == 0;
+#pragma unroll
+          for (int term = 0; term < 3; ++term) {
+            const uint32_t pa = tP + (term == 1 ? 32 : 0);
+            const uint32_t vb = v_base + (term == 2 ? kHalfSlot : 0);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_ts(tOl, pa + kk * 8, sdesc_sw128(vb + kk * 2048, 64 * 128, 1024), idesc,
+                     (!first || term > 0 || kk > 0) ? 1u : 0u);
+          }
+        } else {
+          const bool first = j == n_lin;  // first sparse tile initialises O_s
+          for (int kk = 0; kk < rows / 16; ++kk)
+            mma_ts(tOs, tP + kk * 8, sdesc_sw128(v_base + kk * 2048, rows * 128, 1024), idesc,
+                   (!first || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&bar_v_empty[sv]);
+        mma_commit(&bar_o_done);
+      }
+      __syncwarp();
+    }
+  } else if (warp >= 2 && warp <= 5) {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int wq = warp & 3;
+    const int row = 32 * wq + lane;
+    const int half_bit = wq < 2 ? 1 : 2;  // warp-uniform: rows 0..63 are half 0
+    const uint32_t loff = (uint32_t)(32 * wq) << 16;
+    const float sl2 = a.scale * 1.4426950408889634f;
+    float ms = -INFINITY, ls = 0.f;  // sparse branch running max / sum
+    float ml = -INFINITY, ll = 0.f;  // linear branch running max / sum
+    bool ok = true;
+    for (int j = 0; j < T; ++j) {
+      const int b = j & 1;
+      if (!mbar_wait(&bar_s_full[b], (j >> 1) & 1, status)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int code = tiles[j];
+      const int type = tile_type(code);
+      const int rows = tile_rows(code);
+      const long long nrows = type == kTileChunk ? (long long)a.Lq : a.Lc;
+      const int valid = type == kTileLinear ? 64 : (int)min((long long)rows, nrows - tile_start(code));
+      const bool used = (code & half_bit) != 0;
+      const uint32_t tS = tmem + b * 128 + loff;
+      float alpha = 1.f;
+      bool rescale = false;
+      if (type == kTileLinear) {  // tile-uniform
+        uint32_t h64[64];
+        tmem_ld64_sync(tS, h64);
+        softmax_tile_split(h64, sl2, ml, ll, alpha, rescale, tS);
+      } else if (used) {  // warp-uniform (a warp's 32 rows lie in one 64-row half)
+        uint32_t sr[128];
+        if (rows == 128) {
+          tmem_ld128_sync(tS, sr);
+          if (valid == 128) softmax_tile<128, false>(sr, valid, sl2, ms, ls, alpha, rescale, tS);
+          else softmax_tile<128, true>(sr, valid, sl2, ms, ls, alpha, rescale, tS);
+        } else {
+          uint32_t h64[64];
+          tmem_ld64_sync(tS, h64);
+#pragma unroll
+          for (int k = 0; k < 64; ++k) sr[k] = h64[k];
+          if (valid == 64) softmax_tile<64, false>(sr, valid, sl2, ms, ls, alpha, rescale, tS);
+          else softmax_tile<64, true>(sr, valid, sl2, ms, ls, alpha, rescale, tS);
+        }
+      } else {
+        uint32_t zero[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) zero[k] = 0u;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (c * 32 < rows) tmem_st16(tS + c * 16, zero);
+      }
+      tmem_st_wait();
+      // O holds the P.V products of tiles 0..j-1 once the previous one has completed
+      if (j > 0) {
+        if (!mbar_wait(&bar_o_done, (j - 1) & 1, status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
+      if (__any_sync(0xffffffffu, rescale)) {
+        const uint32_t tO = type == kTileLinear ? tOl : tOs;
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t r[16];
+          tmem_ld16_sync(tO + loff + c * 16, r);
+#pragma unroll
+          for (int k = 0; k < 16; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
+          tmem_st16(tO + loff + c * 16, r);
+        }
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      mbar_arrive(&bar_p_full[b]);
+    }
+    if (ok && T > 0 && mbar_wait(&bar_o_done, (T - 1) & 1, status)) {
+      tc_fence_after();
+      const int grow = q0 + row;
+      // out = g o_s + (1 - g) o_l with g = sigmoid(gate logit) when both branches run
+      float ws = 0.f, wl = 0.f;
+      if (do_sparse && do_lin) {
+        const float g = a.gate_logit ? 1.f / (1.f + expf(-a.gate_logit[h])) : 1.f;
+        ws = g / ls;
+        wl = (1.f - g) / ll;
+      } else if (do_sparse) {
+        ws = 1.f / ls;
+      } else {
+        wl = 1.f / ll;
+      }
+#pragma unroll
+      for (int c = 0; c < D / 16; ++c) {
+        uint32_t rs[16], rl[16];
+        if (do_sparse) tmem_ld16_sync(tOs + loff + c * 16, rs);
+        if (do_lin) tmem_ld16_sync(tOl + loff + c * 16, rl);
+        if (grow < a.Lq) {
+          const long long idx = ((long long)grow * a.H + h) * D + c * 16;
+          float v[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const float vs = do_sparse ? __uint_as_float(rs[k]) * ws : 0.f;
+            const float vl = do_lin ? __uint_as_float(rl[k]) * wl : 0.f;
+            v[k] = vs + vl;
+          }
+          if (a.out_bf16) {
+            uint4 w0, w1;
+            w0.x = pack_bf16x2(v[0], v[1]); w0.y = pack_bf16x2(v[2], v[3]);
+            w0.z = pack_bf16x2(v[4], v[5]); w0.w = pack_bf16x2(v[6], v[7]);
+            w1.x = pack_bf16x2(v[8], v[9]); w1.y = pack_bf16x2(v[10], v[11]);
+            w1.z = pack_bf16x2(v[12], v[13]); w1.w = pack_bf16x2(v[14], v[15]);
+            *reinterpret_cast<uint4*>(a.out_bf16 + idx) = w0;
+            *reinterpret_cast<uint4*>(a.out_bf16 + idx + 8) = w1;
+          } else {
+#pragma unroll
+            for (int k = 0; k < 16; k += 4)
+              *reinterpret_cast<float4*>(a.out_f32 + idx + k) = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+cudaError_t get_encoder() {
+  std::call_once(g_encode_once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode ? cudaSuccess : cudaErrorNotSupported;
+}
+
+// [rows, cols] bf16 row-major, boxes of 64 columns x box_rows rows, 128-byte swizzle.
+cudaError_t make_map(CUtensorMap* m, const void* base, long long rows, long long cols, int box_rows) {
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)(rows > 0 ? rows : 1)};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int D>
+cudaError_t launch_tc(const AttnArgs& a, cudaStream_t s) {
+  const int nQ128 = (a.Lq + 127) / 128, nQ64 = (a.Lq + 63) / 64;
+  const int nKc = (int)((a.Lc + 127) / 128), nKq = nQ64;
+  cudaError_t e = get_encoder();
+  if (e != cudaSuccess) return e;
+  TcMaps maps;
+  const long long HD = (long long)a.H * D;
+  if ((e = make_map(&maps.q, a.Q, a.Lq, HD, 128)) != cudaSuccess) return e;
+  if ((e = make_map(&maps.kq, a.Kq, a.Lq, HD, 64)) != cudaSuccess) return e;
+  if ((e = make_map(&maps.vq, a.Vq, a.Lq, HD, 64)) != cudaSuccess) return e;
+  // maps a launch never reads point at the chunk tensors
+  const bool hist = a.Lc > 0 && a.Kc != nullptr;
+  if ((e = make_map(&maps.kc, hist ? a.Kc : a.Kq, hist ? a.Lc : a.Lq, HD, 128)) != cudaSuccess) return e;
+  if ((e = make_map(&maps.vc, hist ? a.Vc : a.Vq, hist ? a.Lc : a.Lq, HD, 128)) != cudaSuccess) return e;
+  const bool lin = a.EKhi != nullptr;
+  const long long pr = (long long)a.H * a.r;
+  if ((e = make_map(&maps.ekhi, lin ? a.EKhi : a.Kq, lin ? pr : a.Lq, lin ? D : HD, 64)) != cudaSuccess) return e;
+  if ((e = make_map(&maps.eklo, lin ? a.EKlo : a.Kq, lin ? pr : a.Lq, lin ? D : HD, 64)) != cudaSuccess) return e;
+  if ((e = make_map(&maps.fvhi, lin ? a.FVhi : a.Vq, lin ? pr : a.Lq, lin ? D : HD, 64)) != cudaSuccess) return e;
+  if ((e = make_map(&maps.fvlo, lin ? a.FVlo : a.Vq, lin ? pr : a.Lq, lin ? D : HD, 64)) != cudaSuccess) return e;
+  const int n_lin = lin ? a.r / 64 : 0;
+  const size_t smem = 1024 + TcLayout<D>::kBytes + (size_t)(n_lin + nKc + 2 * nKq) * 4;
+  if (smem > 232448) return cudaErrorInvalidConfiguration;
+  e = cudaFuncSetAttribute(sparse_attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  sparse_attn_tc_kernel<D><<<a.H * nQ128, kTcThreads, smem, s>>>(maps, a, nQ128, nKc, nQ64, nKq);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s) {
+  return a.d == 128 ? launch_tc<128>(a, s) : launch_tc<64>(a, s);
+}
+
+}  // namespace hsa

@@ -5,6 +5,7 @@
 // All of these are HBM (or host-link) bound: they stream bf16 rows once with
 // 16-byte vector loads, one thread per 16-byte column chunk, and reduce in fp32
 // in a fixed order (deterministic results).
+#include <cooperative_groups.h>
 #include <float.h>
 
 #include "common.cuh"
@@ -51,8 +52,23 @@ __global__ void __launch_bounds__(256) colsum_partial_kernel(const uint16_t* __r
 }
 
 int colsum_splits(long long n) {
-  long long s = (n + 15) / 16;
+  long long s = (n + 15) / 16;  // 16 rows per split
   return (int)(s < 1 ? 1 : (s > kColMaxSplits ? kColMaxSplits : s));
+}
+
+// Sum of part[q][c] over the splits, with four independent accumulators so that
+// the loads of consecutive splits overlap.
+__device__ __forceinline__ float sum_splits(const float* __restrict__ part, int splits, int C, int c) {
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  int q = 0;
+  for (; q + 4 <= splits; q += 4) {
+    a0 += part[(long long)q * C + c];
+    a1 += part[(long long)(q + 1) * C + c];
+    a2 += part[(long long)(q + 2) * C + c];
+    a3 += part[(long long)(q + 3) * C + c];
+  }
+  for (; q < splits; ++q) a0 += part[(long long)q * C + c];
+  return (a0 + a1) + (a2 + a3);
 }
 
 cudaError_t launch_colsum_partial(const uint16_t* X, long long n, int C, float* part, cudaStream_t s) {
@@ -67,9 +83,7 @@ __global__ void page_summary_final_kernel(const float* __restrict__ part, int sp
                                           float* __restrict__ kbar) {
   int c = blockIdx.x * blockDim.x + threadIdx.x;
   if (c >= C) return;
-  float s = 0.f;
-  for (int q = 0; q < splits; ++q) s += part[(long long)q * C + c];
-  kbar[c] = s / (float)n;
+  kbar[c] = sum_splits(part, splits, C, c) / (float)n;
 }
 
 cudaError_t launch_page_summary_final(const float* part, long long n, int C, float* kbar, cudaStream_t s) {
@@ -78,22 +92,49 @@ cudaError_t launch_page_summary_final(const float* part, long long n, int C, flo
 }
 
 // ------------------------------------------------------------------ page-level retrieval
-// One CTA: qbar = column means of Q, s_p = qbar . kbar_p for candidates, top-Kp
-// (ties -> lower page id), written ascending.
-__global__ void __launch_bounds__(1024) select_pages_final_kernel(
+// One 8-CTA cluster.  CTA k sums the column partials of row splits k, k+8, ... into
+// its shared memory; CTA 0 then reads the eight partial vectors over distributed
+// shared memory in a fixed order (deterministic), forms qbar = column means of Q,
+// scores s_p = qbar . kbar_p for the candidates and keeps the top Kp (ties -> lower
+// page id), written ascending.
+constexpr int kSelCluster = 8;
+
+__global__ void __cluster_dims__(kSelCluster, 1, 1) __launch_bounds__(1024) select_pages_final_kernel(
     const float* __restrict__ part, int splits, long long Lq, int C, const float* __restrict__ kbar, int NP,
     const int32_t* __restrict__ cand_range, int Kp, int32_t* __restrict__ sel_out, float* __restrict__ scores_out,
     int* status) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
   extern __shared__ float sm[];
-  float* qbar = sm;           // [C]
-  float* score = sm + C;      // [NP]
-  int* taken = reinterpret_cast<int*>(score + NP);  // [NP]
+  float* qpart = sm;            // [C] this CTA's share of the split sums
+  float* qbar = sm + C;         // [C] (CTA 0)
+  float* score = qbar + C;      // [NP] (CTA 0)
+  int* taken = reinterpret_cast<int*>(score + NP);  // [NP] (CTA 0)
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32, nwarps = blockDim.x / 32;
   for (int c = tid; c < C; c += blockDim.x) {
-    float s = 0.f;
-    for (int q = 0; q < splits; ++q) s += part[(long long)q * C + c];
-    qbar[c] = s / (float)Lq;
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+    int q = rank;
+    for (; q + 3 * kSelCluster < splits; q += 4 * kSelCluster) {
+      a0 += part[(long long)q * C + c];
+      a1 += part[(long long)(q + kSelCluster) * C + c];
+      a2 += part[(long long)(q + 2 * kSelCluster) * C + c];
+      a3 += part[(long long)(q + 3 * kSelCluster) * C + c];
+    }
+    for (; q < splits; q += kSelCluster) a0 += part[(long long)q * C + c];
+    qpart[c] = (a0 + a1) + (a2 + a3);
   }
+  cluster.sync();
+  if (rank == 0) {
+    for (int c = tid; c < C; c += blockDim.x) {
+      float t = 0.f;
+      for (int k = 0; k < kSelCluster; ++k) t += cluster.map_shared_rank(qpart, k)[c];
+      qbar[c] = t / (float)Lq;
+    }
+  }
+  cluster.sync();  // the other CTAs' shared memory stays valid until CTA 0 has read it
+  if (rank != 0) return;
+
   int first = 0, end = NP;
   if (cand_range) {
     first = cand_range[0];
@@ -138,8 +179,7 @@ __global__ void __launch_bounds__(1024) select_pages_final_kernel(
       taken[best] = 1;
       if (nchosen < 64) chosen[nchosen++] = best;
     }
-    // ascending page order (insertion sort, Kp <= 64)
-    for (int a = 1; a < nchosen; ++a) {
+    for (int a = 1; a < nchosen; ++a) {  // ascending page order (insertion sort, Kp <= 64)
       int v = chosen[a], b = a - 1;
       while (b >= 0 && chosen[b] > v) {
         chosen[b + 1] = chosen[b];
@@ -154,14 +194,14 @@ __global__ void __launch_bounds__(1024) select_pages_final_kernel(
 cudaError_t launch_select_pages_final(const float* part, long long Lq, int C, const float* kbar_pages, int NP,
                                       const int32_t* cand_range, int Kp, int32_t* sel_out, float* scores_out,
                                       int* status, cudaStream_t s) {
-  size_t smem = (size_t)C * 4 + (size_t)NP * 8;
+  size_t smem = (size_t)C * 8 + (size_t)NP * 8;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(select_pages_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
   }
-  select_pages_final_kernel<<<1, 1024, smem, s>>>(part, colsum_splits(Lq), Lq, C, kbar_pages, NP, cand_range, Kp,
-                                                  sel_out, scores_out, status);
+  select_pages_final_kernel<<<kSelCluster, 1024, smem, s>>>(part, colsum_splits(Lq), Lq, C, kbar_pages, NP,
+                                                             cand_range, Kp, sel_out, scores_out, status);
   return cudaGetLastError();
 }
 
@@ -222,71 +262,79 @@ cudaError_t launch_select_prompt(const float* e_cur, const float* e_seg, int n_s
 }
 
 // ------------------------------------------------------------------ gather
-// Unit = (K or V, 128-row block j of the output, head h): 128 rows x d columns.
-// Row R of the output comes from page sel[R / P_tok], row R % P_tok.  Each thread
-// moves one 16-byte chunk of NIT rows (all loads issued before the stores).  For
-// K units the 128-row block mean per head is accumulated on the way (fp32,
-// fixed order) and written to kbar128[j, h, :].
-template <int D>
-__global__ void __launch_bounds__(256) gather_kernel(const uint16_t* const* __restrict__ page_k,
-                                                     const uint16_t* const* __restrict__ page_v, int NP,
-                                                     const int32_t* __restrict__ sel, long long P_tok, int H,
-                                                     long long Lc, uint16_t* __restrict__ Kc,
-                                                     uint16_t* __restrict__ Vc, float* __restrict__ kbar128,
-                                                     int* status) {
-  constexpr int TPR = D / 8;
-  constexpr int RPI = 256 / TPR;
-  constexpr int NIT = 128 / RPI;
-  __shared__ float red[RPI][D];
+// Unit = (K or V, 128-row block j of the output): 128 full rows (all heads).
+// Row R of the output comes from page sel[R / P_tok], row R % P_tok; a row is
+// H*d contiguous bf16 in both the page and the output.  Thread t owns the 16-byte
+// column chunk t of every row of the block and keeps 8 rows in flight; for K units
+// it also accumulates the 128-row block mean of its 8 columns (fp32, fixed order)
+// and writes kbar128[j, :, :] directly.  Page ids and page pointers come from
+// device memory and are checked here (range, 16-byte alignment).
+constexpr int kGatherUnroll = 8;
+
+constexpr int kGatherMaxThreads = 640;  // one thread per 16-byte column up to H*d = 5120
+
+__global__ void __launch_bounds__(kGatherMaxThreads) gather_kernel(
+    const uint16_t* const* __restrict__ page_k, const uint16_t* const* __restrict__ page_v, int NP,
+    const int32_t* __restrict__ sel, long long P_tok, int C, long long Lc, uint16_t* __restrict__ Kc,
+    uint16_t* __restrict__ Vc, float* __restrict__ kbar128, int* status) {
   const long long nblk = (Lc + 127) / 128;
-  long long unit = blockIdx.x;
-  const int h = (int)(unit % H);
-  unit /= H;
-  const long long j = unit % nblk;
-  const int kv = (int)(unit / nblk);
-  const int c = threadIdx.x % TPR, rp = threadIdx.x / TPR;
+  const long long j = blockIdx.x % nblk;
+  const int kv = (int)(blockIdx.x / nblk);
+  const int CV = C / 8;
   const uint16_t* const* pages = kv ? page_v : page_k;
   uint16_t* dst = kv ? Vc : Kc;
-
-  uint4 v[NIT];
-  bool ok[NIT];
+  const long long r0 = j * 128;
+  const int rows = (int)min((long long)128, Lc - r0);
+  const bool pool = kv == 0 && kbar128 != nullptr;
+  const int slot0 = (int)(r0 / P_tok);
+  const long long t0 = r0 - (long long)slot0 * P_tok;
+  for (int cc = threadIdx.x; cc < CV; cc += blockDim.x) {
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    // current page of this block's rows (rows are consecutive: advance slot by slot)
+    int slot = -1;
+    const uint16_t* base = nullptr;
+    long long t = t0;
+    int cur = slot0;
+    for (int i0 = 0; i0 < rows; i0 += kGatherUnroll) {
+      uint4 v[kGatherUnroll];
+      bool ok[kGatherUnroll];
 #pragma unroll
-  for (int it = 0; it < NIT; ++it) {
-    const long long R = j * 128 + rp + it * RPI;
-    ok[it] = false;
-    if (R < Lc) {
-      const int slot = (int)(R / P_tok);
-      const long long t = R - (long long)slot * P_tok;
-      const int p = sel[slot];
-      const uint16_t* base = (p >= 0 && p < NP) ? pages[p] : nullptr;
-      // page pointers come from a device table: check range and 16-byte alignment here
-      if (base != nullptr && (reinterpret_cast<uintptr_t>(base) & 15u) == 0) {
-        v[it] = ld_nc_v4(base + (t * H + h) * D + c * 8);
-        ok[it] = true;
-      } else {
-        set_status(status, HSA_ERR_DEVICE);
+      for (int u = 0; u < kGatherUnroll; ++u) {
+        ok[u] = false;
+        if (i0 + u < rows) {
+          while (t >= P_tok) {
+            t -= P_tok;
+            ++cur;
+          }
+          if (cur != slot) {
+            slot = cur;
+            const int p = sel[slot];
+            base = (p >= 0 && p < NP) ? pages[p] : nullptr;
+            if (base == nullptr || (reinterpret_cast<uintptr_t>(base) & 15u) != 0) {
+              base = nullptr;
+              set_status(status, HSA_ERR_DEVICE);
+            }
+          }
+          if (base != nullptr) {
+            v[u] = ld_nc_v4(base + t * C + cc * 8);
+            ok[u] = true;
+          }
+          ++t;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kGatherUnroll; ++u) {
+        if (ok[u]) {
+          *reinterpret_cast<uint4*>(dst + (r0 + i0 + u) * C + cc * 8) = v[u];
+          if (pool) add8(acc, v[u]);
+        }
       }
     }
-  }
+    if (pool) {
+      float* out = kbar128 + j * C + cc * 8;
+      const float inv = 1.f / (float)rows;
 #pragma unroll
-  for (int it = 0; it < NIT; ++it) {
-    const long long R = j * 128 + rp + it * RPI;
-    if (ok[it]) *reinterpret_cast<uint4*>(dst + (R * H + h) * D + c * 8) = v[it];
-  }
-  if (kv == 0 && kbar128 != nullptr) {
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-#pragma unroll
-    for (int it = 0; it < NIT; ++it)
-      if (ok[it]) add8(acc, v[it]);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) red[rp][c * 8 + k] = acc[k];
-    __syncthreads();
-    const long long rows = min((long long)128, Lc - j * 128);
-    for (int col = threadIdx.x; col < D; col += 256) {
-      float s = 0.f;
-#pragma unroll
-      for (int q = 0; q < RPI; ++q) s += red[q][col];
-      kbar128[(j * H + h) * D + col] = s / (float)rows;
+      for (int k = 0; k < 8; ++k) out[k] = acc[k] * inv;
     }
   }
 }
@@ -296,11 +344,10 @@ cudaError_t launch_gather(const uint16_t* const* page_k, const uint16_t* const* 
                           uint16_t* Vc, float* kbar128, int* status, cudaStream_t s) {
   const long long Lc = (long long)Kp * P_tok;
   const long long nblk = (Lc + 127) / 128;
-  const long long grid = 2 * nblk * H;
-  if (d == 128)
-    gather_kernel<128><<<(unsigned)grid, 256, 0, s>>>(page_k, page_v, NP, sel, P_tok, H, Lc, Kc, Vc, kbar128, status);
-  else
-    gather_kernel<64><<<(unsigned)grid, 256, 0, s>>>(page_k, page_v, NP, sel, P_tok, H, Lc, Kc, Vc, kbar128, status);
+  const int CV = H * d / 8;
+  const int threads = CV >= kGatherMaxThreads ? kGatherMaxThreads : ((CV + 31) / 32) * 32;
+  gather_kernel<<<(unsigned)(2 * nblk), threads, 0, s>>>(page_k, page_v, NP, sel, P_tok, H * d, Lc, Kc, Vc,
+                                                         kbar128, status);
   return cudaGetLastError();
 }
 

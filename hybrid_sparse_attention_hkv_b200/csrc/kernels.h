@@ -39,7 +39,7 @@ cudaError_t launch_block_select(const float* q128, const float* kc128, const flo
                                 int32_t* inter_idx, int32_t* inter_cnt, int32_t* intra_idx, int32_t* intra_cnt,
                                 cudaStream_t s);
 
-// ---------------------------------------------------------------- attn.cu
+// ---------------------------------------------------------------- attn_tc.cu
 struct AttnArgs {
   const uint16_t* Q;
   const uint16_t* Kc;
@@ -49,33 +49,37 @@ struct AttnArgs {
   int H, d, Lq;
   long long Lc;
   float scale;
-  // sparse branch
+  // sparse branch (runs when inter_cnt != NULL)
   const int32_t* inter_idx;
   const int32_t* inter_cnt;
   const int32_t* intra_idx;
   const int32_t* intra_cnt;
-  // linear branch: split-bf16 projections, [H][r][d]
+  // linear branch (runs when EKhi != NULL): split-bf16 projections, [H][r][d]
   const uint16_t* EKhi;
   const uint16_t* EKlo;
   const uint16_t* FVhi;
   const uint16_t* FVlo;
   int r;
+  // both branches: out = g o_s + (1 - g) o_l, g = sigmoid(gate_logit[h]) (NULL -> g = 1)
+  const float* gate_logit;
   // output [Lq, H, d]: fp32 (out_f32) or bf16 (out_bf16)
   float* out_f32;
   uint16_t* out_bf16;
-  // gated merge (sparse kernel only): out = g*o_sparse + (1-g)*o_lin, g = sigmoid(gate_logit[h])
-  const float* o_lin;
-  const float* gate_logit;
   int* status;  // workspace status word (may be NULL)
 };
-cudaError_t launch_sparse_attn(const AttnArgs& a, cudaStream_t s);
-cudaError_t launch_linear_attn(const AttnArgs& a, cudaStream_t s);
+// Sparse and/or linear branch with the gated merge, on tcgen05 / TMEM / TMA.
+cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s);
 
 // ---------------------------------------------------------------- proj.cu
 int proj_splits(int H, int r, long long L);
 cudaError_t launch_proj(const uint16_t* E, const uint16_t* F, long long ef_head_stride, const uint16_t* Kc,
                         const uint16_t* Kq, const uint16_t* Vc, const uint16_t* Vq, int H, int d, int r,
                         long long Lc, int Lq, int splits, float* part, cudaStream_t s);
+// tcgen05 / TMEM / TMA version (proj_tc.cu); partial-sum layout as launch_proj.
+int proj_tc_splits(int H, int r, long long Lc, int Lq);
+cudaError_t launch_proj_tc(const uint16_t* E, const uint16_t* F, long long ef_head_stride, const uint16_t* Kc,
+                           const uint16_t* Kq, const uint16_t* Vc, const uint16_t* Vq, int H, int d, int r,
+                           long long Lc, int Lq, int splits, float* part, int* status, cudaStream_t s);
 cudaError_t launch_proj_reduce(const float* part, int splits, int H, int d, int r, uint16_t* EKhi,
                                uint16_t* EKlo, uint16_t* FVhi, uint16_t* FVlo, cudaStream_t s);
 

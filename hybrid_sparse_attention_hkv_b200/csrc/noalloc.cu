@@ -61,8 +61,8 @@ extern "C" hsa_status_t hkv_select_pages_noalloc(const float* kbar_pages, int NP
   if (NP < 1 || Lq < 1) return hsa::api_fail(HSA_ERR_INVALID_ARG, "%s: NP = %d, Lq = %d must be >= 1", fn, NP, Lq);
   if (Kp < 1 || Kp > NP || Kp > 64)
     return hsa::api_fail(HSA_ERR_INVALID_ARG, "%s: Kp = %d must be in [1, min(NP, 64)]", fn, Kp);
-  if ((size_t)H * d * 4 + (size_t)NP * 8 > 200 * 1024)
-    return hsa::api_fail(HSA_ERR_UNSUPPORTED, "%s: H*d*4 + NP*8 bytes exceed the shared-memory budget", fn);
+  if ((size_t)H * d * 8 + (size_t)NP * 8 > 200 * 1024)
+    return hsa::api_fail(HSA_ERR_UNSUPPORTED, "%s: H*d*8 + NP*8 bytes exceed the shared-memory budget", fn);
   const size_t need = 256 + (size_t)hsa::kColMaxSplits * H * d * sizeof(float);
   if (need > kNoAllocScratchBytes)
     return hsa::api_fail(HSA_ERR_UNSUPPORTED, "%s: H*d = %d needs %zu scratch bytes, the static maximum is %zu", fn,

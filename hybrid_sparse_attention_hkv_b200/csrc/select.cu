@@ -194,13 +194,25 @@ __global__ void __launch_bounds__(kSelThreads) block_select_kernel(
 
   for (int c = tid; c < D; c += kSelThreads) qv[c] = qb[c];
   __syncthreads();
-  for (int j = warp; j < nK; j += kSelThreads / 32) {
-    const float* k = kb + ((long long)j * H + h) * D;
-    float s = 0.f;
+  // scores: each warp takes 8 blocks at a time so that their loads are in flight together
+  constexpr int kB = 8;
+  for (int j0 = warp * kB; j0 < nK; j0 += (kSelThreads / 32) * kB) {
+    float acc[kB];
 #pragma unroll
-    for (int c = lane; c < D; c += 32) s = fmaf(qv[c], k[c], s);
-    s = warp_sum(s);
-    if (lane == 0) e[j] = s * scale;
+    for (int u = 0; u < kB; ++u) {
+      acc[u] = 0.f;
+      const int j = j0 + u;
+      if (j < nK) {
+        const float* k = kb + ((long long)j * H + h) * D;
+#pragma unroll
+        for (int c = lane; c < D; c += 32) acc[u] = fmaf(qv[c], __ldg(k + c), acc[u]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      const float s = warp_sum(acc[u]);
+      if (lane == 0 && j0 + u < nK) e[j0 + u] = s * scale;
+    }
   }
   __syncthreads();
   // row max

@@ -36,8 +36,8 @@
  *     bytes (256-byte aligned) serves every entry point of a configuration.
  *     Calls that share a workspace must be ordered on one stream.
  *   - Supported shapes: d in {64, 128}; H >= 1; block_inter = 128;
- *     block_intra = 64; rank a multiple of 64 in [64, 1024]; (Lc + Lq) a
- *     multiple of 8; Lq >= 1.  Lc may be 0 (no retrieved history) and need not
+ *     block_intra = 64; rank a multiple of 64 in [64, 1024]; Lc and Lq
+ *     multiples of 8; Lq >= 1.  Lc may be 0 (no retrieved history) and need not
  *     be a multiple of 128 (a partial last inter block is the mean of its rows).
  */
 #ifndef HSA_H_
@@ -203,9 +203,10 @@ hsa_status_t hsa_sparse_attn(const hsa_config_t* cfg, const hsa_bf16* Q, const h
 /* Linear branch ([NEWS] HSA paragraph, Linformer-style low rank):
  *   EK_h = E_h [Kc; Kq]_h,  FV_h = F_h [Vc; Vq]_h   (E_h, F_h: [r, L], L = Lc+Lq)
  *   o_linear[t, h, :] = softmax_j(q_t . EK_h[j] * scale) FV_h        (fp32 out)
- * E, F: bf16 [r, L] row-major; head h reads E + h*ef_head_stride (0 = one
- * matrix shared by all heads).  EK/FV are accumulated in fp32 and applied with
- * split-bf16 (hi + lo) operands.  Uses the workspace. */
+ * E, F: bf16 [r, L] row-major; head h reads E + h*ef_head_stride, where
+ * ef_head_stride is 0 (one matrix shared by all heads) or r*L (H matrices
+ * stacked).  EK/FV are accumulated in fp32 and applied with split-bf16 (hi + lo)
+ * operands.  Uses the workspace. */
 hsa_status_t hsa_linear_attn(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc,
                              const hsa_bf16* Vc, const hsa_bf16* Kq, const hsa_bf16* Vq,
                              const hsa_bf16* E, const hsa_bf16* F, long long ef_head_stride,

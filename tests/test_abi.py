@@ -47,7 +47,8 @@ def test_workspace_size_and_shape_checks(lib):
         (hsa.make_config(2, 96, 256, 512, 64), 2),              # head dim
         (hsa.make_config(0, 64, 256, 512, 64), 1),              # heads
         (hsa.make_config(2, 64, 0, 512, 64), 1),                # empty chunk
-        (hsa.make_config(2, 64, 257, 512, 64), 2),              # Lc + Lq not a multiple of 8
+        (hsa.make_config(2, 64, 257, 512, 64), 2),              # Lq not a multiple of 8
+        (hsa.make_config(2, 64, 260, 500, 64), 2),              # Lc, Lq not multiples of 8 (sum is)
         (hsa.make_config(2, 64, 256, -8, 64), 1),               # negative history
         (hsa.make_config(2, 64, 256, 512, 64, block_inter=64), 2),
         (hsa.make_config(2, 64, 256, 512, 64, scale=float("nan")), 1),
