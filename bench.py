@@ -34,11 +34,8 @@ DEFAULT_WORKLOAD = 1
 # keyed by kernel; valid only while that kernel's section of its source file (from its
 # section marker to the next one) is unchanged (sha256 prefix of the section).
 TRAFFIC = {
-    # profiles/sparse_attn_mma_sync_wan1.3b_480p.md
-    "attention_merge": {"file": "attn_tc.cu", "sha": "none yet", "bytes": None},
     # profiles/gather_and_projection_hbm_wan1.3b_480p.md
-    "gather": {"file": "hkv.cu", "sha": "577b859a6a30a103", "bytes": 306822656 + 249974016},
-    "linformer_proj": {"file": "proj.cu", "sha": "2f89ba706af1053b", "bytes": 395510016 + 25282816},
+    "gather": {"file": "hkv.cu", "section": "gather", "sha": "ea6010aad5d6ab04", "bytes": 306762240 + 251291392},
 }
 
 

@@ -25,7 +25,11 @@
 //               when it grows by more than 2^8; finally o_s = O_s / l_s,
 //               o_l = O_l / l_l, out = g o_s + (1 - g) o_l, stored.
 // The tensor core computes S_{j+1} while the softmax warps work on S_j.
-// Every wait is bounded (HSA_ERR_TIMEOUT in the workspace status on expiry).
+// Every wait is bounded (HSA_ERR_TIMEOUT in the workspace status on expiry).  The
+// per-tile waits are per-lane polls of one barrier by a converged warp (a warp-wide
+// vote after each of them cost 7% of the kernel's time); the waits before the first
+// and after the last tile, where the warps go on to warp-collective TMEM access and
+// teardown, take the warp's common answer.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -103,15 +107,7 @@ __device__ __forceinline__ void softmax_tile(const uint32_t (&sr)[128], int vali
     for (int k = 0; k < 16; ++k) {
       const int i = c * 32 + 2 * k;
       const float2 t = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), a2, b2);
-      float p0, p1;
-      if (!MASKED && (k & 3) == 3) {  // every 4th pair on the FMA pipe, the rest on the SFU
-        const float2 e = ex2_poly2(t);
-        p0 = e.x;
-        p1 = e.y;
-      } else {
-        p0 = ex2_approx(t.x);
-        p1 = ex2_approx(t.y);
-      }
+      float p0 = ex2_approx(t.x), p1 = ex2_approx(t.y);
       if (MASKED) {
         if (i >= valid) p0 = 0.f;
         if (i + 1 >= valid) p1 = 0.f;
@@ -334,7 +330,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    bool ok = mbar_wait(&bar_q, 0, status);
+    bool ok = mbar_wait_warp(&bar_q, 0, status);
     tc_fence_after();
     const uint32_t q_base = smem_u32(sQ);
     auto issue_s = [&](int j) -> bool {
@@ -475,7 +471,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_before();
       mbar_arrive(&bar_p_full[b]);
     }
-    if (ok && T > 0 && mbar_wait(&bar_o_done, (T - 1) & 1, status)) {
+    if (ok && T > 0 && mbar_wait_warp(&bar_o_done, (T - 1) & 1, status)) {
       tc_fence_after();
       const int grow = q0 + row;
       // out = g o_s + (1 - g) o_l with g = sigmoid(gate logit) when both branches run

@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(kPjThreads, 1) proj_tc_kernel(const __grid_con
     const int wq = warp & 3;
     const int row = 32 * wq + lane;
     const uint32_t loff = (uint32_t)(32 * wq) << 16;
-    const bool have = nc > 0 && mbar_wait(&bar_acc, 0, a.status);
+    const bool have = nc > 0 && mbar_wait_warp(&bar_acc, 0, a.status);
     if (nc == 0 || have) {
       tc_fence_after();
       float* out = a.part + ((((long long)split * 2 + which) * a.H + h) * a.r) * D;
