@@ -1,6 +1,8 @@
 // C-ABI entry points of the HKV + HSA library: host-side argument checks,
 // workspace layout, per-kernel trace events and the launch sequence of each call.
-// Nothing here allocates, frees or synchronises (hsa_status_read excepted).
+// Nothing here allocates device memory, frees or synchronises (hsa_status_read
+// excepted); hsa_forward creates, on its first call on a thread and device, one
+// side stream and two events that it keeps for that thread.
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
@@ -70,6 +72,8 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 struct Layout {
   size_t status = 0, colpart = 0, q128 = 0, q64 = 0, kq64 = 0, kc128 = 0;
   size_t inter_idx = 0, inter_cnt = 0, intra_idx = 0, intra_cnt = 0;
+  size_t units = 0, n_units = 0, tile_done = 0, part_o = 0, part_ml = 0, part_lin = 0, attn_end = 0;
+  int max_units = 0, max_slots = 0;
   size_t ekhi = 0, eklo = 0, fvhi = 0, fvlo = 0, projpart = 0;
   size_t pages_end = 0;  // bytes needed by the page (HKV) calls
   size_t total = 0;
@@ -96,6 +100,16 @@ Layout make_layout(int H, int d, int Lq, long long Lc, int r) {
   L.inter_cnt = take((size_t)H * nQ128 * 4);
   L.intra_idx = take((size_t)H * nQ64 * nQ64 * 4);
   L.intra_cnt = take((size_t)H * nQ64 * 4);
+  // attention work plan and the partial results of split lists
+  L.max_units = hsa::plan_max_units(H, (int)nQ128);
+  L.max_slots = hsa::plan_max_slots();
+  L.units = take((size_t)L.max_units * 16);
+  L.n_units = take(16);
+  L.tile_done = take((size_t)H * nQ128 * 4);
+  L.part_o = take((size_t)L.max_slots * 128 * d * 4);
+  L.part_ml = take((size_t)L.max_slots * 128 * 8);
+  L.part_lin = take((size_t)L.max_slots * 128 * d * 4);
+  L.attn_end = off;
   const size_t hrd = (size_t)H * r * d;
   L.ekhi = take(hrd * 2);
   L.eklo = take(hrd * 2);
@@ -139,6 +153,29 @@ hsa_status_t check_cfg(const char* fn, const hsa_config_t* c, bool need_rank) {
 }
 
 inline float scale_of(const hsa_config_t* c) { return c->scale > 0.f ? c->scale : 1.0f / sqrtf((float)c->d); }
+
+// A non-blocking side stream and a fork / join event pair per device for this thread.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+constexpr int kMaxDevices = 64;
+thread_local SideStream t_side[kMaxDevices];
+
+cudaError_t side_stream(SideStream** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  SideStream& ss = t_side[dev];
+  if (!ss.s) {
+    if ((e = cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
+    if ((e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming)) != cudaSuccess) return e;
+  }
+  *out = &ss;
+  return cudaSuccess;
+}
 
 hsa_status_t check_ws(const char* fn, const void* ws, size_t ws_bytes, size_t need) {
   if (!ws) return fail(HSA_ERR_WORKSPACE, "%s: workspace is NULL", fn);
@@ -313,15 +350,32 @@ static hsa_status_t run_block_select(const hsa_config_t* cfg, const Layout& L, c
   return HSA_OK;
 }
 
-static hsa::AttnArgs attn_args(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc, const hsa_bf16* Vc,
-                               const hsa_bf16* Kq, const hsa_bf16* Vq) {
+static hsa::AttnArgs attn_args(const hsa_config_t* cfg, const Layout& L, void* ws, const hsa_bf16* Q,
+                               const hsa_bf16* Kc, const hsa_bf16* Vc, const hsa_bf16* Kq, const hsa_bf16* Vq) {
   hsa::AttnArgs a;
   memset(&a, 0, sizeof(a));
   a.Q = Q; a.Kc = Kc; a.Vc = Vc; a.Kq = Kq; a.Vq = Vq;
   a.H = cfg->H; a.d = cfg->d; a.Lq = cfg->Lq; a.Lc = cfg->Lc;
   a.scale = scale_of(cfg);
   a.r = cfg->rank;
+  a.status = status_of(ws);
+  a.max_units = L.max_units;
+  a.max_slots = L.max_slots;
   return a;
+}
+
+// Sparse-branch inputs of `a` and the work plan over them.
+static hsa_status_t run_plan(const Layout& L, const hsa_selection_t& sel, void* ws, hsa::AttnArgs& a,
+                             hsa_stream_t stream) {
+  a.inter_idx = sel.inter_idx; a.inter_cnt = sel.inter_cnt; a.intra_idx = sel.intra_idx; a.intra_cnt = sel.intra_cnt;
+  a.units = at<int4>(ws, L.units);
+  a.n_units = at<int>(ws, L.n_units);
+  a.tile_done = at<int>(ws, L.tile_done);
+  a.part_o = at<float>(ws, L.part_o);
+  a.part_ml = at<float2>(ws, L.part_ml);
+  a.part_lin = at<float>(ws, L.part_lin);
+  HSA_LAUNCH("attn_plan", hsa::launch_attn_plan(a, stream));
+  return HSA_OK;
 }
 
 // Linformer projection (EK, FV as split-bf16 pairs in the workspace); sets the
@@ -372,16 +426,15 @@ hsa_status_t hsa_sparse_attn(const hsa_config_t* cfg, const hsa_bf16* Q, const h
                              const hsa_bf16* Kq, const hsa_bf16* Vq, hsa_selection_t sel, float* o_sparse, void* ws,
                              size_t ws_bytes, hsa_stream_t stream) {
   const char* fn = __func__;
-  (void)ws;
-  (void)ws_bytes;
   TRY(check_cfg(fn, cfg, false));
   TRY(check_tensors(fn, cfg, Q, Kc, Vc, Kq, Vq, true));
   TRY(check_sel(fn, sel));
   REQUIRE_PTR(o_sparse);
-  hsa::AttnArgs a = attn_args(cfg, Q, Kc, Vc, Kq, Vq);
-  a.inter_idx = sel.inter_idx; a.inter_cnt = sel.inter_cnt; a.intra_idx = sel.intra_idx; a.intra_cnt = sel.intra_cnt;
+  const Layout L = make_layout(cfg->H, cfg->d, cfg->Lq, cfg->Lc, 0);
+  TRY(check_ws(fn, ws, ws_bytes, L.attn_end));
+  hsa::AttnArgs a = attn_args(cfg, L, ws, Q, Kc, Vc, Kq, Vq);
+  TRY(run_plan(L, sel, ws, a, stream));
   a.out_f32 = o_sparse;
-  a.status = ws ? status_of(ws) : nullptr;
   HSA_LAUNCH("attention", hsa::launch_attn_tc(a, stream));
   return HSA_OK;
 }
@@ -400,10 +453,9 @@ hsa_status_t hsa_linear_attn(const hsa_config_t* cfg, const hsa_bf16* Q, const h
     return fail(HSA_ERR_UNSUPPORTED, "%s: ef_head_stride must be 0 (shared) or r * (Lc + Lq) (stacked per head)", fn);
   const Layout L = make_layout(cfg->H, cfg->d, cfg->Lq, cfg->Lc, cfg->rank);
   TRY(check_ws(fn, ws, ws_bytes, L.total));
-  hsa::AttnArgs a = attn_args(cfg, Q, Kc, Vc, Kq, Vq);
+  hsa::AttnArgs a = attn_args(cfg, L, ws, Q, Kc, Vc, Kq, Vq);
   TRY(run_projection(cfg, L, Kc, Vc, Kq, Vq, E, F, ef_head_stride, ws, a, stream));
   a.out_f32 = o_linear;
-  a.status = status_of(ws);
   HSA_LAUNCH("attention", hsa::launch_attn_tc(a, stream));
   return HSA_OK;
 }
@@ -437,11 +489,21 @@ hsa_status_t hsa_forward(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_b
     sel.intra_cnt = at<int32_t>(ws, L.intra_cnt);
   }
   TRY(run_block_select(cfg, L, Q, Kc, Kq, kbar128, tau, sel, ws, stream));
-  hsa::AttnArgs a = attn_args(cfg, Q, Kc, Vc, Kq, Vq);
+  hsa::AttnArgs a = attn_args(cfg, L, ws, Q, Kc, Vc, Kq, Vq);
+  // the work plan needs only the selection: it runs on a side stream beside the
+  // projection, joined before the attention
+  SideStream* side = nullptr;
+  cudaError_t e = side_stream(&side);
+  if (e == cudaSuccess) e = cudaEventRecord(side->fork, stream);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(side->s, side->fork, 0);
+  if (e != cudaSuccess) return fail(HSA_ERR_CUDA, "%s: side stream: %s", fn, cudaGetErrorString(e));
+  TRY(run_plan(L, sel, ws, a, side->s));
+  if ((e = cudaEventRecord(side->join, side->s)) != cudaSuccess)
+    return fail(HSA_ERR_CUDA, "%s: side stream: %s", fn, cudaGetErrorString(e));
   TRY(run_projection(cfg, L, Kc, Vc, Kq, Vq, E, F, ef_head_stride, ws, a, stream));
-  a.inter_idx = sel.inter_idx; a.inter_cnt = sel.inter_cnt; a.intra_idx = sel.intra_idx; a.intra_cnt = sel.intra_cnt;
+  if ((e = cudaStreamWaitEvent(stream, side->join, 0)) != cudaSuccess)
+    return fail(HSA_ERR_CUDA, "%s: side stream: %s", fn, cudaGetErrorString(e));
   a.gate_logit = gate_logit;
-  a.status = status_of(ws);
   if (out_is_bf16) a.out_bf16 = static_cast<uint16_t*>(out);
   else a.out_f32 = static_cast<float*>(out);
   HSA_LAUNCH("attention_merge", hsa::launch_attn_tc(a, stream));

@@ -4,11 +4,19 @@
 // news summary, HSA paragraph: exact attention over each head's kept blocks, a
 // low-rank linear global branch, learned gates merging the two).
 //
-// One CTA per (head, 128-query tile).  Its key tiles, in order:
-//   linear tiles  64 rows of EK / FV (split bf16 hi + lo), r / 64 of them;
+// One CTA per work unit (plan.cu): a segment of the key-tile list of one (head,
+// 128-query tile).  The list, in order:
+//   linear tiles  64 rows of EK / FV (split bf16 hi + lo), r / 64 of them, in
+//                 segment 0 only;
 //   cached tiles  one 128-row tile per kept inter block of the cached KV;
 //   chunk tiles   the union of the two 64-query halves' kept 64-row intra blocks,
 //                 each tagged with the halves that use it.
+// A segment takes the sparse tiles whose cumulative cost (2 per cached tile, 1 per
+// chunk tile) falls in its share of the list's cost.  A unit covering its whole
+// list writes the output; a segment of a split list writes its unnormalised O_s
+// with its running (max, sum) to a partial slot (segment 0 adds the weighted
+// linear branch), and the CTA that finishes the list's last segment merges the
+// slots in segment order.
 // 7 warps:
 //   warp 0      TMA producer of the Q tile (once) and of each key tile's K part
 //               (K, or EK_hi + EK_lo) into a 3-slot ring of 128-byte-swizzled
@@ -71,6 +79,24 @@ __device__ __forceinline__ int tc_tile_code(long long start, int type, int mask)
 __device__ __forceinline__ int tile_type(int code) { return (code >> 2) & 3; }
 __device__ __forceinline__ int tile_start(int code) { return code >> 4; }
 __device__ __forceinline__ int tile_rows(int code) { return tile_type(code) == kTileCached ? 128 : 64; }
+
+// 16 output values of row `grow`, head h, columns [16c, 16c + 16), fp32 or bf16.
+__device__ __forceinline__ void store_out16(const AttnArgs& a, int grow, int h, int D, int c, const float (&v)[16]) {
+  const long long idx = ((long long)grow * a.H + h) * D + c * 16;
+  if (a.out_bf16) {
+    uint4 w0, w1;
+    w0.x = pack_bf16x2(v[0], v[1]); w0.y = pack_bf16x2(v[2], v[3]);
+    w0.z = pack_bf16x2(v[4], v[5]); w0.w = pack_bf16x2(v[6], v[7]);
+    w1.x = pack_bf16x2(v[8], v[9]); w1.y = pack_bf16x2(v[10], v[11]);
+    w1.z = pack_bf16x2(v[12], v[13]); w1.w = pack_bf16x2(v[14], v[15]);
+    *reinterpret_cast<uint4*>(a.out_bf16 + idx) = w0;
+    *reinterpret_cast<uint4*>(a.out_bf16 + idx + 8) = w1;
+  } else {
+#pragma unroll
+    for (int k = 0; k < 16; k += 4)
+      *reinterpret_cast<float4*>(a.out_f32 + idx + k) = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+  }
+}
 
 // ------------------------------------------------------------------ kernel
 // Online-softmax step of one query row over one key tile of ROWS columns held in
@@ -186,10 +212,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __shared__ uint32_t s_tmem;
   __shared__ int s_ntiles;
 
+  __shared__ int s_last;
+
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int qb = blockIdx.x % nQ128, h = blockIdx.x / nQ128;
-  const int q0 = qb * 128;
   int* status = a.status;
+  const int HQ = a.H * nQ128;
+  const bool planned = a.units != nullptr;
+  // both loads in flight together (units[] holds the grid's max_units entries)
+  const int4 unit = planned ? a.units[blockIdx.x] : make_int4((int)blockIdx.x, 0, 1, -1);
+  const int n_units = planned ? *a.n_units : HQ;
+  if ((int)blockIdx.x >= n_units) return;  // spare CTA of the upper-bound grid
+  const int tq = unit.x, seg = unit.y, nseg = unit.z, slot0 = unit.w;
+  if (tq < 0 || tq >= HQ || nseg < 1 || seg < 0 || seg >= nseg ||
+      (nseg > 1 && (slot0 < 0 || slot0 + nseg > a.max_slots))) {
+    if (tid == 0) set_status(status, HSA_ERR_DEVICE);
+    return;
+  }
+  const int qb = tq % nQ128, h = tq / nQ128;
+  const int q0 = qb * 128;
 
   if (warp == 0) {
     tmem_alloc(&s_tmem, 512);
@@ -215,7 +255,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   // ---- key-tile list (linear tiles, cached tiles, chunk tiles).  Selection counts
   // and ids come from caller buffers: counts are clamped, out-of-range ids skipped.
-  const bool do_lin = a.EKhi != nullptr;
+  const bool any_lin = a.EKhi != nullptr;
+  const bool do_lin = any_lin && seg == 0;  // the linear tiles belong to segment 0
   const bool do_sparse = a.inter_cnt != nullptr;
   const int n_lin = do_lin ? a.r / 64 : 0;
   const int n_inter = do_sparse ? min(max(a.inter_cnt[(long long)h * nQ128 + qb], 0), nKc) : 0;
@@ -262,8 +303,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const int T = s_ntiles;
-  if (T == 0 && tid == 0) set_status(status, HSA_ERR_DEVICE);  // no key tile: selection buffers were empty
+  // this segment's share of the sparse tiles, by cost (a cached tile costs 2, a chunk tile 1)
+  const int n_chunk = s_ntiles - n_lin - n_inter;
+  const long long cost = 2LL * n_inter + n_chunk;
+  auto cut = [&](long long x) -> int {  // sparse tiles whose cumulative cost before them is < x
+    return x <= 2LL * n_inter ? (int)((x + 1) / 2) : n_inter + (int)(x - 2LL * n_inter);
+  };
+  const int t0 = cut(cost * seg / nseg), t1 = cut(cost * (seg + 1) / nseg);
+  const int T = n_lin + (t1 - t0);
+  // tile j of this unit: the linear tiles, then sparse tiles t0 .. t1 - 1
+  auto tile_at = [&](int j) -> int { return j < n_lin ? tiles[j] : tiles[j + t0]; };
+  if (T == 0 && nseg == 1 && tid == 0) set_status(status, HSA_ERR_DEVICE);  // no key tile: empty selection
   const uint32_t tmem = s_tmem;
   const uint32_t tOs = tmem + 256, tOl = tmem + 256 + D;
   constexpr int kHalfSlot = (D / 64) * 64 * 128;  // 64 rows x D bf16: hi part / lo part of a slot
@@ -280,7 +330,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int s = j % kKStages;
       if (!mbar_wait(&bar_k_empty[s], ((j / kKStages) & 1) ^ 1, status)) break;
       if (lane == 0) {
-        const int code = tiles[j];
+        const int code = tile_at(j);
         const int type = tile_type(code);
         const int rows = tile_rows(code);
         unsigned char* dK = sK + s * Lay::kKVBytes;
@@ -307,7 +357,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int s = j % kVStages;
       if (!mbar_wait(&bar_v_empty[s], ((j / kVStages) & 1) ^ 1, status)) break;
       if (lane == 0) {
-        const int code = tiles[j];
+        const int code = tile_at(j);
         const int type = tile_type(code);
         const int rows = tile_rows(code);
         unsigned char* dV = sV + s * Lay::kKVBytes;
@@ -338,7 +388,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!mbar_wait(&bar_k_full[s], (j / kKStages) & 1, status)) return false;
       tc_fence_after();
       if (lane == 0) {
-        const int code = tiles[j];
+        const int code = tile_at(j);
         const int rows = tile_rows(code);
         const uint32_t idesc = idesc_bf16(128, rows, false, false);
         const uint32_t k_base = smem_u32(sK + s * Lay::kKVBytes);
@@ -367,7 +417,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!mbar_wait(&bar_v_full[sv], (j / kVStages) & 1, status)) break;
       tc_fence_after();
       if (lane == 0) {
-        const int code = tiles[j];
+        const int code = tile_at(j);
         const int rows = tile_rows(code);
         const uint32_t idesc = idesc_bf16(128, D, false, true);
         const uint32_t v_base = smem_u32(sV + sv * Lay::kKVBytes);
@@ -412,7 +462,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         break;
       }
       tc_fence_after();
-      const int code = tiles[j];
+      const int code = tile_at(j);
       const int type = tile_type(code);
       const int rows = tile_rows(code);
       const long long nrows = type == kTileChunk ? (long long)a.Lq : a.Lc;
@@ -471,48 +521,60 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_before();
       mbar_arrive(&bar_p_full[b]);
     }
-    if (ok && T > 0 && mbar_wait_warp(&bar_o_done, (T - 1) & 1, status)) {
+    if (ok && (T == 0 || mbar_wait_warp(&bar_o_done, (T - 1) & 1, status))) {
       tc_fence_after();
       const int grow = q0 + row;
+      const bool valid_row = grow < a.Lq;
       // out = g o_s + (1 - g) o_l with g = sigmoid(gate logit) when both branches run
-      float ws = 0.f, wl = 0.f;
-      if (do_sparse && do_lin) {
-        const float g = a.gate_logit ? 1.f / (1.f + expf(-a.gate_logit[h])) : 1.f;
-        ws = g / ls;
-        wl = (1.f - g) / ll;
-      } else if (do_sparse) {
-        ws = 1.f / ls;
-      } else {
-        wl = 1.f / ll;
-      }
+      const float g = (do_sparse && any_lin && a.gate_logit) ? 1.f / (1.f + expf(-a.gate_logit[h])) : 1.f;
+      const float wl = do_lin ? (do_sparse ? 1.f - g : 1.f) / ll : 0.f;
+      if (nseg == 1) {
+        if (do_sparse && valid_row && !(ls > 0.f)) set_status(status, HSA_ERR_DEVICE);
+        const float ws = (do_sparse && ls > 0.f) ? g / ls : 0.f;
 #pragma unroll
-      for (int c = 0; c < D / 16; ++c) {
-        uint32_t rs[16], rl[16];
-        if (do_sparse) tmem_ld16_sync(tOs + loff + c * 16, rs);
-        if (do_lin) tmem_ld16_sync(tOl + loff + c * 16, rl);
-        if (grow < a.Lq) {
-          const long long idx = ((long long)grow * a.H + h) * D + c * 16;
-          float v[16];
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t rs[16], rl[16];
+          if (do_sparse) tmem_ld16_sync(tOs + loff + c * 16, rs);
+          if (do_lin) tmem_ld16_sync(tOl + loff + c * 16, rl);
+          if (valid_row) {
+            float v[16];
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const float vs = do_sparse ? __uint_as_float(rs[k]) * ws : 0.f;
-            const float vl = do_lin ? __uint_as_float(rl[k]) * wl : 0.f;
-            v[k] = vs + vl;
-          }
-          if (a.out_bf16) {
-            uint4 w0, w1;
-            w0.x = pack_bf16x2(v[0], v[1]); w0.y = pack_bf16x2(v[2], v[3]);
-            w0.z = pack_bf16x2(v[4], v[5]); w0.w = pack_bf16x2(v[6], v[7]);
-            w1.x = pack_bf16x2(v[8], v[9]); w1.y = pack_bf16x2(v[10], v[11]);
-            w1.z = pack_bf16x2(v[12], v[13]); w1.w = pack_bf16x2(v[14], v[15]);
-            *reinterpret_cast<uint4*>(a.out_bf16 + idx) = w0;
-            *reinterpret_cast<uint4*>(a.out_bf16 + idx + 8) = w1;
-          } else {
-#pragma unroll
-            for (int k = 0; k < 16; k += 4)
-              *reinterpret_cast<float4*>(a.out_f32 + idx + k) = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
+            for (int k = 0; k < 16; ++k) {
+              const float vs = do_sparse ? __uint_as_float(rs[k]) * ws : 0.f;
+              const float vl = do_lin ? __uint_as_float(rl[k]) * wl : 0.f;
+              v[k] = vs + vl;
+            }
+            store_out16(a, grow, h, D, c, v);
           }
         }
+      } else {
+        // one segment of a split list: unnormalised O_s and (max, sum); segment 0
+        // also leaves the weighted linear branch at the list's first slot
+        const int slot = slot0 + seg;
+        float* po = a.part_o + ((long long)slot * 128 + row) * D;
+        float* pl = a.part_lin + ((long long)slot0 * 128 + row) * D;
+        const bool had_sparse = T > n_lin;
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t rs[16], rl[16];
+          if (had_sparse) tmem_ld16_sync(tOs + loff + c * 16, rs);
+          if (do_lin) tmem_ld16_sync(tOl + loff + c * 16, rl);
+          if (valid_row) {
+#pragma unroll
+            for (int k = 0; k < 16; k += 4) {
+              *reinterpret_cast<float4*>(po + c * 16 + k) =
+                  had_sparse ? make_float4(__uint_as_float(rs[k]), __uint_as_float(rs[k + 1]),
+                                           __uint_as_float(rs[k + 2]), __uint_as_float(rs[k + 3]))
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+              if (do_lin)
+                *reinterpret_cast<float4*>(pl + c * 16 + k) =
+                    make_float4(__uint_as_float(rl[k]) * wl, __uint_as_float(rl[k + 1]) * wl,
+                                __uint_as_float(rl[k + 2]) * wl, __uint_as_float(rl[k + 3]) * wl);
+            }
+          }
+        }
+        if (valid_row) a.part_ml[(long long)slot * 128 + row] = make_float2(had_sparse && ls > 0.f ? ms : -INFINITY, ls);
+        __threadfence();
       }
     }
   }
@@ -521,6 +583,56 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+  if (nseg > 1) {
+    // the CTA that finishes a split list's last segment merges its segments, in
+    // segment order (which CTA that is does not change the result)
+    if (tid == 0) s_last = atomicAdd(&a.tile_done[tq], 1) == nseg - 1;
+    __syncthreads();
+    if (s_last && warp >= 2 && warp <= 5) {
+      __threadfence();
+      const int row = 32 * (warp & 3) + lane, grow = q0 + row;
+      if (grow < a.Lq) {
+        float M = -INFINITY;
+        for (int k = 0; k < nseg; ++k) M = fmaxf(M, __ldcg(&a.part_ml[(long long)(slot0 + k) * 128 + row]).x);
+        float L = 0.f;
+        for (int k = 0; k < nseg; ++k) {
+          const float2 m_l = __ldcg(&a.part_ml[(long long)(slot0 + k) * 128 + row]);
+          if (m_l.x != -INFINITY) L += m_l.y * exp2f(m_l.x - M);
+        }
+        if (!(L > 0.f)) set_status(status, HSA_ERR_DEVICE);
+        const float g = (any_lin && a.gate_logit) ? 1.f / (1.f + expf(-a.gate_logit[h])) : 1.f;
+        const float ws = L > 0.f ? g / L : 0.f;
+        const float* pl = a.part_lin + ((long long)slot0 * 128 + row) * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 16; ++c) {
+          float v[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) v[k] = 0.f;
+          for (int sg = 0; sg < nseg; ++sg) {
+            const float m_s = __ldcg(&a.part_ml[(long long)(slot0 + sg) * 128 + row]).x;
+            if (m_s == -INFINITY) continue;  // no tile of this segment reaches the row
+            const float w = exp2f(m_s - M);
+            const float* po = a.part_o + ((long long)(slot0 + sg) * 128 + row) * D + c * 16;
+#pragma unroll
+            for (int k = 0; k < 16; k += 4) {
+              const float4 o4 = __ldcg(reinterpret_cast<const float4*>(po + k));
+              v[k] += o4.x * w; v[k + 1] += o4.y * w; v[k + 2] += o4.z * w; v[k + 3] += o4.w * w;
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < 16; ++k) v[k] *= ws;
+          if (any_lin) {
+#pragma unroll
+            for (int k = 0; k < 16; k += 4) {
+              const float4 l4 = __ldcg(reinterpret_cast<const float4*>(pl + c * 16 + k));
+              v[k] += l4.x; v[k + 1] += l4.y; v[k + 2] += l4.z; v[k + 3] += l4.w;
+            }
+          }
+          store_out16(a, grow, h, D, c, v);
+        }
+      }
+    }
   }
 }
 
@@ -577,7 +689,8 @@ cudaError_t launch_tc(const AttnArgs& a, cudaStream_t s) {
   if (smem > 232448) return cudaErrorInvalidConfiguration;
   e = cudaFuncSetAttribute(sparse_attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  sparse_attn_tc_kernel<D><<<a.H * nQ128, kTcThreads, smem, s>>>(maps, a, nQ128, nKc, nQ64, nKq);
+  const int grid = a.units ? a.max_units : a.H * nQ128;
+  sparse_attn_tc_kernel<D><<<grid, kTcThreads, smem, s>>>(maps, a, nQ128, nKc, nQ64, nKq);
   return cudaGetLastError();
 }
 

@@ -39,7 +39,15 @@ cudaError_t launch_block_select(const float* q128, const float* kc128, const flo
                                 int32_t* inter_idx, int32_t* inter_cnt, int32_t* intra_idx, int32_t* intra_cnt,
                                 cudaStream_t s);
 
-// ---------------------------------------------------------------- attn_tc.cu
+// ---------------------------------------------------------------- attn_tc.cu / plan.cu
+// The attention kernel runs one CTA per work unit: a segment of the key-tile list
+// of one (head, 128-query tile).  Lists longer than a segment length are cut into
+// segments of similar length; the CTA that finishes a list's last segment merges
+// the segments' partial results (plan.cu chooses the segments).
+constexpr int kPlanSMs = 148;        // units are sized for this many SMs ...
+constexpr int kPlanUnitsPerSM = 1;   // ... and lists above the cost per SM are split
+constexpr int kPlanMinSegment = 16;  // shortest segment worth a unit of its own
+
 struct AttnArgs {
   const uint16_t* Q;
   const uint16_t* Kc;
@@ -66,9 +74,23 @@ struct AttnArgs {
   float* out_f32;
   uint16_t* out_bf16;
   int* status;  // workspace status word (may be NULL)
+  // work plan (workspace; sparse branch only -- without it, unit u is query tile u whole)
+  int max_units;     // capacity of units (grid size of the attention launch)
+  int max_slots;     // capacity of the partial-result slots
+  int4* units;       // [max_units] (head * nQ128 + query tile, segment, segments, first slot)
+  int* n_units;      // number of units
+  int* tile_done;    // [H * nQ128] segments finished (zeroed by the plan)
+  float* part_o;     // [max_slots][128][d] unnormalised O_s of a segment
+  float2* part_ml;   // [max_slots][128] running max (log2 units) and sum of a segment
+  float* part_lin;   // [max_slots][128][d] weighted linear branch of a split list (at its first slot)
 };
 // Sparse and/or linear branch with the gated merge, on tcgen05 / TMEM / TMA.
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s);
+// The work plan over the selection (plan.cu): one CTA.
+cudaError_t launch_attn_plan(const AttnArgs& a, cudaStream_t s);
+// Capacities used by the workspace layout.
+inline int plan_max_units(int H, int nQ128) { return H * nQ128 + kPlanSMs * kPlanUnitsPerSM + 1; }
+inline int plan_max_slots() { return 2 * kPlanSMs * kPlanUnitsPerSM + 2; }
 
 // ---------------------------------------------------------------- proj.cu
 int proj_splits(int H, int r, long long L);

@@ -12,9 +12,19 @@
 namespace hsa {
 namespace sm100 {
 
-// A wait on an mbarrier gives up after this many polls (each poll suspends the
-// thread for a hardware-chosen time), records HSA_ERR_TIMEOUT and returns false.
-constexpr uint32_t kSpinLimit = 1u << 26;
+// A thread waiting on an mbarrier sleeps in the hardware until the phase completes
+// (or kSuspendNs pass) instead of polling shared memory, which the tensor cores'
+// operand reads keep busy.  A wait gives up after kWaitLimitNs, records
+// HSA_ERR_TIMEOUT and returns false.
+constexpr uint32_t kSuspendNs = 1000000u;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr uint32_t kSpinLimit = 1u << 24;  // polls of a wait without the sleep hint
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -38,10 +48,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
+      : "memory");
+  return ok != 0;
+}
 // Bounded wait for the phase with the given parity to complete.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
+#ifdef HSA_WAIT_POLL
   for (uint32_t i = 0; i < kSpinLimit; ++i)
     if (mbar_try_wait(bar, parity)) return true;
+#else
+  if (mbar_try_wait_sleep(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  do {
+    if (mbar_try_wait_sleep(bar, parity)) return true;
+  } while (global_ns() - t0 < kWaitLimitNs);
+#endif
   set_status(status, HSA_ERR_TIMEOUT);
   return false;
 }
@@ -247,6 +274,23 @@ __device__ __forceinline__ float ex2_approx(float x) {
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Move registers between the warpgroups of a CTA (every thread of a warpgroup
+// executes the same one).  The sum over warpgroups must stay within the registers
+// the CTA was launched with (threads x registers per thread at launch).
+template <uint32_t N>
+__device__ __forceinline__ void regs_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// Barrier `id` (1..15) over `n` threads of the CTA (a multiple of 32).
+__device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
 
 __device__ __forceinline__ bool elect_one() {
   uint32_t pred = 0;

@@ -275,3 +275,32 @@ def test_invalid_arguments_launch_nothing():
     assert e.value.code == 2
     torch.cuda.synchronize()
     assert torch.count_nonzero(out) == 0
+
+
+def test_forward_split_lists_merge():
+    """Lists much longer than the step's cost per SM are cut into segments whose
+    partial results are merged in segment order: same output as the oracle, and the
+    same bits on a second run."""
+    shape = synth.StepShape("h2_d128_lq200_lc8192", H=2, d=128, frames=1, F_tok=200, page_frames=1,
+                            page_tok=1024, NP=10, Kp=8, r=64)
+    ds = DeviceStep(shape, 91)
+    try:
+        hsa.hsa_status_clear(ds.step.ws)
+        ds.run()
+        torch.cuda.synchronize()
+        x, st = ds.x, ds.step
+        first = st.out.clone()
+        ds.run()
+        torch.cuda.synchronize()
+        assert torch.equal(first, st.out)
+        Kc, Vc = bits_of(st.Kc), bits_of(st.Vc)
+        sb = st.selection
+        inter_cnt = sb.inter_cnt.cpu().numpy()
+        assert inter_cnt[0].min() == Kc.shape[0] // 128  # tau = 1 keeps every cached block: long lists
+        sel = oracle.Selection(selection_lists(sb.inter_idx.cpu().numpy(), inter_cnt),
+                               selection_lists(sb.intra_idx.cpu().numpy(), sb.intra_cnt.cpu().numpy()), None, None)
+        ref = oracle.hsa_step(x.Q, Kc, Vc, x.Kq, x.Vq, x.tau, x.z, x.E, x.F, selection=sel)
+        assert_close(st.out.cpu().numpy(), ref["out"], "hsa_forward out (split lists)")
+        assert hsa.hsa_status_read(ds.step.ws) == 0
+    finally:
+        ds.close()
