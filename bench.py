@@ -35,7 +35,12 @@ DEFAULT_WORKLOAD = 1
 # section marker to the next one) is unchanged (sha256 prefix of the section).
 TRAFFIC = {
     # profiles/gather_and_projection_hbm_wan1.3b_480p.md
-    "gather": {"file": "hkv.cu", "section": "gather", "sha": "ea6010aad5d6ab04", "bytes": 306762240 + 251291392},
+    "gather": {"file": "hkv.cu", "section": "gather", "sha": "ea6010aad5d6ab04", "bytes": 306733056 + 251928320},
+    "linformer_proj": {"file": "proj_tc.cu", "section": "kernel", "sha": "083e8f5fb32f84a9",
+                       "bytes": 392173312 + 6182656},
+    # profiles/sparse_attn_tc_wan1.3b_480p.md
+    "attention_merge": {"file": "attn_tc.cu", "section": "kernel", "sha": "6cfb3e60052e490f",
+                        "bytes": 276799744 + 19160832},
 }
 
 
@@ -403,6 +408,10 @@ def run_gpu(args, shape, rank, world, local):
             else:
                 ach = work / (avg_ms / 1e3) / 1e9
                 entry.update({"bound": "hbm", "achieved": ach, "unit": "GB/s", "frac": ach / peaks["hbm_gbs"]})
+        tr = TRAFFIC.get(name)
+        if tr and tr["sha"] == section_sha(os.path.join(ROOT, "hybrid_sparse_attention_hkv_b200", "csrc", tr["file"]),
+                                           tr["section"]):
+            entry["traffic"] = tr["bytes"]
         kernels[name] = entry
     dom = max(kernels, key=lambda k: kernels[k]["share"])
     de = kernels[dom]
