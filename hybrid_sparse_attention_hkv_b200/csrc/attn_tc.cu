@@ -194,6 +194,29 @@ __device__ __forceinline__ void softmax_tile_split(const uint32_t (&sr)[64], flo
   l = l * alpha + (st.x + st.y);
 }
 
+// MMA issue with every loop unrolled at compile time: the descriptors of one tile
+// are its base descriptor plus constant address offsets (in 16-byte units, the
+// descriptor's low field), so consecutive MMAs issue back to back.
+// S (+)= Q K^T over D / 16 steps of 16; K tile of ROWS rows (K-major, 128-byte swizzle).
+template <int D, int ROWS>
+__device__ __forceinline__ void issue_qk(uint32_t tS, uint64_t qd, uint64_t kd, bool accumulate_first) {
+  constexpr uint32_t idesc = idesc_bf16(128, ROWS, false, false);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint64_t qo = (uint64_t)(((kk / 4) * kRegionBytes + (kk % 4) * 32) >> 4);
+    const uint64_t ko = (uint64_t)(((kk / 4) * (ROWS * 128) + (kk % 4) * 32) >> 4);
+    mma_ss(tS, qd + qo, kd + ko, idesc, (accumulate_first || kk > 0) ? 1u : 0u);
+  }
+}
+// O (+)= P V over ROWS / 16 steps; P from TMEM, V tile of ROWS rows (MN-major).
+template <int D, int ROWS>
+__device__ __forceinline__ void issue_pv(uint32_t tO, uint32_t tP, uint64_t vd, bool accumulate_first) {
+  constexpr uint32_t idesc = idesc_bf16(128, D, false, true);
+#pragma unroll
+  for (int kk = 0; kk < ROWS / 16; ++kk)
+    mma_ts(tO, tP + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc, (accumulate_first || kk > 0) ? 1u : 0u);
+}
+
 template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1)
     sparse_attn_tc_kernel(const __grid_constant__ TcMaps maps, const AttnArgs a, int nQ128, int nKc, int nQ64,
@@ -382,26 +405,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     bool ok = mbar_wait_warp(&bar_q, 0, status);
     tc_fence_after();
-    const uint32_t q_base = smem_u32(sQ);
+    const uint64_t qd = sdesc_sw128(smem_u32(sQ), 16, 1024);
     auto issue_s = [&](int j) -> bool {
       const int s = j % kKStages;
       if (!mbar_wait(&bar_k_full[s], (j / kKStages) & 1, status)) return false;
       tc_fence_after();
       if (lane == 0) {
         const int code = tile_at(j);
-        const int rows = tile_rows(code);
-        const uint32_t idesc = idesc_bf16(128, rows, false, false);
-        const uint32_t k_base = smem_u32(sK + s * Lay::kKVBytes);
+        const uint64_t kd = sdesc_sw128(smem_u32(sK + s * Lay::kKVBytes), 16, 1024);
         const uint32_t tS = tmem + (j & 1) * 128;
-        const int parts = tile_type(code) == kTileLinear ? 2 : 1;  // EK_hi then EK_lo
-        for (int part = 0; part < parts; ++part) {
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t qa = q_base + (kk / 4) * kRegionBytes + (kk % 4) * 32;
-            const uint32_t ka = k_base + part * kHalfSlot + (kk / 4) * (rows * 128) + (kk % 4) * 32;
-            mma_ss(tS, sdesc_sw128(qa, 16, 1024), sdesc_sw128(ka, 16, 1024), idesc,
-                   (part > 0 || kk > 0) ? 1u : 0u);
-          }
+        if (tile_type(code) == kTileLinear) {  // EK_hi then EK_lo, 64 rows each
+          issue_qk<D, 64>(tS, qd, kd, false);
+          issue_qk<D, 64>(tS, qd, kd + (uint64_t)(kHalfSlot >> 4), true);
+        } else if (tile_rows(code) == 128) {
+          issue_qk<D, 128>(tS, qd, kd, false);
+        } else {
+          issue_qk<D, 64>(tS, qd, kd, false);
         }
         mma_commit(&bar_k_empty[s]);
         mma_commit(&bar_s_full[j & 1]);
@@ -418,27 +437,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_after();
       if (lane == 0) {
         const int code = tile_at(j);
-        const int rows = tile_rows(code);
-        const uint32_t idesc = idesc_bf16(128, D, false, true);
         const uint32_t v_base = smem_u32(sV + sv * Lay::kKVBytes);
         const uint32_t tP = tmem + (j & 1) * 128;
         if (tile_type(code) == kTileLinear) {
           // O_l += P_hi FV_hi + P_lo FV_hi + P_hi FV_lo; first linear tile initialises O_l
-          const bool first = j == 0;
-#pragma unroll
-          for (int term = 0; term < 3; ++term) {
-            const uint32_t pa = tP + (term == 1 ? 32 : 0);
-            const uint32_t vb = v_base + (term == 2 ? kHalfSlot : 0);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_ts(tOl, pa + kk * 8, sdesc_sw128(vb + kk * 2048, 64 * 128, 1024), idesc,
-                     (!first || term > 0 || kk > 0) ? 1u : 0u);
-          }
+          const uint64_t vhi = sdesc_sw128(v_base, 64 * 128, 1024);
+          const uint64_t vlo = sdesc_sw128(v_base + kHalfSlot, 64 * 128, 1024);
+          issue_pv<D, 64>(tOl, tP, vhi, j > 0);
+          issue_pv<D, 64>(tOl, tP + 32, vhi, true);
+          issue_pv<D, 64>(tOl, tP, vlo, true);
+        } else if (tile_rows(code) == 128) {  // the first sparse tile initialises O_s
+          issue_pv<D, 128>(tOs, tP, sdesc_sw128(v_base, 128 * 128, 1024), j > n_lin);
         } else {
-          const bool first = j == n_lin;  // first sparse tile initialises O_s
-          for (int kk = 0; kk < rows / 16; ++kk)
-            mma_ts(tOs, tP + kk * 8, sdesc_sw128(v_base + kk * 2048, rows * 128, 1024), idesc,
-                   (!first || kk > 0) ? 1u : 0u);
+          issue_pv<D, 64>(tOs, tP, sdesc_sw128(v_base, 64 * 128, 1024), j > n_lin);
         }
         mma_commit(&bar_v_empty[sv]);
         mma_commit(&bar_o_done);
