@@ -104,15 +104,25 @@ __device__ __forceinline__ void store_out16(const AttnArgs& a, int grow, int h, 
 // than 2^8, returning the factor alpha for O), write P = 2^(s*sl2 - m) as packed
 // bf16 pairs over the first ROWS/2 columns of the S buffer, and fold the row sum
 // into l.  MASKED: only the first `valid` keys exist.
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 template <int ROWS, bool MASKED>
 __device__ __forceinline__ void softmax_tile(const uint32_t (&sr)[128], int valid, float sl2, float& m, float& l,
                                              float& alpha, bool& rescale, uint32_t tS) {
   float pm[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) pm[q] = -INFINITY;
+  if (MASKED) {
 #pragma unroll
-  for (int k = 0; k < ROWS; ++k)
-    if (!MASKED || k < valid) pm[k & 7] = fmaxf(pm[k & 7], __uint_as_float(sr[k]));
+    for (int k = 0; k < ROWS; ++k)
+      if (k < valid) pm[k & 7] = fmaxf(pm[k & 7], __uint_as_float(sr[k]));
+  } else {
+#pragma unroll
+    for (int k = 0; k < ROWS; k += 2) pm[(k >> 1) & 7] = fmax3f(pm[(k >> 1) & 7], __uint_as_float(sr[k]), __uint_as_float(sr[k + 1]));
+  }
   const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
   const float mn = mx * sl2;
   if (mn > m + 8.f) {
@@ -133,7 +143,17 @@ __device__ __forceinline__ void softmax_tile(const uint32_t (&sr)[128], int vali
     for (int k = 0; k < 16; ++k) {
       const int i = c * 32 + 2 * k;
       const float2 t = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), a2, b2);
-      float p0 = ex2_approx(t.x), p1 = ex2_approx(t.y);
+      float p0, p1;
+      // a quarter of the pairs on the FMA pipe (ex2_poly2), the rest on the SFU: the
+      // softmax, not the tensor core, bounds the tile rate, and the SFU is its busiest unit
+      if (!MASKED && ((k & 7) == 3 || (k & 7) == 6)) {
+        const float2 e = ex2_poly2(t);
+        p0 = e.x;
+        p1 = e.y;
+      } else {
+        p0 = ex2_approx(t.x);
+        p1 = ex2_approx(t.y);
+      }
       if (MASKED) {
         if (i >= valid) p0 = 0.f;
         if (i + 1 >= valid) p1 = 0.f;
@@ -509,15 +529,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (c * 32 < rows) tmem_st16(tS + c * 16, zero);
       }
       tmem_st_wait();
-      // O holds the P.V products of tiles 0..j-1 once the previous one has completed
-      if (j > 0) {
-        if (!mbar_wait(&bar_o_done, (j - 1) & 1, status)) {
+      if (__any_sync(0xffffffffu, rescale)) {
+        // O holds the P.V products of tiles 0..j-1 once the last of them has completed
+        // (P.V of tile j cannot have started: it waits for this P).  Without a rescale
+        // nothing here touches O, and the wait is skipped.
+        if (j > 0 && !mbar_wait(&bar_o_done, (j - 1) & 1, status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-      }
-      if (__any_sync(0xffffffffu, rescale)) {
         const uint32_t tO = type == kTileLinear ? tOl : tOs;
 #pragma unroll
         for (int c = 0; c < D / 16; ++c) {
