@@ -392,7 +392,7 @@ def run_gpu(args, shape, rank, world, local):
         "linformer_proj": ("tensor", w["proj_flops"]),
         "gather": ("hbm", w["gather_bytes"]),
         "pool": ("hbm", w["pool_bytes"]),
-        "colsum_partial": ("hbm", w["select_pages_bytes"]),
+        "page_scores_partial": ("hbm", w["select_pages_bytes"]),
     }
     kernels = {}
     for name, d in per_kernel.items():

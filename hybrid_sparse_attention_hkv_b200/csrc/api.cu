@@ -303,15 +303,17 @@ hsa_status_t hkv_select_pages(const float* kbar_pages, int NP, const int32_t* ca
   if (Kp < 1 || Kp > NP || Kp > 64) return fail(HSA_ERR_INVALID_ARG, "%s: Kp = %d must be in [1, min(NP, 64)]", fn, Kp);
   if ((size_t)H * d * 8 + (size_t)NP * 8 > 200 * 1024)
     return fail(HSA_ERR_UNSUPPORTED, "%s: H*d*8 + NP*8 bytes exceed the shared-memory budget", fn);
+  if (NP > H * d) return fail(HSA_ERR_UNSUPPORTED, "%s: NP = %d pages exceed H*d = %d", fn, NP, H * d);
   REQUIRE_PTR(kbar_pages);
   REQUIRE_PTR(Q);
   if (!sel_out) return fail(HSA_ERR_INVALID_ARG, "%s: sel_out is NULL", fn);
   const Layout L = make_layout(H, d, 1, 0, 0);
   TRY(check_ws(fn, ws, ws_bytes, L.pages_end));
   float* part = at<float>(ws, L.colpart);
-  HSA_LAUNCH("colsum_partial", hsa::launch_colsum_partial(Q, Lq, H * d, part, stream));
-  HSA_LAUNCH("select_pages_final", hsa::launch_select_pages_final(part, Lq, H * d, kbar_pages, NP, cand_range, Kp,
-                                                                  sel_out, scores_out, status_of(ws), stream));
+  HSA_LAUNCH("page_scores_partial", hsa::launch_page_scores_partial(Q, Lq, H * d, kbar_pages, NP, cand_range, part,
+                                                                    stream));
+  HSA_LAUNCH("select_pages_final", hsa::launch_select_pages_final(part, Lq, NP, cand_range, Kp, sel_out, scores_out,
+                                                                  status_of(ws), stream));
   return HSA_OK;
 }
 

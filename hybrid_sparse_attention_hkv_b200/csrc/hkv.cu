@@ -5,7 +5,6 @@
 // All of these are HBM (or host-link) bound: they stream bf16 rows once with
 // 16-byte vector loads, one thread per 16-byte column chunk, and reduce in fp32
 // in a fixed order (deterministic results).
-#include <cooperative_groups.h>
 #include <float.h>
 
 #include "common.cuh"
@@ -92,116 +91,159 @@ cudaError_t launch_page_summary_final(const float* part, long long n, int C, flo
 }
 
 // ------------------------------------------------------------------ page-level retrieval
-// One 8-CTA cluster.  CTA k sums the column partials of row splits k, k+8, ... into
-// its shared memory; CTA 0 then reads the eight partial vectors over distributed
-// shared memory in a fixed order (deterministic), forms qbar = column means of Q,
-// scores s_p = qbar . kbar_p for the candidates and keeps the top Kp (ties -> lower
-// page id), written ascending.
-constexpr int kSelCluster = 8;
+// s_p = qbar . kbar_p with qbar the column mean of Q.  Pass 1 splits Q's rows over
+// many CTAs; each CTA sums its rows' columns in shared memory and dots that sum
+// with every candidate page's kbar, writing one partial score per page.  Pass 2
+// (one CTA) adds the partials in split order, divides by Lq, ranks the candidates
+// (ties -> lower page id) and writes the top Kp ascending.  Both passes reduce in
+// a fixed order (deterministic).
+constexpr int kScoreThreads = 256;
 
-__global__ void __cluster_dims__(kSelCluster, 1, 1) __launch_bounds__(1024) select_pages_final_kernel(
-    const float* __restrict__ part, int splits, long long Lq, int C, const float* __restrict__ kbar, int NP,
-    const int32_t* __restrict__ cand_range, int Kp, int32_t* __restrict__ sel_out, float* __restrict__ scores_out,
-    int* status) {
-  namespace cg = cooperative_groups;
-  cg::cluster_group cluster = cg::this_cluster();
-  const int rank = (int)cluster.block_rank();
-  extern __shared__ float sm[];
-  float* qpart = sm;            // [C] this CTA's share of the split sums
-  float* qbar = sm + C;         // [C] (CTA 0)
-  float* score = qbar + C;      // [NP] (CTA 0)
-  int* taken = reinterpret_cast<int*>(score + NP);  // [NP] (CTA 0)
-  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32, nwarps = blockDim.x / 32;
-  for (int c = tid; c < C; c += blockDim.x) {
-    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-    int q = rank;
-    for (; q + 3 * kSelCluster < splits; q += 4 * kSelCluster) {
-      a0 += part[(long long)q * C + c];
-      a1 += part[(long long)(q + kSelCluster) * C + c];
-      a2 += part[(long long)(q + 2 * kSelCluster) * C + c];
-      a3 += part[(long long)(q + 3 * kSelCluster) * C + c];
-    }
-    for (; q < splits; q += kSelCluster) a0 += part[(long long)q * C + c];
-    qpart[c] = (a0 + a1) + (a2 + a3);
-  }
-  cluster.sync();
-  if (rank == 0) {
-    for (int c = tid; c < C; c += blockDim.x) {
-      float t = 0.f;
-      for (int k = 0; k < kSelCluster; ++k) t += cluster.map_shared_rank(qpart, k)[c];
-      qbar[c] = t / (float)Lq;
-    }
-  }
-  cluster.sync();  // the other CTAs' shared memory stays valid until CTA 0 has read it
-  if (rank != 0) return;
+int page_score_splits(long long Lq) {
+  long long s = (Lq + 15) / 16;  // at least 16 rows per split
+  return (int)(s < 1 ? 1 : (s > kColMaxSplits ? kColMaxSplits : s));
+}
 
+__global__ void __launch_bounds__(kScoreThreads) page_scores_partial_kernel(
+    const uint16_t* __restrict__ Q, long long Lq, int C, long long rows_per_split, const float* __restrict__ kbar,
+    int NP, const int32_t* __restrict__ cand_range, float* __restrict__ part) {
+  extern __shared__ float colsum[];  // [C]
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const long long r0 = (long long)blockIdx.x * rows_per_split;
+  const long long r1 = min(Lq, r0 + rows_per_split);
+  for (int v = tid; v < C / 8; v += kScoreThreads) {
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    long long r = r0;
+    for (; r + 16 <= r1; r += 16) {  // 16 loads in flight
+      uint4 w[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) w[k] = ld_nc_v4(Q + (r + k) * C + v * 8);
+      asm volatile("" ::: "memory");  // keep the batch of loads ahead of their uses
+#pragma unroll
+      for (int k = 0; k < 16; ++k) add8(acc, w[k]);
+    }
+    for (; r < r1; ++r) add8(acc, ld_nc_v4(Q + r * C + v * 8));
+#pragma unroll
+    for (int k = 0; k < 8; ++k) colsum[v * 8 + k] = acc[k];
+  }
+  __syncthreads();
+  int first = 0, end = NP;
+  if (cand_range) {
+    first = max(cand_range[0], 0);
+    end = min(cand_range[1], NP);
+  }
+  float* out = part + (long long)blockIdx.x * NP;
+  for (int p = first + warp; p < end; p += kScoreThreads / 32) {
+    const float* kb = kbar + (long long)p * C;
+    float sacc = 0.f;
+    constexpr int kBatch = 8;  // float4 loads in flight per lane
+    for (int c0 = lane * 4; c0 < C; c0 += 128 * kBatch) {
+      float4 k4[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int c = c0 + u * 128;
+        k4[u] = c < C ? __ldg(reinterpret_cast<const float4*>(kb + c)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      asm volatile("" ::: "memory");  // keep the batch of loads ahead of their uses
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int c = c0 + u * 128;
+        if (c < C) {
+          sacc = fmaf(colsum[c], k4[u].x, sacc);
+          sacc = fmaf(colsum[c + 1], k4[u].y, sacc);
+          sacc = fmaf(colsum[c + 2], k4[u].z, sacc);
+          sacc = fmaf(colsum[c + 3], k4[u].w, sacc);
+        }
+      }
+    }
+    sacc = warp_sum(sacc);
+    if (lane == 0) out[p] = sacc;
+  }
+}
+
+constexpr int kFinalThreads = 1024;
+
+__global__ void __launch_bounds__(kFinalThreads) select_pages_final_kernel(
+    const float* __restrict__ part, int splits, long long Lq, int NP, const int32_t* __restrict__ cand_range,
+    int Kp, int32_t* __restrict__ sel_out, float* __restrict__ scores_out, int* status) {
+  extern __shared__ float score[];  // [NP]
+  __shared__ int warp_cnt[kFinalThreads / 32];
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   int first = 0, end = NP;
   if (cand_range) {
     first = cand_range[0];
     end = cand_range[1];
   }
-  const bool bad = first < 0 || end > NP || end - first < Kp;
-  for (int p = tid; p < NP; p += blockDim.x) {
-    score[p] = -INFINITY;
-    taken[p] = 0;
-  }
-  __syncthreads();
-  if (bad) {
+  if (first < 0 || end > NP || end - first < Kp) {
     if (tid == 0) set_status(status, HSA_ERR_DEVICE);
-    for (int k = tid; k < Kp; k += blockDim.x) sel_out[k] = -1;
+    for (int k = tid; k < Kp; k += kFinalThreads) sel_out[k] = -1;
     if (scores_out)
-      for (int p = tid; p < NP; p += blockDim.x) scores_out[p] = -INFINITY;
+      for (int p = tid; p < NP; p += kFinalThreads) scores_out[p] = -INFINITY;
     return;
   }
-  for (int p = first + warp; p < end; p += nwarps) {
-    const float* kb = kbar + (long long)p * C;
-    float s = 0.f;
-    for (int c = lane; c < C; c += 32) s = fmaf(qbar[c], kb[c], s);
-    s = warp_sum(s);
-    if (lane == 0) score[p] = s;
+  for (int p = warp; p < NP; p += kFinalThreads / 32) {
+    float sacc = 0.f;
+    if (p >= first && p < end)
+      for (int q = lane; q < splits; q += 32) sacc += part[(long long)q * NP + p];
+    sacc = warp_sum(sacc);
+    if (lane == 0) score[p] = (p >= first && p < end) ? sacc / (float)Lq : -INFINITY;
   }
   __syncthreads();
   if (scores_out)
-    for (int p = tid; p < NP; p += blockDim.x) scores_out[p] = score[p];
-  if (tid == 0) {
-    int chosen[64];
-    int nchosen = 0;
-    for (int k = 0; k < Kp; ++k) {
-      int best = -1;
-      float bv = -INFINITY;
-      for (int p = first; p < end; ++p) {
-        if (taken[p]) continue;
-        if (best < 0 || score[p] > bv) {  // strict: a tie keeps the lower page id
-          best = p;
-          bv = score[p];
-        }
+    for (int p = tid; p < NP; p += kFinalThreads) scores_out[p] = score[p];
+  // a candidate is kept when fewer than Kp candidates rank before it
+  int base = 0;
+  for (int p0 = 0; p0 < NP; p0 += kFinalThreads) {
+    const int p = p0 + tid;
+    bool keep = false;
+    if (p >= first && p < end) {
+      const float sp = score[p];
+      int rank = 0;
+      for (int q = first; q < end && rank < Kp; ++q) {
+        const float sq = score[q];
+        rank += (sq > sp) || (sq == sp && q < p);
       }
-      taken[best] = 1;
-      if (nchosen < 64) chosen[nchosen++] = best;
+      keep = rank < Kp;
     }
-    for (int a = 1; a < nchosen; ++a) {  // ascending page order (insertion sort, Kp <= 64)
-      int v = chosen[a], b = a - 1;
-      while (b >= 0 && chosen[b] > v) {
-        chosen[b + 1] = chosen[b];
-        --b;
-      }
-      chosen[b + 1] = v;
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    if (lane == 0) warp_cnt[warp] = __popc(bal);
+    __syncthreads();
+    int before = base;
+    for (int w = 0; w < warp; ++w) before += warp_cnt[w];
+    if (keep) {
+      const int pos = before + __popc(bal & ((1u << lane) - 1u));
+      if (pos < Kp) sel_out[pos] = p;
     }
-    for (int k = 0; k < nchosen; ++k) sel_out[k] = chosen[k];
+    __syncthreads();
+    for (int w = 0; w < kFinalThreads / 32; ++w) base += warp_cnt[w];
+    __syncthreads();
   }
 }
 
-cudaError_t launch_select_pages_final(const float* part, long long Lq, int C, const float* kbar_pages, int NP,
-                                      const int32_t* cand_range, int Kp, int32_t* sel_out, float* scores_out,
-                                      int* status, cudaStream_t s) {
-  size_t smem = (size_t)C * 8 + (size_t)NP * 8;
+cudaError_t launch_page_scores_partial(const uint16_t* Q, long long Lq, int C, const float* kbar_pages, int NP,
+                                       const int32_t* cand_range, float* part, cudaStream_t s) {
+  const int splits = page_score_splits(Lq);
+  const long long rps = (Lq + splits - 1) / splits;
+  const size_t smem = (size_t)C * 4;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(page_scores_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  page_scores_partial_kernel<<<splits, kScoreThreads, smem, s>>>(Q, Lq, C, rps, kbar_pages, NP, cand_range, part);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_pages_final(const float* part, long long Lq, int NP, const int32_t* cand_range, int Kp,
+                                      int32_t* sel_out, float* scores_out, int* status, cudaStream_t s) {
+  const size_t smem = (size_t)NP * 4;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(select_pages_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
   }
-  select_pages_final_kernel<<<kSelCluster, 1024, smem, s>>>(part, colsum_splits(Lq), Lq, C, kbar_pages, NP,
-                                                             cand_range, Kp, sel_out, scores_out, status);
+  select_pages_final_kernel<<<1, kFinalThreads, smem, s>>>(part, page_score_splits(Lq), Lq, NP, cand_range, Kp,
+                                                           sel_out, scores_out, status);
   return cudaGetLastError();
 }
 

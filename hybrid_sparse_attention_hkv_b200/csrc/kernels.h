@@ -19,9 +19,13 @@ constexpr int kColMaxSplits = 296;  // 2 CTAs per SM for the column-sum partial 
 int colsum_splits(long long n);  // number of row splits used for n rows
 cudaError_t launch_colsum_partial(const uint16_t* X, long long n, int C, float* part, cudaStream_t s);
 cudaError_t launch_page_summary_final(const float* part, long long n, int C, float* kbar, cudaStream_t s);
-cudaError_t launch_select_pages_final(const float* part, long long Lq, int C, const float* kbar_pages, int NP,
-                                      const int32_t* cand_range, int Kp, int32_t* sel_out, float* scores_out,
-                                      int* status, cudaStream_t s);
+// Page-level retrieval: partial scores per row split of Q (pass 1), then one CTA
+// adds them, ranks the candidates and writes the top Kp ascending (pass 2).
+int page_score_splits(long long Lq);  // row splits of pass 1 (<= kColMaxSplits)
+cudaError_t launch_page_scores_partial(const uint16_t* Q, long long Lq, int C, const float* kbar_pages, int NP,
+                                       const int32_t* cand_range, float* part, cudaStream_t s);
+cudaError_t launch_select_pages_final(const float* part, long long Lq, int NP, const int32_t* cand_range, int Kp,
+                                      int32_t* sel_out, float* scores_out, int* status, cudaStream_t s);
 cudaError_t launch_select_prompt(const float* e_cur, const float* e_seg, int n_seg, int dim,
                                  const int32_t* seg_begin, int32_t* seg_out, int32_t* cand_range_out,
                                  cudaStream_t s);

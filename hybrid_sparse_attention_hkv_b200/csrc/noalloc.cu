@@ -63,6 +63,7 @@ extern "C" hsa_status_t hkv_select_pages_noalloc(const float* kbar_pages, int NP
     return hsa::api_fail(HSA_ERR_INVALID_ARG, "%s: Kp = %d must be in [1, min(NP, 64)]", fn, Kp);
   if ((size_t)H * d * 8 + (size_t)NP * 8 > 200 * 1024)
     return hsa::api_fail(HSA_ERR_UNSUPPORTED, "%s: H*d*8 + NP*8 bytes exceed the shared-memory budget", fn);
+  if (NP > H * d) return hsa::api_fail(HSA_ERR_UNSUPPORTED, "%s: NP = %d pages exceed H*d = %d", fn, NP, H * d);
   const size_t need = 256 + (size_t)hsa::kColMaxSplits * H * d * sizeof(float);
   if (need > kNoAllocScratchBytes)
     return hsa::api_fail(HSA_ERR_UNSUPPORTED, "%s: H*d = %d needs %zu scratch bytes, the static maximum is %zu", fn,
@@ -79,10 +80,9 @@ extern "C" hsa_status_t hkv_select_pages_noalloc(const float* kbar_pages, int NP
   int* status = status_out ? reinterpret_cast<int*>(status_out) : static_cast<int*>(base);
   float* part = reinterpret_cast<float*>(static_cast<char*>(base) + 256);
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), stream);
-  if (e == cudaSuccess) e = hsa::launch_colsum_partial(Q, Lq, H * d, part, stream);
+  if (e == cudaSuccess) e = hsa::launch_page_scores_partial(Q, Lq, H * d, kbar_pages, NP, cand_range, part, stream);
   if (e == cudaSuccess)
-    e = hsa::launch_select_pages_final(part, Lq, H * d, kbar_pages, NP, cand_range, Kp, sel_out, scores_out, status,
-                                       stream);
+    e = hsa::launch_select_pages_final(part, Lq, NP, cand_range, Kp, sel_out, scores_out, status, stream);
   if (e != cudaSuccess) return hsa::api_fail(HSA_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(e));
   return HSA_OK;
 }
