@@ -115,7 +115,7 @@ Layout make_layout(int H, int d, int Lq, long long Lc, int r) {
   L.eklo = take(hrd * 2);
   L.fvhi = take(hrd * 2);
   L.fvlo = take(hrd * 2);
-  L.splits = r > 0 ? hsa::proj_tc_splits(H, r, Lc, Lq) : 0;
+  L.splits = r > 0 ? hsa::proj_tc_splits(H, d, r, Lc, Lq) : 0;
   L.projpart = take((size_t)L.splits * 2 * hrd * 4);
   L.total = off;
   return L;

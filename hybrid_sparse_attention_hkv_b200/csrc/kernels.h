@@ -102,7 +102,7 @@ cudaError_t launch_proj(const uint16_t* E, const uint16_t* F, long long ef_head_
                         const uint16_t* Kq, const uint16_t* Vc, const uint16_t* Vq, int H, int d, int r,
                         long long Lc, int Lq, int splits, float* part, cudaStream_t s);
 // tcgen05 / TMEM / TMA version (proj_tc.cu); partial-sum layout as launch_proj.
-int proj_tc_splits(int H, int r, long long Lc, int Lq);
+int proj_tc_splits(int H, int d, int r, long long Lc, int Lq);
 cudaError_t launch_proj_tc(const uint16_t* E, const uint16_t* F, long long ef_head_stride, const uint16_t* Kc,
                            const uint16_t* Kq, const uint16_t* Vc, const uint16_t* Vq, int H, int d, int r,
                            long long Lc, int Lq, int splits, float* part, int* status, cudaStream_t s);

@@ -3,9 +3,11 @@
 // news summary, HSA paragraph: low-rank projection, O(L r)):
 //     EK_h = E_h [Kc; Kq]_h,   FV_h = F_h [Vc; Vq]_h,   E_h, F_h in R^{r x L}.
 //
-// One CTA per (group of up to 4 128-row tiles of r, head, split of L, E.K or F.V):
+// One CTA per (group of 128-row tiles of r, HP heads, split of L, E.K or F.V); with
+// one E shared by all heads, HP = 2 adjacent heads share every E tile (one MMA of
+// N = 2 d covers both), which halves the E traffic:
 //   warp 0      TMA producer: per 64-row chunk of L, the E (or F) tiles [128 x 64]
-//               of every r tile and the K (or V) chunk [64 x d] of the head, into a
+//               of every r tile and the K (or V) chunk [64 x HP d] of the heads, into a
 //               ring of 128-byte-swizzled stages; chunks of the cached KV and of the
 //               chunk KV are separate (E's column offset Lc for the latter), so no
 //               chunk straddles the two tensors;
@@ -46,20 +48,22 @@ struct PjArgs {
   int* status;
 };
 
-template <int D, int MT>
+template <int NB, int MT>  // NB = HP x d accumulator columns per r tile
 struct PjLayout {
   static constexpr int kEBytes = 128 * kChunk * 2;       // one [128 x 64] tile: 16 KB
-  static constexpr int kBBytes = kChunk * D * 2;         // [64 x D]
+  static constexpr int kBBytes = kChunk * NB * 2;        // [64 x NB]
   static constexpr int kStageBytes = MT * kEBytes + kBBytes;
   static constexpr int kStages = (200 * 1024) / kStageBytes > 6 ? 6 : (200 * 1024) / kStageBytes;
   static constexpr int kBytes = kStages * kStageBytes;
-  static constexpr int kTmemCols = MT * D <= 32 ? 32 : (MT * D <= 64 ? 64 : (MT * D <= 128 ? 128 : (MT * D <= 256 ? 256 : 512)));
+  static constexpr int kTmemCols = MT * NB <= 32 ? 32 : (MT * NB <= 64 ? 64 : (MT * NB <= 128 ? 128 : (MT * NB <= 256 ? 256 : 512)));
+  static_assert(MT * NB <= 512, "accumulators exceed TMEM");
 };
 
 // ------------------------------------------------------------------ kernel
-template <int D, int MT>
+template <int D, int MT, int HP>
 __global__ void __launch_bounds__(kPjThreads, 1) proj_tc_kernel(const __grid_constant__ PjMaps maps, const PjArgs a) {
-  using Lay = PjLayout<D, MT>;
+  constexpr int NB = HP * D;
+  using Lay = PjLayout<NB, MT>;
   constexpr int NS = Lay::kStages;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem =
@@ -68,7 +72,7 @@ __global__ void __launch_bounds__(kPjThreads, 1) proj_tc_kernel(const __grid_con
   __shared__ uint32_t s_tmem;
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int rg = blockIdx.x, h = blockIdx.y;
+  const int rg = blockIdx.x, h0 = blockIdx.y * HP;  // first head of this CTA
   const int which = blockIdx.z & 1, split = blockIdx.z >> 1;
   const int c_begin = split * a.chunks_per_split;
   const int c_end = min(a.n_chunks, c_begin + a.chunks_per_split);
@@ -76,7 +80,7 @@ __global__ void __launch_bounds__(kPjThreads, 1) proj_tc_kernel(const __grid_con
   const CUtensorMap* mE = which ? &maps.f : &maps.e;
   const CUtensorMap* mBc = which ? &maps.vc : &maps.kc;
   const CUtensorMap* mBq = which ? &maps.vq : &maps.kq;
-  const int erow0 = (a.per_head ? h * a.r : 0) + rg * MT * 128;
+  const int erow0 = (a.per_head ? h0 * a.r : 0) + rg * MT * 128;  // per-head E only with HP = 1
 
   if (warp == 0) {
     tmem_alloc(&s_tmem, Lay::kTmemCols);
@@ -114,14 +118,14 @@ __global__ void __launch_bounds__(kPjThreads, 1) proj_tc_kernel(const __grid_con
 #pragma unroll
         for (int t = 0; t < MT; ++t) tma_load_2d(st + t * Lay::kEBytes, mE, &bar_full[s], ecol, erow0 + t * 128);
 #pragma unroll
-        for (int c2 = 0; c2 < D / 64; ++c2)
+        for (int c2 = 0; c2 < NB / 64; ++c2)
           tma_load_2d(st + MT * Lay::kEBytes + c2 * (kChunk * 128), cached ? mBc : mBq, &bar_full[s],
-                      h * D + c2 * 64, brow);
+                      h0 * D + c2 * 64, brow);
       }
       __syncwarp();
     }
   } else if (warp == 1) {
-    const uint32_t idesc = idesc_bf16(128, D, false, true);
+    const uint32_t idesc = idesc_bf16(128, NB, false, true);
     bool ok = true;
     for (int i = 0; i < nc; ++i) {
       const int s = i % NS;
@@ -139,7 +143,7 @@ __global__ void __launch_bounds__(kPjThreads, 1) proj_tc_kernel(const __grid_con
           for (int kk = 0; kk < kChunk / 16; ++kk) {
             const uint64_t ad = sdesc_sw128(st + t * Lay::kEBytes + kk * 32, 16, 1024);
             const uint64_t bd = sdesc_sw128(b_base + kk * 2048, kChunk * 128, 1024);
-            mma_ss(tacc + t * D, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+            mma_ss(tacc + t * NB, ad, bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
           }
         }
         mma_commit(&bar_empty[s]);
@@ -155,21 +159,22 @@ __global__ void __launch_bounds__(kPjThreads, 1) proj_tc_kernel(const __grid_con
     const bool have = nc > 0 && mbar_wait_warp(&bar_acc, 0, a.status);
     if (nc == 0 || have) {
       tc_fence_after();
-      float* out = a.part + ((((long long)split * 2 + which) * a.H + h) * a.r) * D;
 #pragma unroll
       for (int t = 0; t < MT; ++t) {
         const int m = (rg * MT + t) * 128 + row;
 #pragma unroll
-        for (int c = 0; c < D / 16; ++c) {
+        for (int c = 0; c < NB / 16; ++c) {
+          // columns [hh d, hh d + d) of the accumulator belong to head h0 + hh
+          float* out = a.part + ((((long long)split * 2 + which) * a.H + h0 + (c * 16) / D) * a.r) * D;
           uint32_t v[16];
           if (nc > 0) {
-            tmem_ld16_sync(tacc + loff + t * D + c * 16, v);
+            tmem_ld16_sync(tacc + loff + t * NB + c * 16, v);
           } else {
 #pragma unroll
             for (int k = 0; k < 16; ++k) v[k] = 0u;
           }
           if (m < a.r) {
-            float4* dst = reinterpret_cast<float4*>(out + (long long)m * D + c * 16);
+            float4* dst = reinterpret_cast<float4*>(out + (long long)m * D + (c * 16) % D);
 #pragma unroll
             for (int k = 0; k < 4; ++k)
               dst[k] = make_float4(__uint_as_float(v[4 * k]), __uint_as_float(v[4 * k + 1]),
@@ -213,26 +218,36 @@ cudaError_t map2d(CUtensorMap* m, const void* base, long long rows, long long co
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int D, int MT>
+template <int D, int MT, int HP>
 cudaError_t launch_mt(const PjMaps& maps, const PjArgs& a, int groups, int splits, cudaStream_t s) {
-  using Lay = PjLayout<D, MT>;
+  using Lay = PjLayout<HP * D, MT>;
   const size_t smem = 1024 + Lay::kBytes;
-  cudaError_t e = cudaFuncSetAttribute(proj_tc_kernel<D, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e =
+      cudaFuncSetAttribute(proj_tc_kernel<D, MT, HP>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  proj_tc_kernel<D, MT><<<dim3(groups, a.H, 2 * splits), kPjThreads, smem, s>>>(maps, a);
+  proj_tc_kernel<D, MT, HP><<<dim3(groups, a.H / HP, 2 * splits), kPjThreads, smem, s>>>(maps, a);
   return cudaGetLastError();
+}
+
+// Heads per CTA: 2 when one E serves every head and H is even, else 1.
+int proj_heads_per_cta(int H, bool per_head) { return (!per_head && H % 2 == 0) ? 2 : 1; }
+// r tiles per CTA: at most 4, and at most 512 TMEM columns of accumulators.
+int proj_tiles_per_cta(int r, int d, int hp) {
+  const int tiles = (r + 127) / 128;
+  const int cap = 512 / (hp * d) < 4 ? 512 / (hp * d) : 4;
+  return tiles < cap ? tiles : cap;
 }
 
 }  // namespace
 
-int proj_tc_groups(int r) {
-  const int tiles = (r + 127) / 128;
-  return (tiles + 3) / 4;
-}
-
-int proj_tc_splits(int H, int r, long long Lc, int Lq) {
+// Splits of L chosen for the shared-E launch (the workspace is sized with them); a
+// per-head-E launch uses the same count with twice the CTAs.
+int proj_tc_splits(int H, int d, int r, long long Lc, int Lq) {
   const long long chunks = (Lc + kChunk - 1) / kChunk + (Lq + kChunk - 1) / kChunk;
-  const long long base = (long long)proj_tc_groups(r) * H * 2;
+  const int hp = proj_heads_per_cta(H, false);
+  const int mt = proj_tiles_per_cta(r, d, hp);
+  const int groups = ((r + 127) / 128 + mt - 1) / mt;
+  const long long base = (long long)groups * (H / hp) * 2;
   int best = 1;
   double best_eff = 0.0;
   for (int s = 1; s <= 16 && s <= chunks; ++s) {
@@ -270,22 +285,36 @@ cudaError_t launch_proj_tc(const uint16_t* E, const uint16_t* F, long long ef_he
   a.chunks_per_split = (a.n_chunks + splits - 1) / splits;
   a.part = part;
   a.status = status;
-  const int tiles = (r + 127) / 128;
-  const int groups = proj_tc_groups(r);
-  const int mt = tiles < 4 ? tiles : 4;
+  const int hp = proj_heads_per_cta(H, a.per_head != 0);
+  const int mt = proj_tiles_per_cta(r, d, hp);
+  const int groups = ((r + 127) / 128 + mt - 1) / mt;
   if (d == 128) {
+    if (hp == 2) {
+      switch (mt) {
+        case 1: return launch_mt<128, 1, 2>(maps, a, groups, splits, s);
+        default: return launch_mt<128, 2, 2>(maps, a, groups, splits, s);
+      }
+    }
     switch (mt) {
-      case 1: return launch_mt<128, 1>(maps, a, groups, splits, s);
-      case 2: return launch_mt<128, 2>(maps, a, groups, splits, s);
-      case 3: return launch_mt<128, 3>(maps, a, groups, splits, s);
-      default: return launch_mt<128, 4>(maps, a, groups, splits, s);
+      case 1: return launch_mt<128, 1, 1>(maps, a, groups, splits, s);
+      case 2: return launch_mt<128, 2, 1>(maps, a, groups, splits, s);
+      case 3: return launch_mt<128, 3, 1>(maps, a, groups, splits, s);
+      default: return launch_mt<128, 4, 1>(maps, a, groups, splits, s);
+    }
+  }
+  if (hp == 2) {
+    switch (mt) {
+      case 1: return launch_mt<64, 1, 2>(maps, a, groups, splits, s);
+      case 2: return launch_mt<64, 2, 2>(maps, a, groups, splits, s);
+      case 3: return launch_mt<64, 3, 2>(maps, a, groups, splits, s);
+      default: return launch_mt<64, 4, 2>(maps, a, groups, splits, s);
     }
   }
   switch (mt) {
-    case 1: return launch_mt<64, 1>(maps, a, groups, splits, s);
-    case 2: return launch_mt<64, 2>(maps, a, groups, splits, s);
-    case 3: return launch_mt<64, 3>(maps, a, groups, splits, s);
-    default: return launch_mt<64, 4>(maps, a, groups, splits, s);
+    case 1: return launch_mt<64, 1, 1>(maps, a, groups, splits, s);
+    case 2: return launch_mt<64, 2, 1>(maps, a, groups, splits, s);
+    case 3: return launch_mt<64, 3, 1>(maps, a, groups, splits, s);
+    default: return launch_mt<64, 4, 1>(maps, a, groups, splits, s);
   }
 }
 
