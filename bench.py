@@ -35,12 +35,12 @@ DEFAULT_WORKLOAD = 1
 # section marker to the next one) is unchanged (sha256 prefix of the section).
 TRAFFIC = {
     # profiles/gather_and_projection_hbm_wan1.3b_480p.md
-    "gather": {"file": "hkv.cu", "section": "gather", "sha": "ea6010aad5d6ab04", "bytes": 306733056 + 251928320},
-    "linformer_proj": {"file": "proj_tc.cu", "section": "kernel", "sha": "083e8f5fb32f84a9",
-                       "bytes": 392173312 + 6182656},
+    "gather": {"file": "hkv.cu", "section": "gather", "sha": "ea6010aad5d6ab04", "bytes": 306732800 + 251682048},
+    "linformer_proj": {"file": "proj_tc.cu", "section": "kernel", "sha": "75f5b56741b141bd",
+                       "bytes": 392642816 + 3636480},
     # profiles/sparse_attn_tc_wan1.3b_480p.md
-    "attention_merge": {"file": "attn_tc.cu", "section": "kernel", "sha": "6cfb3e60052e490f",
-                        "bytes": 276799744 + 19160832},
+    "attention_merge": {"file": "attn_tc.cu", "section": "kernel", "sha": "8169def598c0e796",
+                        "bytes": 276314624 + 18804992},
 }
 
 
