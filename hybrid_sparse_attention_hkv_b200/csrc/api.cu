@@ -2,7 +2,8 @@
 // workspace layout, per-kernel trace events and the launch sequence of each call.
 // Nothing here allocates device memory, frees or synchronises (hsa_status_read
 // excepted); hsa_forward creates, on its first call on a thread and device, one
-// side stream and two events that it keeps for that thread.
+// side stream (for the projection, beside the block selection) and two events
+// that it keeps for that thread.
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
@@ -169,7 +170,10 @@ cudaError_t side_stream(SideStream** out) {
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   SideStream& ss = t_side[dev];
   if (!ss.s) {
-    if ((e = cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking)) != cudaSuccess) return e;
+    // the highest priority: the projection's CTAs are dispatched ahead of the selection's
+    int least = 0, greatest = 0;
+    if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess) return e;
+    if ((e = cudaStreamCreateWithPriority(&ss.s, cudaStreamNonBlocking, greatest)) != cudaSuccess) return e;
     if ((e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
     if ((e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming)) != cudaSuccess) return e;
   }
@@ -490,19 +494,20 @@ hsa_status_t hsa_forward(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_b
     sel.intra_idx = at<int32_t>(ws, L.intra_idx);
     sel.intra_cnt = at<int32_t>(ws, L.intra_cnt);
   }
-  TRY(run_block_select(cfg, L, Q, Kc, Kq, kbar128, tau, sel, ws, stream));
+  // The Linformer projection does not depend on the block selection: it runs on a
+  // side stream while this stream pools, selects and plans; the attention waits for
+  // both.
   hsa::AttnArgs a = attn_args(cfg, L, ws, Q, Kc, Vc, Kq, Vq);
-  // the work plan needs only the selection: it runs on a side stream beside the
-  // projection, joined before the attention
   SideStream* side = nullptr;
   cudaError_t e = side_stream(&side);
   if (e == cudaSuccess) e = cudaEventRecord(side->fork, stream);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(side->s, side->fork, 0);
   if (e != cudaSuccess) return fail(HSA_ERR_CUDA, "%s: side stream: %s", fn, cudaGetErrorString(e));
-  TRY(run_plan(L, sel, ws, a, side->s));
+  TRY(run_projection(cfg, L, Kc, Vc, Kq, Vq, E, F, ef_head_stride, ws, a, side->s));
   if ((e = cudaEventRecord(side->join, side->s)) != cudaSuccess)
     return fail(HSA_ERR_CUDA, "%s: side stream: %s", fn, cudaGetErrorString(e));
-  TRY(run_projection(cfg, L, Kc, Vc, Kq, Vq, E, F, ef_head_stride, ws, a, stream));
+  TRY(run_block_select(cfg, L, Q, Kc, Kq, kbar128, tau, sel, ws, stream));
+  TRY(run_plan(L, sel, ws, a, stream));
   if ((e = cudaStreamWaitEvent(stream, side->join, 0)) != cudaSuccess)
     return fail(HSA_ERR_CUDA, "%s: side stream: %s", fn, cudaGetErrorString(e));
   a.gate_logit = gate_logit;
