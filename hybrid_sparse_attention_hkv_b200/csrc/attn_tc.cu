@@ -23,7 +23,7 @@
 //               buffers (a slot frees when its S MMA ends);
 //   warp 6      TMA producer of the V parts (V, or FV_hi + FV_lo) into a 2-slot
 //               ring (a slot frees when its P.V MMA ends);
-//   warp 1      MMA issuer (lane 0): S_j = Q K_j^T (+ Q EK_lo^T) into one of two
+//   warp 1      MMA issuer (one elected lane): S_j = Q K_j^T (+ Q EK_lo^T) into one of two
 //               TMEM S buffers, then O += P_j V_j with P_j read from TMEM (written
 //               over S_j; for linear tiles P_hi FV_hi + P_lo FV_hi + P_hi FV_lo
 //               into a second accumulator O_l);
@@ -34,10 +34,10 @@
 //               o_l = O_l / l_l, out = g o_s + (1 - g) o_l, stored.
 // The tensor core computes S_{j+1} while the softmax warps work on S_j.
 // Every wait is bounded (HSA_ERR_TIMEOUT in the workspace status on expiry).  The
-// per-tile waits are per-lane polls of one barrier by a converged warp (a warp-wide
-// vote after each of them cost 7% of the kernel's time); the waits before the first
-// and after the last tile, where the warps go on to warp-collective TMEM access and
-// teardown, take the warp's common answer.
+// softmax warps' per-tile waits are per-lane (a warp-wide vote after each of them
+// cost 7% of the kernel's time); the MMA warp, which issues with elect.sync, and the
+// waits before the first and after the last tile, where the warps go on to
+// warp-collective TMEM access and teardown, take the warp's common answer.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -214,9 +214,10 @@ __device__ __forceinline__ void softmax_tile_split(const uint32_t (&sr)[64], flo
   l = l * alpha + (st.x + st.y);
 }
 
-// MMA issue with every loop unrolled at compile time: the descriptors of one tile
-// are its base descriptor plus constant address offsets (in 16-byte units, the
-// descriptor's low field), so consecutive MMAs issue back to back.
+// MMA issue by the whole MMA warp (one elected lane issues), every loop unrolled at
+// compile time: the descriptors of one tile are its base descriptor plus constant
+// address offsets (in 16-byte units, the descriptor's low field), so consecutive
+// MMAs issue back to back.
 // S (+)= Q K^T over D / 16 steps of 16; K tile of ROWS rows (K-major, 128-byte swizzle).
 template <int D, int ROWS>
 __device__ __forceinline__ void issue_qk(uint32_t tS, uint64_t qd, uint64_t kd, bool accumulate_first) {
@@ -225,7 +226,7 @@ __device__ __forceinline__ void issue_qk(uint32_t tS, uint64_t qd, uint64_t kd, 
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint64_t qo = (uint64_t)(((kk / 4) * kRegionBytes + (kk % 4) * 32) >> 4);
     const uint64_t ko = (uint64_t)(((kk / 4) * (ROWS * 128) + (kk % 4) * 32) >> 4);
-    mma_ss(tS, qd + qo, kd + ko, idesc, (accumulate_first || kk > 0) ? 1u : 0u);
+    mma_ss_elect(tS, qd + qo, kd + ko, idesc, (accumulate_first || kk > 0) ? 1u : 0u);
   }
 }
 // O (+)= P V over ROWS / 16 steps; P from TMEM, V tile of ROWS rows (MN-major).
@@ -234,7 +235,7 @@ __device__ __forceinline__ void issue_pv(uint32_t tO, uint32_t tP, uint64_t vd, 
   constexpr uint32_t idesc = idesc_bf16(128, D, false, true);
 #pragma unroll
   for (int kk = 0; kk < ROWS / 16; ++kk)
-    mma_ts(tO, tP + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc, (accumulate_first || kk > 0) ? 1u : 0u);
+    mma_ts_elect(tO, tP + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idesc, (accumulate_first || kk > 0) ? 1u : 0u);
 }
 
 template <int D>
@@ -426,55 +427,52 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     bool ok = mbar_wait_warp(&bar_q, 0, status);
     tc_fence_after();
     const uint64_t qd = sdesc_sw128(smem_u32(sQ), 16, 1024);
+    // The warp stays converged: waits take the warp's common answer, tile codes and
+    // descriptors are warp-uniform, one elected lane issues each MMA and commit.
+    // K and V arrive by TMA on their mbarriers, which orders them for the tensor
+    // core; only P, written to TMEM by the softmax warps, needs the tcgen05 fence.
     auto issue_s = [&](int j) -> bool {
       const int s = j % kKStages;
-      if (!mbar_wait(&bar_k_full[s], (j / kKStages) & 1, status)) return false;
-      tc_fence_after();
-      if (lane == 0) {
-        const int code = tile_at(j);
-        const uint64_t kd = sdesc_sw128(smem_u32(sK + s * Lay::kKVBytes), 16, 1024);
-        const uint32_t tS = tmem + (j & 1) * 128;
-        if (tile_type(code) == kTileLinear) {  // EK_hi then EK_lo, 64 rows each
-          issue_qk<D, 64>(tS, qd, kd, false);
-          issue_qk<D, 64>(tS, qd, kd + (uint64_t)(kHalfSlot >> 4), true);
-        } else if (tile_rows(code) == 128) {
-          issue_qk<D, 128>(tS, qd, kd, false);
-        } else {
-          issue_qk<D, 64>(tS, qd, kd, false);
-        }
-        mma_commit(&bar_k_empty[s]);
-        mma_commit(&bar_s_full[j & 1]);
+      if (!mbar_wait_warp(&bar_k_full[s], (j / kKStages) & 1, status)) return false;
+      const int code = tile_at(j);
+      const uint64_t kd = sdesc_sw128(smem_u32(sK + s * Lay::kKVBytes), 16, 1024);
+      const uint32_t tS = tmem + (j & 1) * 128;
+      if (tile_type(code) == kTileLinear) {  // EK_hi then EK_lo, 64 rows each
+        issue_qk<D, 64>(tS, qd, kd, false);
+        issue_qk<D, 64>(tS, qd, kd + (uint64_t)(kHalfSlot >> 4), true);
+      } else if (tile_rows(code) == 128) {
+        issue_qk<D, 128>(tS, qd, kd, false);
+      } else {
+        issue_qk<D, 64>(tS, qd, kd, false);
       }
-      __syncwarp();
+      mma_commit_elect(&bar_k_empty[s]);
+      mma_commit_elect(&bar_s_full[j & 1]);
       return true;
     };
     if (ok && T > 0) ok = issue_s(0);
     for (int j = 0; ok && j < T; ++j) {
       if (j + 1 < T && !issue_s(j + 1)) break;
-      if (!mbar_wait(&bar_p_full[j & 1], (j >> 1) & 1, status)) break;
+      if (!mbar_wait_warp(&bar_p_full[j & 1], (j >> 1) & 1, status)) break;
       const int sv = j % kVStages;
-      if (!mbar_wait(&bar_v_full[sv], (j / kVStages) & 1, status)) break;
+      if (!mbar_wait_warp(&bar_v_full[sv], (j / kVStages) & 1, status)) break;
       tc_fence_after();
-      if (lane == 0) {
-        const int code = tile_at(j);
-        const uint32_t v_base = smem_u32(sV + sv * Lay::kKVBytes);
-        const uint32_t tP = tmem + (j & 1) * 128;
-        if (tile_type(code) == kTileLinear) {
-          // O_l += P_hi FV_hi + P_lo FV_hi + P_hi FV_lo; first linear tile initialises O_l
-          const uint64_t vhi = sdesc_sw128(v_base, 64 * 128, 1024);
-          const uint64_t vlo = sdesc_sw128(v_base + kHalfSlot, 64 * 128, 1024);
-          issue_pv<D, 64>(tOl, tP, vhi, j > 0);
-          issue_pv<D, 64>(tOl, tP + 32, vhi, true);
-          issue_pv<D, 64>(tOl, tP, vlo, true);
-        } else if (tile_rows(code) == 128) {  // the first sparse tile initialises O_s
-          issue_pv<D, 128>(tOs, tP, sdesc_sw128(v_base, 128 * 128, 1024), j > n_lin);
-        } else {
-          issue_pv<D, 64>(tOs, tP, sdesc_sw128(v_base, 64 * 128, 1024), j > n_lin);
-        }
-        mma_commit(&bar_v_empty[sv]);
-        mma_commit(&bar_o_done);
+      const int code = tile_at(j);
+      const uint32_t v_base = smem_u32(sV + sv * Lay::kKVBytes);
+      const uint32_t tP = tmem + (j & 1) * 128;
+      if (tile_type(code) == kTileLinear) {
+        // O_l += P_hi FV_hi + P_lo FV_hi + P_hi FV_lo; first linear tile initialises O_l
+        const uint64_t vhi = sdesc_sw128(v_base, 64 * 128, 1024);
+        const uint64_t vlo = sdesc_sw128(v_base + kHalfSlot, 64 * 128, 1024);
+        issue_pv<D, 64>(tOl, tP, vhi, j > 0);
+        issue_pv<D, 64>(tOl, tP + 32, vhi, true);
+        issue_pv<D, 64>(tOl, tP, vlo, true);
+      } else if (tile_rows(code) == 128) {  // the first sparse tile initialises O_s
+        issue_pv<D, 128>(tOs, tP, sdesc_sw128(v_base, 128 * 128, 1024), j > n_lin);
+      } else {
+        issue_pv<D, 64>(tOs, tP, sdesc_sw128(v_base, 64 * 128, 1024), j > n_lin);
       }
-      __syncwarp();
+      mma_commit_elect(&bar_v_empty[sv]);
+      mma_commit_elect(&bar_o_done);
     }
   } else if (warp >= 2 && warp <= 5) {
     // ------------------------------------------------------------ softmax + epilogue
