@@ -50,7 +50,10 @@ class HkvHsaStep:
             hkv_page_summary(pages_k[p], self.kbar_pages[p], self.ws)
 
     def __call__(self, Q, Kq, Vq, tau, gate_logit, E, F, e_cur=None, e_seg=None, seg_begin=None,
-                 ef_head_stride=0):
+                 ef_head_stride=0, out=None):
+        """One step on the current stream; the result goes to `out` (same shape and
+        dtype as self.out) when given, else to self.out."""
+        dst = self.out if out is None else out
         cand = None
         if e_cur is not None:
             hkv_select_prompt(e_cur, e_seg, seg_begin, self.seg, self.cand_range)
@@ -58,6 +61,6 @@ class HkvHsaStep:
         hkv_select_pages(self.kbar_pages, Q, self.Kp, self.sel, self.ws, self.scores, cand)
         hkv_gather(self.page_k_ptrs, self.page_v_ptrs, self.sel, self.Kp, self.P_tok, self.H, self.d,
                    self.Kc, self.Vc, self.ws, self.kbar128)
-        hsa_forward(self.cfg, Q, self.Kc, self.Vc, Kq, Vq, tau, gate_logit, E, F, self.out, self.ws,
+        hsa_forward(self.cfg, Q, self.Kc, self.Vc, Kq, Vq, tau, gate_logit, E, F, dst, self.ws,
                     self.kbar128, self.selection, ef_head_stride)
-        return self.out
+        return dst
