@@ -550,7 +550,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_before();
       mbar_arrive(&bar_p_full[b]);
     }
-    if (ok && (T == 0 || mbar_wait_warp(&bar_o_done, (T - 1) & 1, status))) {
+    // Wait for the last two P.V products in order.  The barrier completes one phase
+    // per tile; a wait for the phase of tile T - 1 alone would return at once while
+    // the phase of tile T - 2 is still open (same parity as an already completed
+    // phase), which S_{T-1} does not exclude -- it was issued before P.V of T - 2.
+    // These waits poll (bounded): the softmax warps have no other work left, and
+    // sleeping waits here cost 1 % of the kernel's time.
+    auto wait_poll = [&](uint64_t* bar, uint32_t par) -> bool {
+      bool r = false;
+      for (uint32_t i = 0; i < kSpinLimit && !r; ++i) r = mbar_try_wait(bar, par);
+      if (!r) set_status(status, HSA_ERR_TIMEOUT);
+      return __all_sync(0xffffffffu, r);
+    };
+    if (ok && T >= 2) ok = wait_poll(&bar_o_done, (T - 2) & 1);
+    if (ok && (T == 0 || wait_poll(&bar_o_done, (T - 1) & 1))) {
       tc_fence_after();
       const int grow = q0 + row;
       const bool valid_row = grow < a.Lq;

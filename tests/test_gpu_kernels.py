@@ -229,6 +229,40 @@ def test_no_history(Lq, d, H):
     assert_close(out.cpu().numpy(), ref["out"], "Lc = 0")
 
 
+@pytest.mark.parametrize("Lq,d,H", [(64, 128, 2), (64, 64, 3), (192, 128, 2)])
+def test_fused_merge_short_lists(Lq, d, H):
+    """Units with two or three key tiles (one linear tile, one or two chunk tiles): the
+    fused output is repeatable and equals the gated merge of the two branches run
+    alone.  With so few tiles the P.V product of the next-to-last tile can still be
+    running when the softmax ends, so the epilogue must wait for both last products."""
+    shape = synth.StepShape("short", H=H, d=d, frames=1, F_tok=Lq, page_frames=1, page_tok=8, NP=1, Kp=1, r=64)
+    x = synth.make_inputs(shape, 21)
+    E = to_dev(x.E[:, shape.page_tok:].copy())
+    F = to_dev(x.F[:, shape.page_tok:].copy())
+    cfg = make_config(H, d, Lq, 0, 64)
+    ws = hsa.workspace(cfg)
+    sel = SelectionBuffers.empty(cfg)
+    Q, Kq, Vq = to_dev(x.Q), to_dev(x.Kq), to_dev(x.Vq)
+    tau = torch.from_numpy(x.tau).cuda()
+    z = torch.from_numpy(x.z).cuda()
+    outs = []
+    for _ in range(3):
+        out = torch.empty(Lq, H, d, dtype=torch.float32, device="cuda")
+        hsa.hsa_forward(cfg, Q, None, None, Kq, Vq, tau, z, E, F, out, ws, sel=sel)
+        outs.append(out)
+    o_s = torch.empty_like(outs[0])
+    o_l = torch.empty_like(outs[0])
+    hsa.hsa_sparse_attn(cfg, Q, None, None, Kq, Vq, sel, o_s, ws)
+    hsa.hsa_linear_attn(cfg, Q, None, None, Kq, Vq, E, F, o_l, ws)
+    torch.cuda.synchronize()
+    assert hsa.hsa_status_read(ws) == 0
+    for out in outs[1:]:
+        assert torch.equal(out, outs[0])
+    g = torch.sigmoid(z).view(1, H, 1)
+    merged = g * o_s + (1 - g) * o_l
+    assert float((outs[0] - merged).abs().max()) <= 1e-5
+
+
 # ----------------------------------------------------------------- device-side status and argument checks
 
 def test_device_status_short_candidate_range():
