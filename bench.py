@@ -39,8 +39,8 @@ TRAFFIC = {
     "linformer_proj": {"file": "proj_tc.cu", "section": "kernel", "sha": "75f5b56741b141bd",
                        "bytes": 392642816 + 3636480},
     # profiles/sparse_attn_tc_wan1.3b_480p.md
-    "attention_merge": {"file": "attn_tc.cu", "section": "kernel", "sha": "6b61432575ea718e",
-                        "bytes": 276499200 + 20734720},
+    "attention_merge": {"file": "attn_tc.cu", "section": "kernel", "sha": "4cb6ffdabc6aea75",
+                        "bytes": 278155264 + 20598528},
 }
 
 
