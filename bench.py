@@ -3,8 +3,10 @@
 One step = page-level retrieval (hkv_select_pages) + active-cache gather
 (hkv_gather, with the fused 128-row K pooling) + hsa_forward (pooling, block
 selection, Linformer projection and attention, sparse attention with the gated
-merge), on the Wan-1.3B-shaped 480p workload: 12 heads, d = 128, a 4680-query
-chunk, 16 history pages of 12480 tokens resident in HBM, Kp = 4, r = 256.
+merge).  The default workload is the largest one: the 14B-shaped 720p step (40
+heads, d = 128, a 10800-query chunk, 12 history pages of 28800 tokens resident in
+HBM, Kp = 4, r = 512).  ``--workload I`` selects another (0 tiny, 1 Wan-1.3B
+480p, 2 14B 480p, 3 14B 720p, 4 90-second horizon with host-pinned pages).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload I]
 
@@ -28,17 +30,17 @@ sys.path.insert(0, ROOT)
 
 METRIC = "HSA layer query-tokens/s + eff. TFLOP/s on 1 B200; % tensor/HBM roofline"
 UNIT = "query-tokens/s"
-DEFAULT_WORKLOAD = 1
+DEFAULT_WORKLOAD = 3
 
 # DRAM traffic per launch from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
 # keyed by kernel; valid only while that kernel's section of its source file (from its
 # section marker to the next one) is unchanged (sha256 prefix of the section).
 TRAFFIC = {
-    # profiles/gather_and_projection_hbm_wan1.3b_480p.md
+    # ncu capture of the gather and the projection at the Wan-1.3B 480p workload
     "gather": {"file": "hkv.cu", "section": "gather", "sha": "ea6010aad5d6ab04", "bytes": 306732800 + 251682048},
     "linformer_proj": {"file": "proj_tc.cu", "section": "kernel", "sha": "75f5b56741b141bd",
                        "bytes": 392642816 + 3636480},
-    # profiles/sparse_attn_tc_wan1.3b_480p.md
+    # ncu capture of the attention kernel at the Wan-1.3B 480p workload
     "attention_merge": {"file": "attn_tc.cu", "section": "kernel", "sha": "4cb6ffdabc6aea75",
                         "bytes": 278155264 + 20598528},
 }
@@ -180,32 +182,62 @@ def oracle_summaries(x, shape):
     return np.stack([oracle.page_summary(x.pages_k[p], np.float32) for p in range(shape.NP)])
 
 
-def oracle_step_sample(x, shape, kbar, heads=None, rows_per_step=None):
-    """Time the fp64 oracle on one step, or on a bounded sample of it: page retrieval +
-    gather, then the HSA of the given heads on the given number of query rows; the
-    step time is extrapolated as t_retrieval + H/len(heads) * t_heads * Lq/rows."""
+def oracle_sample_plan(shape, small=False):
+    """The bounded sample the fp64 oracle is timed on: (heads, query rows).  Whole step
+    for the tiny workload; otherwise the first, middle and last head (tau 1.00, ~0.68,
+    0.35) on the rows of three 128-row query blocks (first, middle, last); `small`
+    (one step of the reference arm) takes one head and one query block."""
+    import numpy as np
+    if shape.Lq <= 512 and shape.H <= 4:
+        return list(range(shape.H)), None
+    nQ = -(-shape.Lq // 128)
+    if small:
+        return [0], np.arange(0, min(128, shape.Lq))
+    heads = sorted({0, shape.H // 2, shape.H - 1})
+    blocks = sorted({0, nQ // 2, nQ - 1})
+    rows = np.concatenate([np.arange(128 * b, min(128 * (b + 1), shape.Lq)) for b in blocks])
+    return heads, rows
+
+
+def oracle_step_sample(x, shape, kbar, heads, rows):
+    """Time the fp64 oracle, phase by phase, on a bounded sample of one step:
+      t_r            page retrieval + gather (whole, all heads);
+      t_fixed[h]     block selection (whole maps) + Linformer projection (whole) of head h;
+      t_rows[h]      both attention branches and the merge of head h on `rows`.
+    Step time (extrapolated unless the sample is the whole step):
+      t_r + (H / len(heads)) * sum_h (t_fixed[h] + t_rows[h] * Lq / len(rows))."""
     import numpy as np
     import oracle
-    heads = list(range(shape.H)) if heads is None else list(heads)
-    nrows = shape.Lq if rows_per_step is None else min(rows_per_step, shape.Lq)
-    rows = None if nrows == shape.Lq else np.linspace(0, shape.Lq - 1, nrows).astype(np.int64)
+    nrows = shape.Lq if rows is None else len(rows)
     t0 = time.perf_counter()
     sel, _ = oracle.select_pages(kbar, x.Q, shape.Kp)
     Kc = oracle.gather_pages(x.pages_k, sel)
     Vc = oracle.gather_pages(x.pages_v, sel)
     t_r = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    hs = np.array(heads)
-    oracle.hsa_step(x.Q[:, hs], Kc[:, hs], Vc[:, hs], x.Kq[:, hs], x.Vq[:, hs], x.tau[hs], x.z[hs], x.E, x.F,
-                    rows=rows)
-    t_h = time.perf_counter() - t0
-    t_step = t_r + t_h * (shape.H / len(heads)) * (shape.Lq / nrows)
-    if len(heads) == shape.H and nrows == shape.Lq:
+    per_head = 0.0
+    timed = t_r
+    for h in heads:
+        hs = [h]
+        Qh, Kch, Vch, Kqh, Vqh = x.Q[:, hs], Kc[:, hs], Vc[:, hs], x.Kq[:, hs], x.Vq[:, hs]
+        t0 = time.perf_counter()
+        selh = oracle.block_select(Qh, Kch, Kqh, x.tau[hs])
+        EK, FV = oracle.linear_projection(x.E, x.F, Kch, Kqh, Vch, Vqh)
+        t1 = time.perf_counter()
+        o_s = oracle.sparse_attention(Qh, Kch, Vch, Kqh, Vqh, selh.inter, selh.intra, rows=rows)
+        o_l = oracle.linear_attention(Qh, EK, FV, rows=rows)
+        oracle.gated_merge(o_s, o_l, x.z[hs])
+        t2 = time.perf_counter()
+        per_head += (t1 - t0) + (t2 - t1) * shape.Lq / nrows
+        timed += t2 - t0
+    t_step = t_r + per_head * shape.H / len(heads)
+    whole = len(heads) == shape.H and nrows == shape.Lq
+    if whole:
         sample = "the whole step: page retrieval, gather, block selection, both branches and merge, all heads and rows"
     else:
-        sample = (f"page retrieval + gather, then HSA of heads {heads} on {nrows} of {shape.Lq} query rows; step time "
-                  f"extrapolated as t_retrieval + (H/heads) * t_heads * (Lq/rows)")
-    return t_step, sample, t_r + t_h
+        sample = (f"page retrieval + gather (whole); heads {list(heads)}: block selection and projection (whole), "
+                  f"both branches + merge on {nrows} of {shape.Lq} query rows; step time extrapolated as "
+                  f"t_retrieval + (H/heads) * sum_h (t_select_proj + t_rows * Lq/rows)")
+    return {"t_step": t_step, "sample": sample, "timed_seconds": timed, "extrapolated": not whole}
 
 
 def blas_threads():
@@ -225,6 +257,23 @@ def cpu_model():
     except OSError:
         pass
     return "unknown"
+
+
+def measure_host_link(dev, nbytes=256 << 20, reps=5):
+    """Best pinned host -> device copy bandwidth (GB/s) over `reps` copies of `nbytes`."""
+    import torch
+    src = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    dst = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    best = 0.0
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        dst.copy_(src, non_blocking=True)
+        e1.record()
+        e1.synchronize()
+        best = max(best, nbytes / (e0.elapsed_time(e1) / 1e3) / 1e9)
+    del src, dst
+    return best
 
 
 # ------------------------------------------------------------------ distributed plumbing
@@ -262,41 +311,51 @@ def max_over_ranks(value, world, device="cpu"):
 
 # ------------------------------------------------------------------ arms
 def run_reference(args, shape, rank, world):
-    """The oracle as it stands, on the host cores, a bounded sample per step."""
+    """The oracle as it stands, on the host cores: every step times a bounded sample
+    of the step (one head, one query block, plus the whole page retrieval and
+    gather) and extrapolates the step time from it; the line says so."""
     if rank != 0:
         return None
     import synth
     x = synth.make_inputs(shape, synth.seed_of(args.workload))
     kbar = oracle_summaries(x, shape)
-    # each step: one head (rotating) on a row sample sized so that K + W steps stay
-    # within a few minutes (all rows for up to ~50 steps, fewer rows beyond)
-    rows = max(64, shape.Lq // max(1, (args.steps + args.warmup) // 50))
-    for k in range(args.warmup):
-        oracle_step_sample(x, shape, kbar, heads=[k % shape.H], rows_per_step=rows)
-    ts = []
-    sample = ""
+    heads, rows = oracle_sample_plan(shape, small=True)
+    for _ in range(args.warmup):
+        oracle_step_sample(x, shape, kbar, heads, rows)
+    ts, timed = [], 0.0
+    r = None
     for k in range(args.steps):
-        t, sample, _ = oracle_step_sample(x, shape, kbar, heads=[k % shape.H], rows_per_step=rows)
-        ts.append(t)
+        hk = [k % shape.H] if len(heads) < shape.H else heads  # rotate the sampled head
+        r = oracle_step_sample(x, shape, kbar, hk, rows)
+        ts.append(r["t_step"])
+        timed += r["timed_seconds"]
     t_step = statistics.mean(ts)
     value = shape.Lq / t_step
     cores = blas_threads()
+    sample = r["sample"] + "; the sampled head rotates over the steps"
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
         "config": workload_config(shape, args),
+        "extrapolated": r["extrapolated"], "timed_seconds": timed,
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
-                         "cpu": cpu_model()},
+                         "extrapolated": r["extrapolated"], "timed_seconds": timed, "cpu": cpu_model()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
+
+
+def input_bytes(shape):
+    """Bytes of one step's inputs: the page store, Q / Kq / Vq and E / F (bf16)."""
+    hd = shape.H * shape.d
+    return 2.0 * (2 * shape.NP * shape.P_tok * hd + 3 * shape.Lq * hd + 2 * shape.r * shape.L)
 
 
 def workload_config(shape, args):
     return {"workload": shape.name, "H": shape.H, "d": shape.d, "Lq": shape.Lq, "Lc": shape.Lc, "L": shape.L,
             "P_tok": shape.P_tok, "NP": shape.NP, "Kp": shape.Kp, "r": shape.r, "block_inter": 128,
             "block_intra": 64, "tau": "1.00 -> 0.35 linear across heads", "pages": "host-pinned" if shape.host_pages else "HBM",
-            "l2": "flushed between timed steps (256 MiB write); inputs 1.3 GB > L2",
+            "l2": f"flushed between timed steps (256 MiB write); inputs {input_bytes(shape) / 1e9:.2f} GB",
             "parallelism": f"replicas x{getattr(args, 'gpus', 1)}"}
 
 
@@ -413,12 +472,19 @@ def run_gpu(args, shape, rank, world, local):
     f_sparse = 4.0 * shape.d * pairs
     f_total = f_sparse + w["proj_flops"] + w["lin_attn_flops"]
     eff_tflops = f_total / (ms_per_step / 1e3) / 1e12
+    # tensor peak: the burst figure (measured at the maximum SM clock) when the timed
+    # region ran at that clock, else the sustained one (measured under the power cap)
+    sm, smax = clk.get("sm_mhz"), clk.get("sm_max_mhz")
+    at_max = sm is None or not smax or sm >= 0.97 * smax
+    t_kind = "burst" if at_max else "sustained"
+    t_peak = peaks["bf16_tflops"] if at_max else peaks["bf16_tflops_sustained"]
+    host_gbs = measure_host_link(dev) if shape.host_pages else None
     kernel_work = {
         # the fused attention kernel: selected-block FLOPs of the sparse branch plus the
         # useful FLOPs of the linear branch (the split-precision extra products not counted)
         "attention_merge": ("tensor", f_sparse + w["lin_attn_flops"]),
         "linformer_proj": ("tensor", w["proj_flops"]),
-        "gather": ("hbm", w["gather_bytes"]),
+        "gather": ("host-link", w["gather_bytes"] / 2) if shape.host_pages else ("hbm", w["gather_bytes"]),
         "pool": ("hbm", w["pool_bytes"]),
         "page_scores_partial": ("hbm", w["select_pages_bytes"]),
     }
@@ -431,11 +497,17 @@ def run_gpu(args, shape, rank, world, local):
             bound, work = kernel_work[name]
             if bound == "tensor":
                 ach = work / (avg_ms / 1e3) / 1e12
-                entry.update({"bound": "tensor", "achieved": ach, "unit": "TFLOP/s",
-                              "frac": ach / peaks["bf16_tflops_sustained"]})
+                entry.update({"bound": "tensor", "achieved": ach, "unit": "TFLOP/s", "peak": t_peak,
+                              "frac": ach / t_peak, "frac_burst": ach / peaks["bf16_tflops"],
+                              "frac_sustained": ach / peaks["bf16_tflops_sustained"]})
+            elif bound == "host-link":
+                ach = work / (avg_ms / 1e3) / 1e9  # bytes read over the host link (K and V pages)
+                entry.update({"bound": "host-link", "achieved": ach, "unit": "GB/s", "peak": host_gbs,
+                              "frac": ach / host_gbs if host_gbs else None})
             else:
                 ach = work / (avg_ms / 1e3) / 1e9
-                entry.update({"bound": "hbm", "achieved": ach, "unit": "GB/s", "frac": ach / peaks["hbm_gbs"]})
+                entry.update({"bound": "hbm", "achieved": ach, "unit": "GB/s", "peak": peaks["hbm_gbs"],
+                              "frac": ach / peaks["hbm_gbs"]})
         tr = TRAFFIC.get(name)
         if tr and tr["sha"] == section_sha(os.path.join(ROOT, "hybrid_sparse_attention_hkv_b200", "csrc", tr["file"]),
                                            tr["section"]):
@@ -444,15 +516,18 @@ def run_gpu(args, shape, rank, world, local):
     dom = max(kernels, key=lambda k: kernels[k]["share"])
     de = kernels[dom]
     bound = de.get("bound", "hbm")
-    peak = peaks["bf16_tflops_sustained"] if bound == "tensor" else peaks["hbm_gbs"]
     traffic = None
     tr = TRAFFIC.get(dom)
     if tr and tr["sha"] == section_sha(os.path.join(ROOT, "hybrid_sparse_attention_hkv_b200", "csrc", tr["file"]),
                                        tr["section"]):
         traffic = tr["bytes"]
-    roofline = {"kernel": dom, "bound": bound, "achieved": de.get("achieved"), "peak": peak,
-                "unit": "TFLOP/s" if bound == "tensor" else "GB/s", "frac": de.get("frac"), "traffic": traffic,
-                "peak_source": f"{peaks['source']} ({'bf16 sustained' if bound == 'tensor' else 'HBM copy'})"}
+    peak_source = {"tensor": f"{peaks['source']} bf16 {t_kind} (median SM clock {sm} of {smax} MHz)",
+                   "hbm": f"{peaks['source']} HBM copy",
+                   "host-link": "pinned host-to-device copy measured in this run"}.get(bound, "")
+    roofline = {"kernel": dom, "bound": bound, "achieved": de.get("achieved"), "peak": de.get("peak"),
+                "unit": de.get("unit"), "frac": de.get("frac"), "traffic": traffic, "peak_source": peak_source}
+    if bound == "tensor":
+        roofline.update({"frac_burst": de["frac_burst"], "frac_sustained": de["frac_sustained"]})
 
     res = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -470,9 +545,11 @@ def run_gpu(args, shape, rank, world, local):
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        t_step, sample, spent = oracle_step_sample(ds.x, shape, oracle_summaries(ds.x, shape))
-        res["cpu_baseline"] = {"value": shape.Lq / t_step, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-                               "sample": sample, "seconds": spent, "cpu": cpu_model()}
+        heads, rows = oracle_sample_plan(shape)
+        r = oracle_step_sample(ds.x, shape, oracle_summaries(ds.x, shape), heads, rows)
+        res["cpu_baseline"] = {"value": shape.Lq / r["t_step"], "unit": UNIT, "cores": blas_threads(),
+                               "kind": "oracle", "sample": r["sample"], "extrapolated": r["extrapolated"],
+                               "timed_seconds": r["timed_seconds"], "cpu": cpu_model()}
     ds.close()
     return res if rank == 0 else None
 

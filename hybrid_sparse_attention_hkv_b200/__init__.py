@@ -24,7 +24,8 @@ EXPORTED = [
     "hsa_status_string", "hsa_last_error_detail", "hsa_workspace_size", "hsa_status_clear", "hsa_status_read",
     "hkv_page_summary", "hkv_select_prompt", "hkv_select_pages", "hkv_select_pages_noalloc", "hkv_gather",
     "hsa_block_select", "hsa_sparse_attn", "hsa_linear_attn", "hsa_forward",
-    "hsa_trace_begin", "hsa_trace_count", "hsa_trace_end",
+    "hsa_trace_begin", "hsa_trace_count", "hsa_trace_end", "hsa_set_wait_limit", "hsa_selftest_wait",
+    "hsa_thread_release",
 ]
 
 
@@ -76,6 +77,9 @@ def load_library(path: str = LIB_PATH):
         "hsa_trace_begin": (I, [P, I, P]),
         "hsa_trace_count": (I, []),
         "hsa_trace_end": (I, []),
+        "hsa_set_wait_limit": (I, [P, ctypes.c_uint, P]),
+        "hsa_selftest_wait": (I, [P, P, P]),
+        "hsa_thread_release": (I, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -123,6 +127,20 @@ def hsa_status_read(ws, stream=None) -> int:
     st = ctypes.c_int(0)
     _check(load_library().hsa_status_read(_p(ws), _stream(stream), ctypes.byref(st)), "hsa_status_read")
     return st.value
+
+
+def hsa_set_wait_limit(ws, limit_us: int, stream=None):
+    """Limit of the bounded device waits of kernels using `ws` (microseconds; 0 = 2 s default)."""
+    _check(load_library().hsa_set_wait_limit(_p(ws), int(limit_us), _stream(stream)), "hsa_set_wait_limit")
+
+
+def hsa_selftest_wait(ws, waited_ns=None, stream=None):
+    """Run the timeout self-test kernel (an mbarrier wait nothing completes)."""
+    _check(load_library().hsa_selftest_wait(_p(ws), _p(waited_ns), _stream(stream)), "hsa_selftest_wait")
+
+
+def hsa_thread_release():
+    _check(load_library().hsa_thread_release(), "hsa_thread_release")
 
 
 @dataclass

@@ -1,9 +1,9 @@
 // C-ABI entry points of the HKV + HSA library: host-side argument checks,
 // workspace layout, per-kernel trace events and the launch sequence of each call.
-// Nothing here allocates device memory, frees or synchronises (hsa_status_read
-// excepted); hsa_forward creates, on its first call on a thread and device, one
-// side stream (for the projection, beside the block selection) and two events
-// that it keeps for that thread.
+// Nothing here allocates device memory, frees or synchronises (hsa_status_read and
+// hsa_thread_release excepted); hsa_forward creates, on its first call on a thread
+// and device, one side stream (for the projection, beside the block selection) and
+// two events that it keeps for that thread until hsa_thread_release.
 #include <math.h>
 #include <stdarg.h>
 #include <stdio.h>
@@ -67,6 +67,12 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
   do {                                                                                  \
     if ((p) != nullptr && !aligned16(p))                                                \
       return fail(HSA_ERR_INVALID_ARG, "%s: " #p " is not 16-byte aligned", fn);        \
+  } while (0)
+
+#define OPTIONAL_PTR8(p)                                                                \
+  do {                                                                                  \
+    if ((p) != nullptr && (reinterpret_cast<uintptr_t>(p) & 7u) != 0)                   \
+      return fail(HSA_ERR_INVALID_ARG, "%s: " #p " is not 8-byte aligned", __func__);   \
   } while (0)
 
 // Workspace layout shared by every entry point (offsets in bytes).
@@ -170,12 +176,21 @@ cudaError_t side_stream(SideStream** out) {
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   SideStream& ss = t_side[dev];
   if (!ss.s) {
-    // the highest priority: the projection's CTAs are dispatched ahead of the selection's
+    // the highest priority: the projection's CTAs are dispatched ahead of the selection's.
+    // All three objects are created before any is kept, so a failure leaves none behind.
     int least = 0, greatest = 0;
-    if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess) return e;
-    if ((e = cudaStreamCreateWithPriority(&ss.s, cudaStreamNonBlocking, greatest)) != cudaSuccess) return e;
-    if ((e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
-    if ((e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming)) != cudaSuccess) return e;
+    SideStream n;
+    e = cudaDeviceGetStreamPriorityRange(&least, &greatest);
+    if (e == cudaSuccess) e = cudaStreamCreateWithPriority(&n.s, cudaStreamNonBlocking, greatest);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&n.fork, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&n.join, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      if (n.join) cudaEventDestroy(n.join);
+      if (n.fork) cudaEventDestroy(n.fork);
+      if (n.s) cudaStreamDestroy(n.s);
+      return e;
+    }
+    ss = n;
   }
   *out = &ss;
   return cudaSuccess;
@@ -246,6 +261,23 @@ hsa_status_t hsa_status_clear(void* ws, hsa_stream_t stream) {
   return e == cudaSuccess ? HSA_OK : fail(HSA_ERR_CUDA, "hsa_status_clear: %s", cudaGetErrorString(e));
 }
 
+hsa_status_t hsa_set_wait_limit(void* ws, unsigned int limit_us, hsa_stream_t stream) {
+  if (!ws) return fail(HSA_ERR_WORKSPACE, "hsa_set_wait_limit: workspace is NULL");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    return fail(HSA_ERR_WORKSPACE, "hsa_set_wait_limit: workspace not 256-byte aligned");
+  cudaError_t e = hsa::launch_set_wait_limit(status_of(ws), limit_us, stream);
+  return e == cudaSuccess ? HSA_OK : fail(HSA_ERR_CUDA, "hsa_set_wait_limit: %s", cudaGetErrorString(e));
+}
+
+hsa_status_t hsa_selftest_wait(void* ws, unsigned long long* waited_ns, hsa_stream_t stream) {
+  if (!ws) return fail(HSA_ERR_WORKSPACE, "hsa_selftest_wait: workspace is NULL");
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    return fail(HSA_ERR_WORKSPACE, "hsa_selftest_wait: workspace not 256-byte aligned");
+  OPTIONAL_PTR8(waited_ns);
+  cudaError_t e = hsa::launch_wait_selftest(status_of(ws), waited_ns, stream);
+  return e == cudaSuccess ? HSA_OK : fail(HSA_ERR_CUDA, "hsa_selftest_wait: %s", cudaGetErrorString(e));
+}
+
 hsa_status_t hsa_status_read(const void* ws, hsa_stream_t stream, int* status) {
   if (!ws || !status) return fail(HSA_ERR_INVALID_ARG, "hsa_status_read: NULL argument");
   cudaError_t e = cudaStreamSynchronize(stream);
@@ -267,6 +299,26 @@ hsa_status_t hsa_trace_end(void) {
   t_names = nullptr;
   t_pairs = 0;
   return HSA_OK;
+}
+
+hsa_status_t hsa_thread_release(void) {
+  int cur = -1;
+  cudaError_t e = cudaGetDevice(&cur);
+  if (e != cudaSuccess) return fail(HSA_ERR_CUDA, "hsa_thread_release: %s", cudaGetErrorString(e));
+  cudaError_t first = cudaSuccess;
+  for (int dev = 0; dev < kMaxDevices; ++dev) {
+    SideStream& ss = t_side[dev];
+    if (!ss.s) continue;
+    cudaError_t r = cudaSetDevice(dev);
+    if (r == cudaSuccess) r = cudaStreamSynchronize(ss.s);
+    if (r == cudaSuccess) r = cudaEventDestroy(ss.join);
+    if (r == cudaSuccess) r = cudaEventDestroy(ss.fork);
+    if (r == cudaSuccess) r = cudaStreamDestroy(ss.s);
+    if (r == cudaSuccess) ss = SideStream();
+    else if (first == cudaSuccess) first = r;
+  }
+  cudaSetDevice(cur);
+  return first == cudaSuccess ? HSA_OK : fail(HSA_ERR_CUDA, "hsa_thread_release: %s", cudaGetErrorString(first));
 }
 
 // ------------------------------------------------------------------ HKV

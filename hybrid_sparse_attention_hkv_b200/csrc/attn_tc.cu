@@ -252,7 +252,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   int* tiles = reinterpret_cast<int*>(smem + Lay::kBytes);  // [r/64 + nKc + nKq]
   int* flags = tiles + (a.EKhi ? a.r / 64 : 0) + nKc + nKq; // [nKq]
   __shared__ __align__(8) uint64_t bar_q, bar_k_full[kKStages], bar_k_empty[kKStages], bar_v_full[kVStages],
-      bar_v_empty[kVStages], bar_s_full[2], bar_p_full[2], bar_o_done;
+      bar_v_empty[kVStages], bar_s_full[2], bar_p_full[2], bar_o_done, bar_final;
   __shared__ uint32_t s_tmem;
   __shared__ int s_ntiles;
 
@@ -260,6 +260,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   int* status = a.status;
+  const uint64_t wlim = wait_limit_ns(status);
   const int HQ = a.H * nQ128;
   const bool planned = a.units != nullptr;
   // both loads in flight together (units[] holds the grid's max_units entries)
@@ -294,6 +295,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&bar_p_full[b], 128);
     }
     mbar_init(&bar_o_done, 1);
+    mbar_init(&bar_final, 1);
     fence_barrier_init();
   }
 
@@ -372,7 +374,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     for (int j = 0; j < T; ++j) {
       const int s = j % kKStages;
-      if (!mbar_wait(&bar_k_empty[s], ((j / kKStages) & 1) ^ 1, status)) break;
+      if (!mbar_wait(&bar_k_empty[s], ((j / kKStages) & 1) ^ 1, status, wlim)) break;
       if (lane == 0) {
         const int code = tile_at(j);
         const int type = tile_type(code);
@@ -399,7 +401,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ------------------------------------------------------------ V producer
     for (int j = 0; j < T; ++j) {
       const int s = j % kVStages;
-      if (!mbar_wait(&bar_v_empty[s], ((j / kVStages) & 1) ^ 1, status)) break;
+      if (!mbar_wait(&bar_v_empty[s], ((j / kVStages) & 1) ^ 1, status, wlim)) break;
       if (lane == 0) {
         const int code = tile_at(j);
         const int type = tile_type(code);
@@ -424,7 +426,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    bool ok = mbar_wait_warp(&bar_q, 0, status);
+    bool ok = mbar_wait_warp(&bar_q, 0, status, wlim);
     tc_fence_after();
     const uint64_t qd = sdesc_sw128(smem_u32(sQ), 16, 1024);
     // The warp stays converged: waits take the warp's common answer, tile codes and
@@ -433,7 +435,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // core; only P, written to TMEM by the softmax warps, needs the tcgen05 fence.
     auto issue_s = [&](int j) -> bool {
       const int s = j % kKStages;
-      if (!mbar_wait_warp(&bar_k_full[s], (j / kKStages) & 1, status)) return false;
+      if (!mbar_wait_warp(&bar_k_full[s], (j / kKStages) & 1, status, wlim)) return false;
       const int code = tile_at(j);
       const uint64_t kd = sdesc_sw128(smem_u32(sK + s * Lay::kKVBytes), 16, 1024);
       const uint32_t tS = tmem + (j & 1) * 128;
@@ -452,9 +454,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (ok && T > 0) ok = issue_s(0);
     for (int j = 0; ok && j < T; ++j) {
       if (j + 1 < T && !issue_s(j + 1)) break;
-      if (!mbar_wait_warp(&bar_p_full[j & 1], (j >> 1) & 1, status)) break;
+      if (!mbar_wait_warp(&bar_p_full[j & 1], (j >> 1) & 1, status, wlim)) break;
       const int sv = j % kVStages;
-      if (!mbar_wait_warp(&bar_v_full[sv], (j / kVStages) & 1, status)) break;
+      if (!mbar_wait_warp(&bar_v_full[sv], (j / kVStages) & 1, status, wlim)) break;
       tc_fence_after();
       const int code = tile_at(j);
       const uint32_t v_base = smem_u32(sV + sv * Lay::kKVBytes);
@@ -473,6 +475,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       mma_commit_elect(&bar_v_empty[sv]);
       mma_commit_elect(&bar_o_done);
+      // one-shot: completes once every MMA of the unit has completed
+      if (j == T - 1) mma_commit_elect(&bar_final);
     }
   } else if (warp >= 2 && warp <= 5) {
     // ------------------------------------------------------------ softmax + epilogue
@@ -486,7 +490,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     bool ok = true;
     for (int j = 0; j < T; ++j) {
       const int b = j & 1;
-      if (!mbar_wait(&bar_s_full[b], (j >> 1) & 1, status)) {
+      if (!mbar_wait(&bar_s_full[b], (j >> 1) & 1, status, wlim)) {
         ok = false;
         break;
       }
@@ -531,7 +535,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // O holds the P.V products of tiles 0..j-1 once the last of them has completed
         // (P.V of tile j cannot have started: it waits for this P).  Without a rescale
         // nothing here touches O, and the wait is skipped.
-        if (j > 0 && !mbar_wait(&bar_o_done, (j - 1) & 1, status)) {
+        if (j > 0 && !mbar_wait(&bar_o_done, (j - 1) & 1, status, wlim)) {
           ok = false;
           break;
         }
@@ -550,20 +554,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       tc_fence_before();
       mbar_arrive(&bar_p_full[b]);
     }
-    // Wait for the last two P.V products in order.  The barrier completes one phase
-    // per tile; a wait for the phase of tile T - 1 alone would return at once while
-    // the phase of tile T - 2 is still open (same parity as an already completed
-    // phase), which S_{T-1} does not exclude -- it was issued before P.V of T - 2.
-    // These waits poll (bounded): the softmax warps have no other work left, and
-    // sleeping waits here cost 1 % of the kernel's time.
+    // Wait for every P.V product of the unit on the one-shot barrier the MMA warp
+    // commits after its last P.V (phase 0, so the parity names it unambiguously; the
+    // per-tile barrier can be up to two phases ahead or behind here).  The wait polls
+    // (bounded): the softmax warps have no other work left, and sleeping waits here
+    // cost 1 % of the kernel's time.
     auto wait_poll = [&](uint64_t* bar, uint32_t par) -> bool {
       bool r = false;
       for (uint32_t i = 0; i < kSpinLimit && !r; ++i) r = mbar_try_wait(bar, par);
       if (!r) set_status(status, HSA_ERR_TIMEOUT);
       return __all_sync(0xffffffffu, r);
     };
-    if (ok && T >= 2) ok = wait_poll(&bar_o_done, (T - 2) & 1);
-    if (ok && (T == 0 || wait_poll(&bar_o_done, (T - 1) & 1))) {
+    if (ok && (T == 0 || wait_poll(&bar_final, 0))) {
       tc_fence_after();
       const int grow = q0 + row;
       const bool valid_row = grow < a.Lq;

@@ -13,10 +13,26 @@ constexpr int kBlockInter = 128;
 constexpr int kBlockIntra = 64;
 
 // ------------------------------------------------------------------ status word
-// The first 256 bytes of every workspace hold the device status (an hsa_status_t).
-// Kernels record only the first failure.
+// The first 256 bytes of every workspace are its header:
+//   int32 [0]  device status (an hsa_status_t); kernels record only the first failure
+//   int32 [1]  reserved
+//   uint32[2]  kWaitTag when word 3 holds a limit set by hsa_set_wait_limit
+//   uint32[3]  limit of every bounded device wait, in microseconds
+constexpr uint32_t kWaitTag = 0x54494157u;  // "WAIT"
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
+
 __device__ __forceinline__ void set_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
+}
+
+// Wait limit of a kernel whose `status` points at a workspace header: the host-set
+// limit when the tag is present, else 2 s.
+__device__ __forceinline__ uint64_t wait_limit_ns(const int* status) {
+  if (status != nullptr) {
+    const uint32_t* w = reinterpret_cast<const uint32_t*>(status);
+    if (w[2] == kWaitTag && w[3] != 0u) return (uint64_t)w[3] * 1000ull;
+  }
+  return kDefaultWaitLimitNs;
 }
 
 // ------------------------------------------------------------------ bf16
@@ -53,38 +69,6 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-
-// 16-byte cp.async global -> shared; src_bytes = 0 zero-fills the destination.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, int src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(dst), "l"(src), "r"(src_bytes));
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N)); }
-
-// ------------------------------------------------------------------ warp MMA (sm_80+ form)
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
-}
-
-// D(16x8 f32) += A(16x16 bf16, row) * B(16x8 bf16, col)
-__device__ __forceinline__ void mma_bf16(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// Shared-memory tiles are rows of 16-byte chunks; chunk c of row r is stored at
-// chunk (c ^ (r & 7)) so that 8 consecutive rows of one chunk column hit 8
-// different bank groups (conflict-free ldmatrix).
-__device__ __forceinline__ int swz(int row, int chunk) { return chunk ^ (row & 7); }
 
 template <typename T>
 __device__ __forceinline__ T warp_sum(T v) {

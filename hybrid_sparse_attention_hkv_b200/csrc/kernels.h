@@ -97,16 +97,21 @@ inline int plan_max_units(int H, int nQ128) { return H * nQ128 + kPlanSMs * kPla
 inline int plan_max_slots() { return 2 * kPlanSMs * kPlanUnitsPerSM + 2; }
 
 // ---------------------------------------------------------------- proj.cu
-int proj_splits(int H, int r, long long L);
-cudaError_t launch_proj(const uint16_t* E, const uint16_t* F, long long ef_head_stride, const uint16_t* Kc,
-                        const uint16_t* Kq, const uint16_t* Vc, const uint16_t* Vq, int H, int d, int r,
-                        long long Lc, int Lq, int splits, float* part, cudaStream_t s);
-// tcgen05 / TMEM / TMA version (proj_tc.cu); partial-sum layout as launch_proj.
+// tcgen05 / TMEM / TMA projection (proj_tc.cu): partial sums [splits][2][H][r][d] fp32
+// (EK then FV), reduced by launch_proj_reduce (proj.cu).
 int proj_tc_splits(int H, int d, int r, long long Lc, int Lq);
 cudaError_t launch_proj_tc(const uint16_t* E, const uint16_t* F, long long ef_head_stride, const uint16_t* Kc,
                            const uint16_t* Kq, const uint16_t* Vc, const uint16_t* Vq, int H, int d, int r,
                            long long Lc, int Lq, int splits, float* part, int* status, cudaStream_t s);
 cudaError_t launch_proj_reduce(const float* part, int splits, int H, int d, int r, uint16_t* EKhi,
                                uint16_t* EKlo, uint16_t* FVhi, uint16_t* FVlo, cudaStream_t s);
+
+// ---------------------------------------------------------------- waits.cu
+// Write the wait limit (microseconds; 0 = the 2 s default) into a workspace header.
+cudaError_t launch_set_wait_limit(int* header, uint32_t limit_us, cudaStream_t s);
+// One thread waits on an mbarrier nothing arrives at; the bounded wait must give up
+// after the header's limit and record HSA_ERR_TIMEOUT.  waited_ns (optional) gets
+// the time the wait took.
+cudaError_t launch_wait_selftest(int* status, unsigned long long* waited_ns, cudaStream_t s);
 
 }  // namespace hsa

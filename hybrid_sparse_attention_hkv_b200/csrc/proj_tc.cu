@@ -72,6 +72,7 @@ __global__ void __launch_bounds__(kPjThreads, 1) proj_tc_kernel(const __grid_con
   __shared__ uint32_t s_tmem;
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const uint64_t wlim = wait_limit_ns(a.status);
   const int rg = blockIdx.x, h0 = blockIdx.y * HP;  // first head of this CTA
   const int which = blockIdx.z & 1, split = blockIdx.z >> 1;
   const int c_begin = split * a.chunks_per_split;
@@ -107,7 +108,7 @@ __global__ void __launch_bounds__(kPjThreads, 1) proj_tc_kernel(const __grid_con
     }
     for (int i = 0; i < nc; ++i) {
       const int s = i % NS;
-      if (!mbar_wait(&bar_empty[s], ((i / NS) & 1) ^ 1, a.status)) break;
+      if (!mbar_wait(&bar_empty[s], ((i / NS) & 1) ^ 1, a.status, wlim)) break;
       if (lane == 0) {
         const int c = c_begin + i;
         const bool cached = c < a.n_chunks_c;
@@ -129,7 +130,7 @@ __global__ void __launch_bounds__(kPjThreads, 1) proj_tc_kernel(const __grid_con
     bool ok = true;
     for (int i = 0; i < nc; ++i) {
       const int s = i % NS;
-      if (!mbar_wait(&bar_full[s], (i / NS) & 1, a.status)) {
+      if (!mbar_wait(&bar_full[s], (i / NS) & 1, a.status, wlim)) {
         ok = false;
         break;
       }
@@ -156,7 +157,7 @@ __global__ void __launch_bounds__(kPjThreads, 1) proj_tc_kernel(const __grid_con
     const int wq = warp & 3;
     const int row = 32 * wq + lane;
     const uint32_t loff = (uint32_t)(32 * wq) << 16;
-    const bool have = nc > 0 && mbar_wait_warp(&bar_acc, 0, a.status);
+    const bool have = nc > 0 && mbar_wait_warp(&bar_acc, 0, a.status, wlim);
     if (nc == 0 || have) {
       tc_fence_after();
 #pragma unroll

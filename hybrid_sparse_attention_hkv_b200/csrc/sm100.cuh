@@ -14,10 +14,10 @@ namespace sm100 {
 
 // A thread waiting on an mbarrier sleeps in the hardware until the phase completes
 // (or kSuspendNs pass) instead of polling shared memory, which the tensor cores'
-// operand reads keep busy.  A wait gives up after kWaitLimitNs, records
-// HSA_ERR_TIMEOUT and returns false.
+// operand reads keep busy.  A wait gives up after `limit_ns` (the kernel reads it
+// once from its workspace header: wait_limit_ns), records HSA_ERR_TIMEOUT and
+// returns false.
 constexpr uint32_t kSuspendNs = 1000000u;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint32_t kSpinLimit = 1u << 24;  // polls of a bounded polling wait
 
 __device__ __forceinline__ uint64_t global_ns() {
@@ -58,20 +58,20 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
   return ok != 0;
 }
 // Bounded wait for the phase with the given parity to complete.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status, uint64_t limit_ns) {
   if (mbar_try_wait_sleep(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   do {
     if (mbar_try_wait_sleep(bar, parity)) return true;
-  } while (global_ns() - t0 < kWaitLimitNs);
+  } while (global_ns() - t0 < limit_ns);
   set_status(status, HSA_ERR_TIMEOUT);
   return false;
 }
 
 // The same wait for a whole warp: every lane waits, and the warp agrees on the
 // outcome (one lane's timeout counts for all), so the lanes never diverge.
-__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int* status) {
-  const bool ok = mbar_wait(bar, parity, status);
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int* status, uint64_t limit_ns) {
+  const bool ok = mbar_wait(bar, parity, status, limit_ns);
   return __all_sync(0xffffffffu, ok);
 }
 

@@ -19,8 +19,11 @@
  *     A history page is K_p, V_p in [P_tok, H, d].
  *   - Every pointer argument is a DEVICE pointer (or, where stated, a pointer
  *     to page-locked host memory mapped into the device address space), 16-byte
- *     aligned.  The caller owns all memory: the library never allocates, frees
- *     or synchronises (hsa_status_read is the one documented exception).
+ *     aligned.  The caller owns all memory: the library never allocates or
+ *     frees device memory and never synchronises a caller's stream
+ *     (hsa_status_read and hsa_thread_release are the documented exceptions).
+ *     hsa_forward keeps, per host thread and device, one side stream and two
+ *     events that it creates on its first call; hsa_thread_release destroys them.
  *   - All work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
  *     the legacy default stream).
  *   - Arguments are validated on the host before anything is launched; a
@@ -102,8 +105,27 @@ hsa_status_t hsa_workspace_size(const hsa_config_t* cfg, int NP, int P_tok, size
 hsa_status_t hsa_status_clear(void* ws, hsa_stream_t stream);
 
 /* Synchronise `stream`, then copy the device status word of `ws` into *status
- * (an hsa_status_t value).  The only call that synchronises. */
+ * (an hsa_status_t value).  Synchronises. */
 hsa_status_t hsa_status_read(const void* ws, hsa_stream_t stream, int* status);
+
+/* Limit of every bounded device wait of the kernels that use `ws` (mbarrier
+ * waits of the tensor-core kernels), in microseconds; 0 restores the 2 s
+ * default.  Enqueued on `stream`; kept in the workspace header until changed
+ * (hsa_status_clear leaves it).  A wait that runs out records HSA_ERR_TIMEOUT in
+ * the status word and its kernel drains its copies and MMAs and exits. */
+hsa_status_t hsa_set_wait_limit(void* ws, unsigned int limit_us, hsa_stream_t stream);
+
+/* Self-test of the timeout path (failure detection; the paper has no
+ * counterpart): one thread waits on an mbarrier that nothing arrives at, with no
+ * copy or MMA in flight.  The wait gives up after the workspace's wait limit and
+ * sets HSA_ERR_TIMEOUT in its status word; the context stays usable.
+ * waited_ns: optional device uint64 that receives the time the wait took. */
+hsa_status_t hsa_selftest_wait(void* ws, unsigned long long* waited_ns, hsa_stream_t stream);
+
+/* Destroy the side stream and events hsa_forward created for this host thread
+ * (on every device it ran on), after waiting for the work queued on them.  Call
+ * it before a thread that used hsa_forward exits, or to release the handles. */
+hsa_status_t hsa_thread_release(void);
 
 /* ---------------------------------------------------------------- HKV ---- */
 
@@ -158,15 +180,17 @@ hsa_status_t hkv_gather(const hsa_bf16* const* page_k, const hsa_bf16* const* pa
  * of the call, a runtime whose memory plan is fixed before it serves, or a loop
  * where an allocation could stall the device -- and so cannot provide the
  * workspace hkv_select_pages uses for its column-sum partials.
- * Same inputs, outputs and results as hkv_select_pages; the scratch lives in a
- * static device array of 8 MiB inside the library (held by every GPU that loads
- * the library until the process exits), so 256 + 296 * H * d * 4 bytes must fit:
- * H * d <= 7084, else HSA_ERR_UNSUPPORTED.  Calls no allocator.
+ * Same inputs, outputs and results as hkv_select_pages; the scratch (the partial
+ * page scores, 256 + 296 * NP * 4 bytes at most) lives in a static device array
+ * of 2.3 MiB inside the library, held by every GPU that loads the library until
+ * the process exits: NP <= 2048 pages, else HSA_ERR_UNSUPPORTED.  Calls no
+ * allocator.
  * status_out: optional device int32 that receives the device status
  * (HSA_ERR_DEVICE for a candidate range shorter than Kp); cleared by the call.
  * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current) and caches it: make that
- * first call before any stream capture.  Every call on a device shares the
+ * (cudaGetSymbolAddress, with that device current) and caches it with the
+ * device's current context (a new context, after cudaDeviceReset, looks it up
+ * again): make that first call before any stream capture.  Every call on a device shares the
  * array: calls whose kernels could overlap on the GPU race and must be ordered
  * (one stream, or events). */
 hsa_status_t hkv_select_pages_noalloc(const float* kbar_pages, int NP, const int32_t* cand_range,

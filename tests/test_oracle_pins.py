@@ -401,3 +401,76 @@ def test_no_history_reduces_to_chunk_attention():
     o = oracle.sparse_attention(Q, empty, empty, Kq, Vq, sel.inter, sel.intra, None, 16, 8)
     ref = sdpa(oracle.widen(Q), oracle.widen(Kq), oracle.widen(Vq), 1 / math.sqrt(d))
     np.testing.assert_allclose(o, ref, rtol=1e-11, atol=1e-12)
+
+
+def _frac(s):
+    n, d = s.split("/")
+    return int(n) / int(d)
+
+
+def test_block_select_golden(golden_dir):
+    """Block pooling + block scores + per-map softmax + per-head threshold, composed, at
+    tau < 1, against hand-derived masses and kept lists.  The fixture is built so that
+    pooling Q at the wrong block size, one joint inter+intra softmax, a swapped head
+    index or the wrong head's tau each changes a kept list."""
+    g = load(golden_dir, "block_select.json")
+    Q64 = np.asarray(g["Q64_blocks"], dtype=np.float32)     # [H][4][d]
+    Kc128 = np.asarray(g["Kc128_blocks"], dtype=np.float32)  # [H][4][d]
+    Kq64 = np.asarray(g["Kq64_blocks"], dtype=np.float32)    # [H][4][d]
+    Q = bf16(np.repeat(Q64.transpose(1, 0, 2), 64, axis=0))    # [256, H, d]
+    Kc = bf16(np.repeat(Kc128.transpose(1, 0, 2), 128, axis=0))  # [512, H, d]
+    Kq = bf16(np.repeat(Kq64.transpose(1, 0, 2), 64, axis=0))  # [256, H, d]
+    tau = np.asarray(g["tau"], dtype=np.float32)
+    sel = oracle.block_select(Q, Kc, Kq, tau, scale=math.log(2.0), dtype=np.float64)
+    want_pi = np.array([[[_frac(x) for x in row] for row in head] for head in g["p_inter"]])
+    want_pq = np.array([[[_frac(x) for x in row] for row in head] for head in g["p_intra"]])
+    np.testing.assert_allclose(sel.p_inter, want_pi, rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(sel.p_intra, want_pq, rtol=1e-12, atol=1e-15)
+    assert [[r.tolist() for r in h] for h in sel.inter] == g["keep_inter"]
+    assert [[r.tolist() for r in h] for h in sel.intra] == g["keep_intra"]
+    # the fp32 decision precision gives the same lists here (no mass within 1e-5 of a threshold)
+    sel32 = oracle.block_select(Q, Kc, Kq, tau, scale=math.log(2.0), dtype=np.float32)
+    assert [[r.tolist() for r in h] for h in sel32.inter] == g["keep_inter"]
+    assert [[r.tolist() for r in h] for h in sel32.intra] == g["keep_intra"]
+
+
+def test_block_select_golden_rejects_plausible_mistakes(golden_dir):
+    """Planted mistakes (built on the CPU from the oracle's own parts) disagree with the
+    golden lists: queries pooled at 64 for the inter map, at 128 for the intra map, one
+    joint softmax over the inter and intra rows of a query, the wrong head's keys."""
+    g = load(golden_dir, "block_select.json")
+    Q = bf16(np.repeat(np.asarray(g["Q64_blocks"], np.float32).transpose(1, 0, 2), 64, axis=0))
+    Kc = bf16(np.repeat(np.asarray(g["Kc128_blocks"], np.float32).transpose(1, 0, 2), 128, axis=0))
+    Kq = bf16(np.repeat(np.asarray(g["Kq64_blocks"], np.float32).transpose(1, 0, 2), 64, axis=0))
+    tau = np.asarray(g["tau"])
+    sc = math.log(2.0)
+    want_inter, want_intra = g["keep_inter"], g["keep_intra"]
+
+    def keep(p, h):
+        return [oracle.keep_blocks(p[h, i], tau[h]).tolist() for i in range(p.shape[1])]
+
+    kc128 = oracle.block_means(Kc, 128)
+    kq64 = oracle.block_means(Kq, 64)
+    # inter map scored with 64-row query means (rows 0 and 2 stand for the two 128-row blocks)
+    p_bad = oracle.block_probs(oracle.block_means(Q, 64)[::2], kc128, sc)
+    assert [keep(p_bad, h) for h in range(2)] != want_inter
+    # intra map scored with 128-row query means (each used for both of its 64-row halves)
+    p_bad = oracle.block_probs(np.repeat(oracle.block_means(Q, 128), 2, axis=0), kq64, sc)
+    assert [keep(p_bad, h) for h in range(2)] != want_intra
+    # one joint softmax over [inter row of the 128-block | intra row of the 64-block]
+    q128, q64 = oracle.block_means(Q, 128), oracle.block_means(Q, 64)
+    joint_intra = []
+    for h in range(2):
+        rows = []
+        for i in range(4):
+            s = np.concatenate([q128[i // 2, h] @ kc128[:, h].T, q64[i, h] @ kq64[:, h].T]) * sc
+            w = np.exp(s - s.max())
+            kept = oracle.keep_blocks(w / w.sum(), tau[h])
+            rows.append([int(j) - 4 for j in kept if j >= 4])
+        joint_intra.append(rows)
+    assert joint_intra != want_intra
+    # head 1 scored against head 0's keys
+    swapped = Kc.copy()
+    swapped[:, 1] = Kc[:, 0]
+    assert [r.tolist() for r in oracle.block_select(Q, swapped, Kq, tau, scale=sc, dtype=np.float64).inter[1]] \
+        != want_inter[1]

@@ -57,10 +57,20 @@ def test_noalloc_page_selection_matches_workspace_version():
 
 
 def test_noalloc_rejects_sizes_beyond_the_static_maximum():
+    """The static scratch holds the partial page scores of at most 2048 pages; one page
+    more is rejected on the host with a clear error and nothing is launched."""
     import hybrid_sparse_attention_hkv_b200 as hsa
     lib = hsa.load_library()
-    big = torch.zeros(8, 64, 128, dtype=torch.bfloat16, device="cuda")  # H*d = 8192 > 7084
-    kbar = torch.zeros(4, 64, 128, dtype=torch.float32, device="cuda")
-    sel = torch.zeros(2, dtype=torch.int32, device="cuda")
-    assert _c_call(lib, kbar, big, 2, sel, None, None, None) == 2
+    H, d, NP = 40, 128, 2049  # NP <= H * d, so only the static maximum rejects it
+    Q = torch.zeros(8, H, d, dtype=torch.bfloat16, device="cuda")
+    kbar = torch.zeros(NP, H, d, dtype=torch.float32, device="cuda")
+    sel = torch.full((2,), -7, dtype=torch.int32, device="cuda")
+    assert _c_call(lib, kbar, Q, 2, sel, None, None, None) == 2
     assert b"static maximum" in lib.hsa_last_error_detail()
+    torch.cuda.synchronize()
+    assert torch.all(sel == -7)
+    # the largest page count it serves still runs
+    kbar = kbar[:2048].contiguous()
+    assert _c_call(lib, kbar, Q, 2, sel, None, None, None) == 0, lib.hsa_last_error_detail()
+    torch.cuda.synchronize()
+    assert sel.cpu().tolist() == [0, 1]  # all scores tie at 0: the lowest page ids
