@@ -16,6 +16,7 @@ Prints one JSON line (rank 0).  N > 1 runs one independent replica per GPU
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import os
@@ -259,6 +260,61 @@ def cpu_model():
     return "unknown"
 
 
+def _time_ms(fn, n, stream=None):
+    """Mean device time (ms) of n calls of fn on the current stream (CUDA events)."""
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(s)
+    for _ in range(n):
+        fn()
+    e1.record(s)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / n
+
+
+def host_tier_report(ds, shape, args, host_gbs):
+    """The host-pinned history three ways: the step as timed (pages fetched into the
+    store's HBM slots; after the warm-up the selected pages are resident, as when
+    consecutive chunks retrieve the same pages), the gather straight from the host
+    tier (zero-copy), and a cold fetch (every selected page promoted over the link)."""
+    import hybrid_sparse_attention_hkv_b200 as hsa
+    st, store = ds.step, ds.store
+    n = max(3, min(args.steps, 10))
+    kp, vp = ds.host_tables
+    zero_copy = _time_ms(lambda: hsa.hkv_gather(kp, vp, st.sel, shape.Kp, shape.P_tok, shape.H, shape.d, st.Kc, st.Vc,
+                                                st.ws, st.kbar128), n)
+
+    def cold():
+        hsa.load_library().hkv_store_init(ctypes.byref(store.desc), None)
+        store.fetch(st.sel, st.ws)
+
+    cold_ms = _time_ms(cold, n)
+    store_gather = _time_ms(lambda: hsa.hkv_gather(st.page_k_ptrs, st.page_v_ptrs, st.sel, shape.Kp, shape.P_tok,
+                                                   shape.H, shape.d, st.Kc, st.Vc, st.ws, st.kbar128), n)
+    store.fetch(st.sel, st.ws)  # resident again for what follows
+    page_bytes = 2.0 * shape.P_tok * shape.H * shape.d * 2  # K and V of one page
+    return {"slots": store.S, "pages": shape.NP,
+            "zero_copy_gather_ms": zero_copy, "zero_copy_GBps": shape.Kp * page_bytes / (zero_copy / 1e3) / 1e9,
+            "cold_fetch_ms": cold_ms, "cold_fetch_GBps": shape.Kp * page_bytes / (cold_ms / 1e3) / 1e9,
+            "resident_gather_ms": store_gather, "host_link_copy_GBps": host_gbs,
+            "note": "value / ms_per_step: steady state with the selected pages resident in the HBM slots"}
+
+
+def reuse_report(ds, shape, args):
+    """Multi-step reuse: retrieval, gather and the history's projection once per chunk
+    (prepare_chunk), then one hsa_forward_reuse per denoising step."""
+    st = ds.step
+    n = max(3, min(args.steps, 20))
+    chunk_ms = _time_ms(lambda: st.prepare_chunk(ds.Q, ds.E, ds.F, ds.e_cur, ds.e_seg, ds.seg_begin), n)
+    step_ms = _time_ms(lambda: st.denoise_step(ds.Q, ds.Kq, ds.Vq, ds.tau, ds.z, ds.E, ds.F), n)
+    return {"chunk_ms": chunk_ms, "denoise_step_ms": step_ms,
+            "query_tokens_per_s_4_steps": 4 * shape.Lq / ((chunk_ms + 4 * step_ms) / 1e3),
+            "note": "chunk = page retrieval + gather + the cached KV's Linformer products; step = block selection, "
+                    "the chunk's projection, both branches and the merge; L2 not flushed"}
+
+
 def measure_host_link(dev, nbytes=256 << 20, reps=5):
     """Best pinned host -> device copy bandwidth (GB/s) over `reps` copies of `nbytes`."""
     import torch
@@ -370,7 +426,8 @@ def run_gpu(args, shape, rank, world, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     seed = synth.seed_of(args.workload) + rank  # each replica its own seeded inputs
-    ds = DeviceStep(shape, seed)
+    # a history on the host tier is read through the tiered page store (Kp + 4 HBM slots)
+    ds = DeviceStep(shape, seed, store_slots=(shape.Kp + 4) if shape.host_pages else 0)
     st = ds.step
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
@@ -544,6 +601,9 @@ def run_gpu(args, shape, rank, world, local):
                 "copies": "pinned host buffers; H2D of step k+1 and D2H of step k-1 on copy streams beside step k"},
         "clocks": clk,
     }
+    if shape.host_pages:
+        res["host_tier"] = host_tier_report(ds, shape, args, host_gbs)
+    res["reuse"] = reuse_report(ds, shape, args)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         heads, rows = oracle_sample_plan(shape)
         r = oracle_step_sample(ds.x, shape, oracle_summaries(ds.x, shape), heads, rows)

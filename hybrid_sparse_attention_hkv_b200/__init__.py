@@ -25,7 +25,9 @@ EXPORTED = [
     "hkv_page_summary", "hkv_select_prompt", "hkv_select_pages", "hkv_select_pages_noalloc", "hkv_gather",
     "hsa_block_select", "hsa_sparse_attn", "hsa_linear_attn", "hsa_forward",
     "hsa_trace_begin", "hsa_trace_count", "hsa_trace_end", "hsa_set_wait_limit", "hsa_selftest_wait",
-    "hsa_thread_release",
+    "hsa_thread_release", "hsa_prepare_history", "hsa_forward_reuse",
+    "hkv_store_state_size", "hkv_store_init", "hkv_store_tables", "hkv_store_seal", "hkv_store_fetch",
+    "hkv_store_prefetch", "hkv_store_residency",
 ]
 
 
@@ -39,6 +41,13 @@ class Config(ctypes.Structure):
     _fields_ = [("H", ctypes.c_int), ("d", ctypes.c_int), ("Lq", ctypes.c_int), ("Lc", ctypes.c_int),
                 ("block_inter", ctypes.c_int), ("block_intra", ctypes.c_int), ("rank", ctypes.c_int),
                 ("scale", ctypes.c_float)]
+
+
+class StoreDesc(ctypes.Structure):
+    """hkv_store_t: the memories of a tiered page store (all device addresses)."""
+    _fields_ = [("NP", ctypes.c_int), ("S", ctypes.c_int), ("P_tok", ctypes.c_int), ("H", ctypes.c_int),
+                ("d", ctypes.c_int), ("host_k", ctypes.c_void_p), ("host_v", ctypes.c_void_p),
+                ("slot_k", ctypes.c_void_p), ("slot_v", ctypes.c_void_p), ("state", ctypes.c_void_p)]
 
 
 class _Selection(ctypes.Structure):
@@ -77,6 +86,16 @@ def load_library(path: str = LIB_PATH):
         "hsa_trace_begin": (I, [P, I, P]),
         "hsa_trace_count": (I, []),
         "hsa_trace_end": (I, []),
+        "hsa_prepare_history": (I, [CP, P, P, P, P, L, P, S, P]),
+        "hsa_forward_reuse": (I, [CP, P, P, P, P, P, P, P, P, P, P, L, P, I, ctypes.POINTER(_Selection), P, S,
+                                  P]),
+        "hkv_store_state_size": (S, [I, I]),
+        "hkv_store_init": (I, [ctypes.POINTER(StoreDesc), P]),
+        "hkv_store_tables": (I, [ctypes.POINTER(StoreDesc), ctypes.POINTER(P), ctypes.POINTER(P)]),
+        "hkv_store_seal": (I, [ctypes.POINTER(StoreDesc), I, P, P, P, P, S, P]),
+        "hkv_store_fetch": (I, [ctypes.POINTER(StoreDesc), P, I, P, S, P]),
+        "hkv_store_prefetch": (I, [ctypes.POINTER(StoreDesc), P, P, I, I, P, S, P]),
+        "hkv_store_residency": (I, [ctypes.POINTER(StoreDesc), P, P, P]),
         "hsa_set_wait_limit": (I, [P, ctypes.c_uint, P]),
         "hsa_selftest_wait": (I, [P, P, P]),
         "hsa_thread_release": (I, []),
@@ -228,6 +247,22 @@ def hsa_forward(cfg, Q, Kc, Vc, Kq, Vq, tau, gate_logit, E, F, out, ws, kbar128=
                                       _p(tau), _p(gate_logit), _p(E), _p(F), ef_head_stride, _p(out),
                                       1 if out.dtype == torch.bfloat16 else 0, csel, _p(ws), ws.numel(),
                                       _stream(stream)), "hsa_forward")
+
+
+def hsa_prepare_history(cfg, Kc, Vc, E, F, ws, ef_head_stride=0, stream=None):
+    """Once per chunk: project the cached KV (E Kc, F Vc) into the workspace."""
+    _check(load_library().hsa_prepare_history(ctypes.byref(cfg), _p(Kc), _p(Vc), _p(E), _p(F), ef_head_stride,
+                                              _p(ws), ws.numel(), _stream(stream)), "hsa_prepare_history")
+
+
+def hsa_forward_reuse(cfg, Q, Kc, Vc, Kq, Vq, tau, gate_logit, E, F, out, ws, kbar128=None, sel=None,
+                      ef_head_stride=0, stream=None):
+    """One denoising step against the history prepared by hsa_prepare_history."""
+    csel = ctypes.byref(sel.c()) if sel is not None else None
+    _check(load_library().hsa_forward_reuse(ctypes.byref(cfg), _p(Q), _p(Kc), _p(Vc), _p(Kq), _p(Vq), _p(kbar128),
+                                            _p(tau), _p(gate_logit), _p(E), _p(F), ef_head_stride, _p(out),
+                                            1 if out.dtype == torch.bfloat16 else 0, csel, _p(ws), ws.numel(),
+                                            _stream(stream)), "hsa_forward_reuse")
 
 
 # ---------------------------------------------------------------- tracing

@@ -81,7 +81,7 @@ struct Layout {
   size_t inter_idx = 0, inter_cnt = 0, intra_idx = 0, intra_cnt = 0;
   size_t units = 0, n_units = 0, tile_done = 0, part_o = 0, part_ml = 0, part_lin = 0, attn_end = 0;
   int max_units = 0, max_slots = 0;
-  size_t ekhi = 0, eklo = 0, fvhi = 0, fvlo = 0, projpart = 0;
+  size_t ekhi = 0, eklo = 0, fvhi = 0, fvlo = 0, projpart = 0, ekfv_hist = 0;
   size_t pages_end = 0;  // bytes needed by the page (HKV) calls
   size_t total = 0;
   int splits = 0;
@@ -122,8 +122,9 @@ Layout make_layout(int H, int d, int Lq, long long Lc, int r) {
   L.eklo = take(hrd * 2);
   L.fvhi = take(hrd * 2);
   L.fvlo = take(hrd * 2);
-  L.splits = r > 0 ? hsa::proj_tc_splits(H, d, r, Lc, Lq) : 0;
+  L.splits = r > 0 ? hsa::proj_tc_splits(H, d, r, Lc, Lq, hsa::kProjAll) : 0;
   L.projpart = take((size_t)L.splits * 2 * hrd * 4);
+  L.ekfv_hist = take(2 * hrd * 4);  // E Kc and F Vc (fp32), kept over a chunk's denoising steps
   L.total = off;
   return L;
 }
@@ -333,7 +334,7 @@ hsa_status_t hkv_page_summary(const hsa_bf16* K_page, int P_tok, int H, int d, f
   const Layout L = make_layout(H, d, 1, 0, 0);
   TRY(check_ws(fn, ws, ws_bytes, L.pages_end));
   float* part = at<float>(ws, L.colpart);
-  HSA_LAUNCH("colsum_partial", hsa::launch_colsum_partial(K_page, P_tok, H * d, part, stream));
+  HSA_LAUNCH("colsum_partial", hsa::launch_colsum_partial(K_page, P_tok, H * d, part, nullptr, stream));
   HSA_LAUNCH("page_summary_final", hsa::launch_page_summary_final(part, P_tok, H * d, kbar, stream));
   return HSA_OK;
 }
@@ -391,6 +392,112 @@ hsa_status_t hkv_gather(const hsa_bf16* const* page_k, const hsa_bf16* const* pa
   return HSA_OK;
 }
 
+// ------------------------------------------------------------------ tiered page store
+
+static hsa_status_t store_desc(const char* fn, const hkv_store_t* st, hsa::StoreDesc* out) {
+  if (!st) return fail(HSA_ERR_INVALID_ARG, "%s: store is NULL", fn);
+  TRY(check_heads(fn, st->H, st->d));
+  if (st->NP < 1 || st->S < 1 || st->P_tok < 1)
+    return fail(HSA_ERR_INVALID_ARG, "%s: NP = %d, S = %d, P_tok = %d must be >= 1", fn, st->NP, st->S, st->P_tok);
+  REQUIRE_PTR(st->host_k);
+  REQUIRE_PTR(st->host_v);
+  REQUIRE_PTR(st->slot_k);
+  REQUIRE_PTR(st->slot_v);
+  if (!st->state || (reinterpret_cast<uintptr_t>(st->state) & 255u) != 0)
+    return fail(HSA_ERR_INVALID_ARG, "%s: state must be non-NULL and 256-byte aligned", fn);
+  out->NP = st->NP;
+  out->S = st->S;
+  out->P_tok = st->P_tok;
+  out->C = st->H * st->d;
+  out->host_k = st->host_k;
+  out->host_v = st->host_v;
+  out->slot_k = st->slot_k;
+  out->slot_v = st->slot_v;
+  out->state = static_cast<unsigned char*>(st->state);
+  return HSA_OK;
+}
+
+size_t hkv_store_state_size(int NP, int S) {
+  if (NP < 1 || S < 1) return 0;
+  return hsa::store_state_bytes(NP, S);
+}
+
+hsa_status_t hkv_store_init(const hkv_store_t* st, hsa_stream_t stream) {
+  const char* fn = __func__;
+  hsa::StoreDesc sd;
+  TRY(store_desc(fn, st, &sd));
+  HSA_LAUNCH("store_init", hsa::launch_store_init(sd, stream));
+  return HSA_OK;
+}
+
+hsa_status_t hkv_store_tables(const hkv_store_t* st, const hsa_bf16* const** table_k,
+                              const hsa_bf16* const** table_v) {
+  const char* fn = __func__;
+  hsa::StoreDesc sd;
+  TRY(store_desc(fn, st, &sd));
+  if (!table_k || !table_v) return fail(HSA_ERR_INVALID_ARG, "%s: NULL output", fn);
+  unsigned char* base = static_cast<unsigned char*>(st->state);
+  *table_k = reinterpret_cast<const hsa_bf16* const*>(base + hsa::store_table_offset(st->NP, 0));
+  *table_v = reinterpret_cast<const hsa_bf16* const*>(base + hsa::store_table_offset(st->NP, 1));
+  return HSA_OK;
+}
+
+hsa_status_t hkv_store_seal(const hkv_store_t* st, int page, const hsa_bf16* K_rows, const hsa_bf16* V_rows,
+                            float* kbar_out, void* ws, size_t ws_bytes, hsa_stream_t stream) {
+  const char* fn = __func__;
+  hsa::StoreDesc sd;
+  TRY(store_desc(fn, st, &sd));
+  if (page < 0 || page >= st->NP) return fail(HSA_ERR_INVALID_ARG, "%s: page %d outside [0, %d)", fn, page, st->NP);
+  REQUIRE_PTR(K_rows);
+  REQUIRE_PTR(V_rows);
+  REQUIRE_PTR(kbar_out);
+  const Layout L = make_layout(st->H, st->d, 1, 0, 0);
+  TRY(check_ws(fn, ws, ws_bytes, L.pages_end));
+  const long long pe = (long long)st->P_tok * sd.C;
+  float* part = at<float>(ws, L.colpart);
+  // K: the copy into the host tier and the page summary in one pass; V: a plain copy
+  HSA_LAUNCH("seal_colsum", hsa::launch_colsum_partial(K_rows, st->P_tok, sd.C, part, st->host_k + page * pe, stream));
+  HSA_LAUNCH("page_summary_final", hsa::launch_page_summary_final(part, st->P_tok, sd.C, kbar_out, stream));
+  cudaError_t e = cudaMemcpyAsync(st->host_v + page * pe, V_rows, (size_t)pe * 2, cudaMemcpyDefault, stream);
+  if (e != cudaSuccess) return fail(HSA_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(e));
+  return HSA_OK;
+}
+
+hsa_status_t hkv_store_fetch(const hkv_store_t* st, const int32_t* sel, int Kp, void* ws, size_t ws_bytes,
+                             hsa_stream_t stream) {
+  const char* fn = __func__;
+  hsa::StoreDesc sd;
+  TRY(store_desc(fn, st, &sd));
+  if (Kp < 1 || Kp > st->NP) return fail(HSA_ERR_INVALID_ARG, "%s: Kp = %d must be in [1, NP]", fn, Kp);
+  if (!sel) return fail(HSA_ERR_INVALID_ARG, "%s: sel is NULL", fn);
+  TRY(check_ws(fn, ws, ws_bytes, 256));
+  HSA_LAUNCH("store_fetch", hsa::launch_store_fetch(sd, sel, Kp, status_of(ws), stream));
+  return HSA_OK;
+}
+
+hsa_status_t hkv_store_prefetch(const hkv_store_t* st, const float* scores, const int32_t* protect, int n_protect,
+                                int m, void* ws, size_t ws_bytes, hsa_stream_t stream) {
+  const char* fn = __func__;
+  hsa::StoreDesc sd;
+  TRY(store_desc(fn, st, &sd));
+  if (!scores) return fail(HSA_ERR_INVALID_ARG, "%s: scores is NULL", fn);
+  if (n_protect < 0 || (n_protect > 0 && !protect)) return fail(HSA_ERR_INVALID_ARG, "%s: bad protect list", fn);
+  if (m < 0) return fail(HSA_ERR_INVALID_ARG, "%s: m = %d must be >= 0", fn, m);
+  TRY(check_ws(fn, ws, ws_bytes, 256));
+  HSA_LAUNCH("store_prefetch", hsa::launch_store_prefetch(sd, scores, protect, n_protect, m, status_of(ws), stream));
+  return HSA_OK;
+}
+
+hsa_status_t hkv_store_residency(const hkv_store_t* st, int32_t* slot_of_page, int32_t* page_of_slot,
+                                 hsa_stream_t stream) {
+  const char* fn = __func__;
+  hsa::StoreDesc sd;
+  TRY(store_desc(fn, st, &sd));
+  if (!slot_of_page && !page_of_slot) return fail(HSA_ERR_INVALID_ARG, "%s: no output", fn);
+  HSA_LAUNCH("store_slots", hsa::launch_store_slots(sd, slot_of_page, page_of_slot, stream));
+  return HSA_OK;
+}
+
 // ------------------------------------------------------------------ HSA
 
 static hsa_status_t run_block_select(const hsa_config_t* cfg, const Layout& L, const hsa_bf16* Q, const hsa_bf16* Kc,
@@ -437,19 +544,26 @@ static hsa_status_t run_plan(const Layout& L, const hsa_selection_t& sel, void* 
 }
 
 // Linformer projection (EK, FV as split-bf16 pairs in the workspace); sets the
-// linear-branch fields of `a`.
+// linear-branch fields of `a`.  which_part = kProjAll projects the whole active KV;
+// kProjChunk projects only the current chunk's KV and adds the cached KV's products
+// that hsa_prepare_history left in the workspace.
 static hsa_status_t run_projection(const hsa_config_t* cfg, const Layout& L, const hsa_bf16* Kc, const hsa_bf16* Vc,
                                    const hsa_bf16* Kq, const hsa_bf16* Vq, const hsa_bf16* E, const hsa_bf16* F,
-                                   long long ef_head_stride, void* ws, hsa::AttnArgs& a, hsa_stream_t stream) {
+                                   long long ef_head_stride, void* ws, hsa::AttnArgs& a, int which_part,
+                                   hsa_stream_t stream) {
   float* part = at<float>(ws, L.projpart);
   uint16_t* ekhi = at<uint16_t>(ws, L.ekhi);
   uint16_t* eklo = at<uint16_t>(ws, L.eklo);
   uint16_t* fvhi = at<uint16_t>(ws, L.fvhi);
   uint16_t* fvlo = at<uint16_t>(ws, L.fvlo);
+  int splits = hsa::proj_tc_splits(cfg->H, cfg->d, cfg->rank, cfg->Lc, cfg->Lq, which_part);
+  if (splits > L.splits) splits = L.splits;
   HSA_LAUNCH("linformer_proj", hsa::launch_proj_tc(E, F, ef_head_stride, Kc, Kq, Vc, Vq, cfg->H, cfg->d, cfg->rank,
-                                                   cfg->Lc, cfg->Lq, L.splits, part, status_of(ws), stream));
-  HSA_LAUNCH("linformer_reduce", hsa::launch_proj_reduce(part, L.splits, cfg->H, cfg->d, cfg->rank, ekhi, eklo, fvhi,
-                                                         fvlo, stream));
+                                                   cfg->Lc, cfg->Lq, which_part, splits, part, status_of(ws),
+                                                   stream));
+  const float* add = which_part == hsa::kProjChunk ? at<float>(ws, L.ekfv_hist) : nullptr;
+  HSA_LAUNCH("linformer_reduce", hsa::launch_proj_reduce(part, splits, cfg->H, cfg->d, cfg->rank, add, nullptr, ekhi,
+                                                         eklo, fvhi, fvlo, stream));
   a.EKhi = ekhi; a.EKlo = eklo; a.FVhi = fvhi; a.FVlo = fvlo;
   return HSA_OK;
 }
@@ -512,18 +626,18 @@ hsa_status_t hsa_linear_attn(const hsa_config_t* cfg, const hsa_bf16* Q, const h
   const Layout L = make_layout(cfg->H, cfg->d, cfg->Lq, cfg->Lc, cfg->rank);
   TRY(check_ws(fn, ws, ws_bytes, L.total));
   hsa::AttnArgs a = attn_args(cfg, L, ws, Q, Kc, Vc, Kq, Vq);
-  TRY(run_projection(cfg, L, Kc, Vc, Kq, Vq, E, F, ef_head_stride, ws, a, stream));
+  TRY(run_projection(cfg, L, Kc, Vc, Kq, Vq, E, F, ef_head_stride, ws, a, hsa::kProjAll, stream));
   a.out_f32 = o_linear;
   HSA_LAUNCH("attention", hsa::launch_attn_tc(a, stream));
   return HSA_OK;
 }
 
-hsa_status_t hsa_forward(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc, const hsa_bf16* Vc,
-                         const hsa_bf16* Kq, const hsa_bf16* Vq, const float* kbar128, const float* tau,
-                         const float* gate_logit, const hsa_bf16* E, const hsa_bf16* F, long long ef_head_stride,
-                         void* out, int out_is_bf16, const hsa_selection_t* sel_out, void* ws, size_t ws_bytes,
-                         hsa_stream_t stream) {
-  const char* fn = __func__;
+static hsa_status_t forward_impl(const char* fn, const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc,
+                                 const hsa_bf16* Vc, const hsa_bf16* Kq, const hsa_bf16* Vq, const float* kbar128,
+                                 const float* tau, const float* gate_logit, const hsa_bf16* E, const hsa_bf16* F,
+                                 long long ef_head_stride, void* out, int out_is_bf16,
+                                 const hsa_selection_t* sel_out, void* ws, size_t ws_bytes, int which_part,
+                                 hsa_stream_t stream) {
   TRY(check_cfg(fn, cfg, true));
   TRY(check_tensors(fn, cfg, Q, Kc, Vc, Kq, Vq, true));
   OPTIONAL_PTR(kbar128);
@@ -555,7 +669,7 @@ hsa_status_t hsa_forward(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_b
   if (e == cudaSuccess) e = cudaEventRecord(side->fork, stream);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(side->s, side->fork, 0);
   if (e != cudaSuccess) return fail(HSA_ERR_CUDA, "%s: side stream: %s", fn, cudaGetErrorString(e));
-  TRY(run_projection(cfg, L, Kc, Vc, Kq, Vq, E, F, ef_head_stride, ws, a, side->s));
+  TRY(run_projection(cfg, L, Kc, Vc, Kq, Vq, E, F, ef_head_stride, ws, a, which_part, side->s));
   if ((e = cudaEventRecord(side->join, side->s)) != cudaSuccess)
     return fail(HSA_ERR_CUDA, "%s: side stream: %s", fn, cudaGetErrorString(e));
   TRY(run_block_select(cfg, L, Q, Kc, Kq, kbar128, tau, sel, ws, stream));
@@ -567,6 +681,54 @@ hsa_status_t hsa_forward(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_b
   else a.out_f32 = static_cast<float*>(out);
   HSA_LAUNCH("attention_merge", hsa::launch_attn_tc(a, stream));
   return HSA_OK;
+}
+
+hsa_status_t hsa_forward(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc, const hsa_bf16* Vc,
+                         const hsa_bf16* Kq, const hsa_bf16* Vq, const float* kbar128, const float* tau,
+                         const float* gate_logit, const hsa_bf16* E, const hsa_bf16* F, long long ef_head_stride,
+                         void* out, int out_is_bf16, const hsa_selection_t* sel_out, void* ws, size_t ws_bytes,
+                         hsa_stream_t stream) {
+  return forward_impl(__func__, cfg, Q, Kc, Vc, Kq, Vq, kbar128, tau, gate_logit, E, F, ef_head_stride, out,
+                      out_is_bf16, sel_out, ws, ws_bytes, hsa::kProjAll, stream);
+}
+
+hsa_status_t hsa_prepare_history(const hsa_config_t* cfg, const hsa_bf16* Kc, const hsa_bf16* Vc, const hsa_bf16* E,
+                                 const hsa_bf16* F, long long ef_head_stride, void* ws, size_t ws_bytes,
+                                 hsa_stream_t stream) {
+  const char* fn = __func__;
+  TRY(check_cfg(fn, cfg, true));
+  if (cfg->Lc > 0) {
+    REQUIRE_PTR(Kc);
+    REQUIRE_PTR(Vc);
+  }
+  REQUIRE_PTR(E);
+  REQUIRE_PTR(F);
+  if (ef_head_stride != 0 && ef_head_stride != (long long)cfg->rank * (cfg->Lc + cfg->Lq))
+    return fail(HSA_ERR_UNSUPPORTED, "%s: ef_head_stride must be 0 (shared) or r * (Lc + Lq) (stacked per head)", fn);
+  const Layout L = make_layout(cfg->H, cfg->d, cfg->Lq, cfg->Lc, cfg->rank);
+  TRY(check_ws(fn, ws, ws_bytes, L.total));
+  float* part = at<float>(ws, L.projpart);
+  int splits = hsa::proj_tc_splits(cfg->H, cfg->d, cfg->rank, cfg->Lc, cfg->Lq, hsa::kProjCached);
+  if (splits > L.splits) splits = L.splits;
+  // the chunk tensors are not read by this launch; their maps point at the history
+  const hsa_bf16* Kq = cfg->Lc > 0 ? Kc : E;
+  const hsa_bf16* Vq = cfg->Lc > 0 ? Vc : F;
+  HSA_LAUNCH("linformer_proj_history",
+             hsa::launch_proj_tc(E, F, ef_head_stride, Kc, Kq, Vc, Vq, cfg->H, cfg->d, cfg->rank, cfg->Lc, cfg->Lq,
+                                 hsa::kProjCached, splits, part, status_of(ws), stream));
+  HSA_LAUNCH("linformer_reduce_history",
+             hsa::launch_proj_reduce(part, splits, cfg->H, cfg->d, cfg->rank, nullptr, at<float>(ws, L.ekfv_hist),
+                                     nullptr, nullptr, nullptr, nullptr, stream));
+  return HSA_OK;
+}
+
+hsa_status_t hsa_forward_reuse(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc, const hsa_bf16* Vc,
+                               const hsa_bf16* Kq, const hsa_bf16* Vq, const float* kbar128, const float* tau,
+                               const float* gate_logit, const hsa_bf16* E, const hsa_bf16* F,
+                               long long ef_head_stride, void* out, int out_is_bf16, const hsa_selection_t* sel_out,
+                               void* ws, size_t ws_bytes, hsa_stream_t stream) {
+  return forward_impl(__func__, cfg, Q, Kc, Vc, Kq, Vq, kbar128, tau, gate_logit, E, F, ef_head_stride, out,
+                      out_is_bf16, sel_out, ws, ws_bytes, hsa::kProjChunk, stream);
 }
 
 }  // extern "C"

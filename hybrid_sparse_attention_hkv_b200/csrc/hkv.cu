@@ -16,8 +16,11 @@ namespace hsa {
 // part[s][c] = sum over the rows of split s of X[row][c]; X: [n, C] bf16, C % 8 == 0.
 // A CTA owns a contiguous row range; thread t reads 16-byte column vector (t % CV)
 // of rows r0 + (t / CV), r0 + (t / CV) + RP, ...  (RP = 256 / CV row phases).
+// copy_dst (optional): every row read is also written there (page seal: the copy
+// into the store and the summary in one pass).
 __global__ void __launch_bounds__(256) colsum_partial_kernel(const uint16_t* __restrict__ X, long long n, int C,
-                                                             long long rows_per_split, float* __restrict__ part) {
+                                                             long long rows_per_split, float* __restrict__ part,
+                                                             uint16_t* __restrict__ copy_dst) {
   __shared__ float red[2048];
   const int CV = C / 8;
   const long long r0 = (long long)blockIdx.x * rows_per_split;
@@ -29,7 +32,11 @@ __global__ void __launch_bounds__(256) colsum_partial_kernel(const uint16_t* __r
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (rp < RP) {
 #pragma unroll 4
-      for (long long r = r0 + rp; r < r1; r += RP) add8(acc, ld_nc_v4(X + r * C + v * 8));
+      for (long long r = r0 + rp; r < r1; r += RP) {
+        const uint4 w = ld_nc_v4(X + r * C + v * 8);
+        if (copy_dst) *reinterpret_cast<uint4*>(copy_dst + r * C + v * 8) = w;
+        add8(acc, w);
+      }
 #pragma unroll
       for (int k = 0; k < 8; ++k) red[rp * C + v * 8 + k] = acc[k];
     }
@@ -43,7 +50,11 @@ __global__ void __launch_bounds__(256) colsum_partial_kernel(const uint16_t* __r
     for (int v = threadIdx.x; v < CV; v += 256) {
       float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll 4
-      for (long long r = r0; r < r1; ++r) add8(acc, ld_nc_v4(X + r * C + v * 8));
+      for (long long r = r0; r < r1; ++r) {
+        const uint4 w = ld_nc_v4(X + r * C + v * 8);
+        if (copy_dst) *reinterpret_cast<uint4*>(copy_dst + r * C + v * 8) = w;
+        add8(acc, w);
+      }
 #pragma unroll
       for (int k = 0; k < 8; ++k) out[v * 8 + k] = acc[k];
     }
@@ -70,10 +81,11 @@ __device__ __forceinline__ float sum_splits(const float* __restrict__ part, int 
   return (a0 + a1) + (a2 + a3);
 }
 
-cudaError_t launch_colsum_partial(const uint16_t* X, long long n, int C, float* part, cudaStream_t s) {
+cudaError_t launch_colsum_partial(const uint16_t* X, long long n, int C, float* part, uint16_t* copy_dst,
+                                  cudaStream_t s) {
   int splits = colsum_splits(n);
   long long rps = (n + splits - 1) / splits;
-  colsum_partial_kernel<<<splits, 256, 0, s>>>(X, n, C, rps, part);
+  colsum_partial_kernel<<<splits, 256, 0, s>>>(X, n, C, rps, part, copy_dst);
   return cudaGetLastError();
 }
 

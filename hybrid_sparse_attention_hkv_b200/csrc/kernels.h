@@ -17,7 +17,8 @@ hsa_status_t api_fail(hsa_status_t code, const char* fmt, ...);
 constexpr int kColMaxSplits = 296;  // 2 CTAs per SM for the column-sum partial pass
 
 int colsum_splits(long long n);  // number of row splits used for n rows
-cudaError_t launch_colsum_partial(const uint16_t* X, long long n, int C, float* part, cudaStream_t s);
+cudaError_t launch_colsum_partial(const uint16_t* X, long long n, int C, float* part, uint16_t* copy_dst,
+                                  cudaStream_t s);
 cudaError_t launch_page_summary_final(const float* part, long long n, int C, float* kbar, cudaStream_t s);
 // Page-level retrieval: partial scores per row split of Q (pass 1), then one CTA
 // adds them, ranks the candidates and writes the top Kp ascending (pass 2).
@@ -32,6 +33,26 @@ cudaError_t launch_select_prompt(const float* e_cur, const float* e_seg, int n_s
 cudaError_t launch_gather(const uint16_t* const* page_k, const uint16_t* const* page_v, int NP,
                           const int32_t* sel, int Kp, long long P_tok, int H, int d, uint16_t* Kc,
                           uint16_t* Vc, float* kbar128, int* status, cudaStream_t s);
+
+// ---------------------------------------------------------------- store.cu
+// Tiered page store: device-side residency state (layout in store.cu).
+struct StoreDesc {
+  int NP, S;
+  long long P_tok;
+  int C;                   // H * d
+  const uint16_t* host_k;  // [NP][P_tok][C] (device view of mapped page-locked host memory)
+  const uint16_t* host_v;
+  uint16_t* slot_k;        // [S][P_tok][C] device memory
+  uint16_t* slot_v;
+  unsigned char* state;
+};
+size_t store_state_bytes(int NP, int S);
+size_t store_table_offset(int NP, int kv);  // byte offset of the K (kv = 0) or V page table
+cudaError_t launch_store_init(const StoreDesc& st, cudaStream_t s);
+cudaError_t launch_store_fetch(const StoreDesc& st, const int32_t* sel, int Kp, int* status, cudaStream_t s);
+cudaError_t launch_store_prefetch(const StoreDesc& st, const float* scores, const int32_t* protect, int n_protect,
+                                  int m, int* status, cudaStream_t s);
+cudaError_t launch_store_slots(const StoreDesc& st, int32_t* slot_of_page, int32_t* page_of_slot, cudaStream_t s);
 
 // ---------------------------------------------------------------- select.cu
 constexpr int kMaxSelBlocks = 8192;  // blocks per selection row (inter: ceil(Lc/128), intra: ceil(Lq/64))
@@ -98,13 +119,22 @@ inline int plan_max_slots() { return 2 * kPlanSMs * kPlanUnitsPerSM + 2; }
 
 // ---------------------------------------------------------------- proj.cu
 // tcgen05 / TMEM / TMA projection (proj_tc.cu): partial sums [splits][2][H][r][d] fp32
-// (EK then FV), reduced by launch_proj_reduce (proj.cu).
-int proj_tc_splits(int H, int d, int r, long long Lc, int Lq);
+// (EK then FV), reduced by launch_proj_reduce (proj.cu).  A launch covers the rows of
+// the whole active KV (kProjAll), of the cached KV only (kProjCached: the part that
+// stays fixed over a chunk's denoising steps) or of the current chunk only (kProjChunk).
+constexpr int kProjAll = 0;
+constexpr int kProjCached = 1;
+constexpr int kProjChunk = 2;
+int proj_tc_splits(int H, int d, int r, long long Lc, int Lq, int which_part);
 cudaError_t launch_proj_tc(const uint16_t* E, const uint16_t* F, long long ef_head_stride, const uint16_t* Kc,
                            const uint16_t* Kq, const uint16_t* Vc, const uint16_t* Vq, int H, int d, int r,
-                           long long Lc, int Lq, int splits, float* part, int* status, cudaStream_t s);
-cudaError_t launch_proj_reduce(const float* part, int splits, int H, int d, int r, uint16_t* EKhi,
-                               uint16_t* EKlo, uint16_t* FVhi, uint16_t* FVlo, cudaStream_t s);
+                           long long Lc, int Lq, int which_part, int splits, float* part, int* status,
+                           cudaStream_t s);
+// Sum the split partials in a fixed order, plus `add` ([2][H][r][d] fp32, nullable):
+// into fp32 sums `sum_out` when it is given, else into the split-bf16 pairs.
+cudaError_t launch_proj_reduce(const float* part, int splits, int H, int d, int r, const float* add,
+                               float* sum_out, uint16_t* EKhi, uint16_t* EKlo, uint16_t* FVhi, uint16_t* FVlo,
+                               cudaStream_t s);
 
 // ---------------------------------------------------------------- waits.cu
 // Write the wait limit (microseconds; 0 = the 2 s default) into a workspace header.

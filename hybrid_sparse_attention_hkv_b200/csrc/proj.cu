@@ -10,8 +10,10 @@
 
 namespace hsa {
 
-// Sum the split partials (fixed order) and store hi = bf16(v), lo = bf16(v - hi).
+// Sum the split partials (fixed order), add `add` when given, and store either the
+// fp32 sums (sum_out) or hi = bf16(v), lo = bf16(v - hi).
 __global__ void proj_reduce_kernel(const float* __restrict__ part, int splits, long long per_which,
+                                   const float* __restrict__ add, float* __restrict__ sum_out,
                                    uint16_t* __restrict__ EKhi, uint16_t* __restrict__ EKlo,
                                    uint16_t* __restrict__ FVhi, uint16_t* __restrict__ FVlo) {
   const long long i4 = (long long)blockIdx.x * blockDim.x + threadIdx.x;  // float4 index over 2 * per_which
@@ -23,6 +25,14 @@ __global__ void proj_reduce_kernel(const float* __restrict__ part, int splits, l
   for (int s = 0; s < splits; ++s) {
     const float4 v = *reinterpret_cast<const float4*>(part + ((long long)s * 2 + which) * per_which + off);
     acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+  }
+  if (add) {
+    const float4 v = *reinterpret_cast<const float4*>(add + e);
+    acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+  }
+  if (sum_out) {
+    *reinterpret_cast<float4*>(sum_out + e) = acc;
+    return;
   }
   __nv_bfloat16 h[4], l[4];
   split_bf16(acc.x, h[0], l[0]);
@@ -40,11 +50,13 @@ __global__ void proj_reduce_kernel(const float* __restrict__ part, int splits, l
   *reinterpret_cast<uint2*>(lo + off) = lv;
 }
 
-cudaError_t launch_proj_reduce(const float* part, int splits, int H, int d, int r, uint16_t* EKhi,
-                               uint16_t* EKlo, uint16_t* FVhi, uint16_t* FVlo, cudaStream_t s) {
+cudaError_t launch_proj_reduce(const float* part, int splits, int H, int d, int r, const float* add,
+                               float* sum_out, uint16_t* EKhi, uint16_t* EKlo, uint16_t* FVhi, uint16_t* FVlo,
+                               cudaStream_t s) {
   const long long per_which = (long long)H * r * d;
   const long long n4 = 2 * per_which / 4;
-  proj_reduce_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, s>>>(part, splits, per_which, EKhi, EKlo, FVhi, FVlo);
+  proj_reduce_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, s>>>(part, splits, per_which, add, sum_out, EKhi, EKlo,
+                                                                  FVhi, FVlo);
   return cudaGetLastError();
 }
 

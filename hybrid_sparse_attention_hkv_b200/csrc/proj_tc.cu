@@ -43,6 +43,7 @@ struct PjArgs {
   int per_head;      // E/F maps hold H stacked [r, L] matrices
   int n_chunks_c;    // ceil(Lc / 64)
   int n_chunks;      // n_chunks_c + ceil(Lq / 64)
+  int chunk_lo, chunk_hi;  // chunks [chunk_lo, chunk_hi) of [0, n_chunks) make up this launch
   int chunks_per_split;
   float* part;       // [splits][2][H][r][D]
   int* status;
@@ -75,8 +76,8 @@ __global__ void __launch_bounds__(kPjThreads, 1) proj_tc_kernel(const __grid_con
   const uint64_t wlim = wait_limit_ns(a.status);
   const int rg = blockIdx.x, h0 = blockIdx.y * HP;  // first head of this CTA
   const int which = blockIdx.z & 1, split = blockIdx.z >> 1;
-  const int c_begin = split * a.chunks_per_split;
-  const int c_end = min(a.n_chunks, c_begin + a.chunks_per_split);
+  const int c_begin = a.chunk_lo + split * a.chunks_per_split;
+  const int c_end = min(a.chunk_hi, c_begin + a.chunks_per_split);
   const int nc = max(0, c_end - c_begin);
   const CUtensorMap* mE = which ? &maps.f : &maps.e;
   const CUtensorMap* mBc = which ? &maps.vc : &maps.kc;
@@ -241,10 +242,16 @@ int proj_tiles_per_cta(int r, int d, int hp) {
 
 }  // namespace
 
-// Splits of L chosen for the shared-E launch (the workspace is sized with them); a
-// per-head-E launch uses the same count with twice the CTAs.
-int proj_tc_splits(int H, int d, int r, long long Lc, int Lq) {
-  const long long chunks = (Lc + kChunk - 1) / kChunk + (Lq + kChunk - 1) / kChunk;
+// Splits of the chunk range of a launch (`part` selects all chunks, the cached KV's
+// or the current chunk's), chosen for the shared-E launch (the workspace is sized
+// with the largest); a per-head-E launch uses the same count with twice the CTAs.
+static long long part_chunks(long long Lc, int Lq, int part) {
+  const long long cc = (Lc + kChunk - 1) / kChunk, cq = (Lq + kChunk - 1) / kChunk;
+  return part == kProjCached ? cc : (part == kProjChunk ? cq : cc + cq);
+}
+
+int proj_tc_splits(int H, int d, int r, long long Lc, int Lq, int part) {
+  const long long chunks = part_chunks(Lc, Lq, part);
   const int hp = proj_heads_per_cta(H, false);
   const int mt = proj_tiles_per_cta(r, d, hp);
   const int groups = ((r + 127) / 128 + mt - 1) / mt;
@@ -265,7 +272,8 @@ int proj_tc_splits(int H, int d, int r, long long Lc, int Lq) {
 
 cudaError_t launch_proj_tc(const uint16_t* E, const uint16_t* F, long long ef_head_stride, const uint16_t* Kc,
                            const uint16_t* Kq, const uint16_t* Vc, const uint16_t* Vq, int H, int d, int r,
-                           long long Lc, int Lq, int splits, float* part, int* status, cudaStream_t s) {
+                           long long Lc, int Lq, int which_part, int splits, float* part, int* status,
+                           cudaStream_t s) {
   cudaError_t e = encoder();
   if (e != cudaSuccess) return e;
   const long long L = Lc + Lq;
@@ -283,7 +291,9 @@ cudaError_t launch_proj_tc(const uint16_t* E, const uint16_t* F, long long ef_he
   a.per_head = ef_head_stride != 0;
   a.n_chunks_c = (int)((Lc + kChunk - 1) / kChunk);
   a.n_chunks = a.n_chunks_c + (Lq + kChunk - 1) / kChunk;
-  a.chunks_per_split = (a.n_chunks + splits - 1) / splits;
+  a.chunk_lo = which_part == kProjChunk ? a.n_chunks_c : 0;
+  a.chunk_hi = which_part == kProjCached ? a.n_chunks_c : a.n_chunks;
+  a.chunks_per_split = (a.chunk_hi - a.chunk_lo + splits - 1) / splits;
   a.part = part;
   a.status = status;
   const int hp = proj_heads_per_cta(H, a.per_head != 0);

@@ -12,7 +12,7 @@ from __future__ import annotations
 import torch
 
 from . import (SelectionBuffers, hkv_gather, hkv_page_summary, hkv_select_pages, hkv_select_prompt,
-               hsa_forward, hsa_workspace_size, make_config)
+               hsa_forward, hsa_forward_reuse, hsa_prepare_history, hsa_workspace_size, make_config)
 
 
 def page_pointers(pages: torch.Tensor) -> torch.Tensor:
@@ -26,8 +26,12 @@ def page_pointers(pages: torch.Tensor) -> torch.Tensor:
 
 class HkvHsaStep:
     def __init__(self, H, d, Lq, P_tok, NP, Kp, rank, page_k_ptrs, page_v_ptrs, out_dtype=torch.float32,
-                 scale=0.0, device="cuda"):
+                 scale=0.0, device="cuda", store=None):
+        """page_k_ptrs / page_v_ptrs: device int64 page tables read by the gather.  With a
+        tiered page store (`store`, a PageStore), pass its tables: every retrieval is
+        then followed by the store's fetch (the selected pages made resident in HBM)."""
         self.H, self.d, self.Lq, self.P_tok, self.NP, self.Kp, self.rank = H, d, Lq, P_tok, NP, Kp, rank
+        self.store = store
         self.Lc = Kp * P_tok
         self.cfg = make_config(H, d, Lq, self.Lc, rank, scale)
         dev = torch.device(device)
@@ -59,8 +63,40 @@ class HkvHsaStep:
             hkv_select_prompt(e_cur, e_seg, seg_begin, self.seg, self.cand_range)
             cand = self.cand_range
         hkv_select_pages(self.kbar_pages, Q, self.Kp, self.sel, self.ws, self.scores, cand)
+        if self.store is not None:
+            self.store.fetch(self.sel, self.ws)
         hkv_gather(self.page_k_ptrs, self.page_v_ptrs, self.sel, self.Kp, self.P_tok, self.H, self.d,
                    self.Kc, self.Vc, self.ws, self.kbar128)
         hsa_forward(self.cfg, Q, self.Kc, self.Vc, Kq, Vq, tau, gate_logit, E, F, dst, self.ws,
                     self.kbar128, self.selection, ef_head_stride)
         return dst
+
+    # ------------------------------------------------------------ multi-step reuse
+    def prepare_chunk(self, Q, E, F, e_cur=None, e_seg=None, seg_begin=None, ef_head_stride=0):
+        """Once per chunk: retrieval (prompt-level, page-level) with the chunk's queries,
+        the gather of the active cache, and the cached KV's Linformer products."""
+        cand = None
+        if e_cur is not None:
+            hkv_select_prompt(e_cur, e_seg, seg_begin, self.seg, self.cand_range)
+            cand = self.cand_range
+        hkv_select_pages(self.kbar_pages, Q, self.Kp, self.sel, self.ws, self.scores, cand)
+        if self.store is not None:
+            self.store.fetch(self.sel, self.ws)
+        hkv_gather(self.page_k_ptrs, self.page_v_ptrs, self.sel, self.Kp, self.P_tok, self.H, self.d,
+                   self.Kc, self.Vc, self.ws, self.kbar128)
+        hsa_prepare_history(self.cfg, self.Kc, self.Vc, E, F, self.ws, ef_head_stride)
+
+    def denoise_step(self, Q, Kq, Vq, tau, gate_logit, E, F, ef_head_stride=0, out=None):
+        """One denoising step of the prepared chunk (block selection, both branches, merge)."""
+        dst = self.out if out is None else out
+        hsa_forward_reuse(self.cfg, Q, self.Kc, self.Vc, Kq, Vq, tau, gate_logit, E, F, dst, self.ws,
+                          self.kbar128, self.selection, ef_head_stride)
+        return dst
+
+    def prefetch(self, m, ws, stream=None):
+        """Speculative promotion of the m best-scoring pages not selected by the last
+        retrieval (its scores), e.g. on a side stream during the chunk's denoising
+        steps.  `ws` is a workspace of its own (its status word), so that it does not
+        race with the steps' use of self.ws."""
+        if self.store is not None:
+            self.store.prefetch(self.scores, self.sel, m, ws, stream)

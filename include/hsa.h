@@ -198,6 +198,78 @@ hsa_status_t hkv_select_pages_noalloc(const float* kbar_pages, int NP, const int
                                       int32_t* sel_out, float* scores_out, int32_t* status_out,
                                       hsa_stream_t stream);
 
+/* ------------------------------------------------- tiered page store ---- */
+
+/* Hierarchical KV page store ([NEWS] HKV paragraph: pages live in a hierarchy of
+ * memories ranked by cost, unselected pages are demoted to cheaper memory and GPU
+ * occupancy stays bounded; [PROJ] "three-tier hierarchical KV cache").  Two tiers:
+ * every sealed page in page-locked host memory mapped into the device address
+ * space (its authoritative copy: pages do not change once sealed), and up to S
+ * pages also in an HBM slot pool.  The store keeps, on the device, a page table
+ * (per page, the address hkv_gather reads: its slot when resident, else its host
+ * copy) and the residency state; every decision is made on the device from the
+ * device-side selection, in a fixed order, so no call waits for the host.
+ * The caller allocates all memory:
+ *   host_k, host_v  device view of mapped page-locked host memory, [NP][P_tok][H][d]
+ *   slot_k, slot_v  device memory, [S][P_tok][H][d]
+ *   state           device memory of hkv_store_state_size(NP, S) bytes, 256-aligned
+ * Calls on one store must be ordered (one stream, or events). */
+typedef struct {
+  int NP;            /* pages of the host tier */
+  int S;             /* HBM slots */
+  int P_tok, H, d;   /* page geometry */
+  hsa_bf16* host_k;
+  hsa_bf16* host_v;
+  hsa_bf16* slot_k;
+  hsa_bf16* slot_v;
+  void* state;
+} hkv_store_t;
+
+/* Bytes of the state buffer (0 for NP < 1 or S < 1). */
+size_t hkv_store_state_size(int NP, int S);
+
+/* Every page on the host tier, every slot free (enqueued on `stream`). */
+hsa_status_t hkv_store_init(const hkv_store_t* st, hsa_stream_t stream);
+
+/* Device addresses of the store's K and V page tables (arrays of NP page
+ * pointers inside `state`), to pass to hkv_gather.  Host-only, launches nothing. */
+hsa_status_t hkv_store_tables(const hkv_store_t* st, const hsa_bf16* const** table_k,
+                              const hsa_bf16* const** table_v);
+
+/* Seal page `page` ([NEWS] HKV paragraph: pages of Psize frames): copy its P_tok
+ * rows K_rows, V_rows ([P_tok, H, d] bf16, device) into the host tier and write
+ * its summary kbar_out[H*d] (the mean key per head, as hkv_page_summary) in the
+ * same pass over K.  Uses the workspace (hsa_workspace_size with any cfg of these
+ * H, d). */
+hsa_status_t hkv_store_seal(const hkv_store_t* st, int page, const hsa_bf16* K_rows, const hsa_bf16* V_rows,
+                            float* kbar_out, void* ws, size_t ws_bytes, hsa_stream_t stream);
+
+/* Promotion on demand: make the Kp selected pages sel[0..Kp) (device int32, e.g.
+ * from hkv_select_pages) resident.  A resident page is touched (its slot's
+ * last-use tick set to this call's); a missing page takes the lowest free slot,
+ * else the least recently used slot whose page is not selected (ties -> lower
+ * slot), whose page is demoted to the host tier; the page is then copied from the
+ * host tier into the slot over the host link.  Fewer slots than missing pages, or
+ * an out-of-range page id, set HSA_ERR_DEVICE in the workspace status (such a
+ * page stays on the host tier and hkv_gather still reads it there). */
+hsa_status_t hkv_store_fetch(const hkv_store_t* st, const int32_t* sel, int Kp, void* ws, size_t ws_bytes,
+                             hsa_stream_t stream);
+
+/* Speculative promotion: of the pages outside protect[0..n_protect) (device
+ * int32; typically the current selection) with a finite score in scores[NP]
+ * (device fp32, e.g. hkv_select_pages' scores_out), the m best (score descending,
+ * ties -> lower page) are made resident in that order, as hkv_store_fetch would,
+ * but never evicting a protected page or one made resident by this call; stops
+ * when no slot is left.  Meant for a side stream while a chunk's denoising steps
+ * run, so that the next chunk's fetch finds its pages in HBM. */
+hsa_status_t hkv_store_prefetch(const hkv_store_t* st, const float* scores, const int32_t* protect, int n_protect,
+                                int m, void* ws, size_t ws_bytes, hsa_stream_t stream);
+
+/* Copy the residency state out: slot_of_page[NP] (-1 = host tier only) and
+ * page_of_slot[S] (-1 = free); either may be NULL.  Device int32 buffers. */
+hsa_status_t hkv_store_residency(const hkv_store_t* st, int32_t* slot_of_page, int32_t* page_of_slot,
+                                 hsa_stream_t stream);
+
 /* ---------------------------------------------------------------- HSA ---- */
 
 /* Head-adaptive block selection ([NEWS] HSA paragraph).  Pools Q and Kc into
@@ -250,6 +322,31 @@ hsa_status_t hsa_forward(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_b
                          const hsa_bf16* E, const hsa_bf16* F, long long ef_head_stride,
                          void* out, int out_is_bf16, const hsa_selection_t* sel_out,
                          void* ws, size_t ws_bytes, hsa_stream_t stream);
+
+/* Multi-step reuse ([NEWS] HKV paragraph: retrieval assembles the active cache of
+ * the current chunk; kernel paragraph: KV reorganisation and copies dominate the
+ * preprocessing; reading: a chunk is denoised over several steps against one
+ * retrieval, so the history part of the step is done once per chunk).
+ *
+ * hsa_prepare_history projects the cached KV once per chunk:
+ *   EKc_h = E_h[:, 0:Lc] Kc_h,   FVc_h = F_h[:, 0:Lc] Vc_h        (fp32, kept in ws)
+ * hsa_forward_reuse is hsa_forward for one denoising step of that chunk: it
+ * projects only the chunk's own keys and values and adds the kept products,
+ *   EK_h = EKc_h + E_h[:, Lc:L] Kq_h,   FV_h = FVc_h + F_h[:, Lc:L] Vq_h,
+ * then selects blocks, runs both branches and merges exactly as hsa_forward (same
+ * arguments and results).  Kc, Vc, E, F and the workspace must be the ones given
+ * to the last hsa_prepare_history of this workspace; Q, Kq, Vq, tau and the gate
+ * logits may change from step to step.  kbar128 from hkv_gather stays valid for
+ * the chunk.  Both use the workspace; the kept products live in it (2 H r d fp32). */
+hsa_status_t hsa_prepare_history(const hsa_config_t* cfg, const hsa_bf16* Kc, const hsa_bf16* Vc,
+                                 const hsa_bf16* E, const hsa_bf16* F, long long ef_head_stride,
+                                 void* ws, size_t ws_bytes, hsa_stream_t stream);
+hsa_status_t hsa_forward_reuse(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc,
+                               const hsa_bf16* Vc, const hsa_bf16* Kq, const hsa_bf16* Vq,
+                               const float* kbar128, const float* tau, const float* gate_logit,
+                               const hsa_bf16* E, const hsa_bf16* F, long long ef_head_stride,
+                               void* out, int out_is_bf16, const hsa_selection_t* sel_out,
+                               void* ws, size_t ws_bytes, hsa_stream_t stream);
 
 /* Optional per-kernel timing hook (tracing).  When `events` is non-NULL, the
  * next entry-point calls on this thread record events[2*k] before and

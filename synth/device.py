@@ -49,7 +49,9 @@ class MappedHostBuffer:
 class DeviceStep:
     """Seeded inputs of one step uploaded for the GPU path, plus its HkvHsaStep."""
 
-    def __init__(self, shape: StepShape, seed: int, out_dtype=torch.float32, x=None):
+    def __init__(self, shape: StepShape, seed: int, out_dtype=torch.float32, x=None, store_slots=0):
+        """store_slots > 0 (host-pinned workloads): the pages are read through a tiered
+        page store with that many HBM slots instead of straight from the host tier."""
         from hybrid_sparse_attention_hkv_b200.step import HkvHsaStep, page_pointers
         self.shape = shape
         NP, P, H, d = shape.NP, shape.P_tok, shape.H, shape.d
@@ -68,14 +70,20 @@ class DeviceStep:
         self.tau = torch.from_numpy(x.tau).cuda()
         self.z = torch.from_numpy(x.z).cuda()
         stride = P * H * d * 2
+        self.store = None
         if self.host:
             kp = torch.tensor([self.host[0].dev_ptr + p * stride for p in range(NP)], dtype=torch.int64, device="cuda")
             vp = torch.tensor([self.host[1].dev_ptr + p * stride for p in range(NP)], dtype=torch.int64, device="cuda")
+            self.host_tables = (kp, vp)  # straight from the host tier (zero-copy gather)
             self.pages_k = self.pages_v = None
+            if store_slots:
+                from hybrid_sparse_attention_hkv_b200.store import PageStore
+                self.store = PageStore(NP, store_slots, P, H, d, host=self.host)
+                kp, vp = self.store.page_tables()
         else:
             self.pages_k, self.pages_v = to_dev(x.pages_k), to_dev(x.pages_v)
             kp, vp = page_pointers(self.pages_k), page_pointers(self.pages_v)
-        self.step = HkvHsaStep(H, d, shape.Lq, P, NP, shape.Kp, shape.r, kp, vp, out_dtype)
+        self.step = HkvHsaStep(H, d, shape.Lq, P, NP, shape.Kp, shape.r, kp, vp, out_dtype, store=self.store)
         if self.host:
             # summaries read the mapped host pages directly
             from hybrid_sparse_attention_hkv_b200 import hkv_page_summary
@@ -95,6 +103,9 @@ class DeviceStep:
                          self.E, self.F, self.e_cur, self.e_seg, self.seg_begin)
 
     def close(self):
+        if self.store is not None:
+            self.store.close()  # the host tier belongs to this object: freed below
+            self.store = None
         if self.host:
             for b in self.host:
                 b.free()

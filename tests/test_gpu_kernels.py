@@ -397,3 +397,41 @@ def test_bounded_wait_times_out_and_context_stays_usable():
     hsa.hsa_set_wait_limit(ws, 0)  # back to the default
     hsa.hsa_selftest_wait(ws)  # default limit 2 s: still a timeout, bounded
     assert hsa.hsa_status_read(ws) == 5
+
+
+# ----------------------------------------------------------------- multi-step reuse
+
+@pytest.mark.parametrize("shape", SMALL, ids=_ids)
+def test_multi_step_reuse(shape):
+    """Retrieval, gather and the history's Linformer products once per chunk; three
+    denoising steps with fresh chunk tensors.  Each step equals hsa_forward on the same
+    inputs (same selections, outputs within fp32 summation-order differences) and the
+    oracle's HSA step within the tolerance."""
+    ds = DeviceStep(shape, 55)
+    try:
+        st, x = ds.step, ds.x
+        st.prepare_chunk(ds.Q, ds.E, ds.F)
+        Kc, Vc = bits_of(st.Kc), bits_of(st.Vc)
+        Lq, H, d = shape.Lq, shape.H, shape.d
+        for k in range(3):
+            Qb = synth.normal_bf16((Lq, H, d), 600 + k, 1)
+            Kqb = synth.normal_bf16((Lq, H, d), 600 + k, 2)
+            Vqb = synth.normal_bf16((Lq, H, d), 600 + k, 3)
+            Q, Kq, Vq = to_dev(Qb), to_dev(Kqb), to_dev(Vqb)
+            out_r = st.denoise_step(Q, Kq, Vq, ds.tau, ds.z, ds.E, ds.F, out=torch.empty_like(st.out))
+            sel_f = SelectionBuffers.empty(st.cfg)
+            out_f = torch.empty_like(st.out)
+            hsa.hsa_forward(st.cfg, Q, st.Kc, st.Vc, Kq, Vq, ds.tau, ds.z, ds.E, ds.F, out_f, st.ws, st.kbar128,
+                            sel=sel_f)
+            torch.cuda.synchronize()
+            sb = st.selection
+            for a, b in ((sb.inter_cnt, sel_f.inter_cnt), (sb.intra_cnt, sel_f.intra_cnt)):
+                assert torch.equal(a, b)
+            assert float((out_r - out_f).abs().max()) <= 1e-4
+            sel = oracle.Selection(selection_lists(sb.inter_idx.cpu().numpy(), sb.inter_cnt.cpu().numpy()),
+                                   selection_lists(sb.intra_idx.cpu().numpy(), sb.intra_cnt.cpu().numpy()), None, None)
+            ref = oracle.hsa_step(Qb, Kc, Vc, Kqb, Vqb, x.tau, x.z, x.E, x.F, selection=sel)
+            assert_close(out_r.cpu().numpy(), ref["out"], f"denoising step {k}")
+        assert hsa.hsa_status_read(st.ws) == 0
+    finally:
+        ds.close()
