@@ -27,8 +27,10 @@ EXPORTED = [
     "hsa_trace_begin", "hsa_trace_count", "hsa_trace_end", "hsa_set_wait_limit", "hsa_selftest_wait",
     "hsa_thread_release", "hsa_prepare_history", "hsa_forward_reuse",
     "hkv_store_state_size", "hkv_store_init", "hkv_store_tables", "hkv_store_seal", "hkv_store_fetch",
-    "hkv_store_prefetch", "hkv_store_residency",
+    "hkv_store_prefetch", "hkv_store_residency", "hkv_select_pages_policy", "hkv_page_scores", "hkv_select_top",
 ]
+
+POLICY_SCORE, POLICY_RECENT, POLICY_RANDOM = 0, 1, 2
 
 
 class HsaError(RuntimeError):
@@ -89,6 +91,9 @@ def load_library(path: str = LIB_PATH):
         "hsa_prepare_history": (I, [CP, P, P, P, P, L, P, S, P]),
         "hsa_forward_reuse": (I, [CP, P, P, P, P, P, P, P, P, P, P, L, P, I, ctypes.POINTER(_Selection), P, S,
                                   P]),
+        "hkv_select_pages_policy": (I, [I, P, I, P, P, I, I, I, I, P, P, P, P, S, P]),
+        "hkv_page_scores": (I, [P, I, P, P, I, I, I, P, P, S, P]),
+        "hkv_select_top": (I, [P, I, P, I, P, P, S, P]),
         "hkv_store_state_size": (S, [I, I]),
         "hkv_store_init": (I, [ctypes.POINTER(StoreDesc), P]),
         "hkv_store_tables": (I, [ctypes.POINTER(StoreDesc), ctypes.POINTER(P), ctypes.POINTER(P)]),
@@ -202,6 +207,30 @@ def hkv_select_pages(kbar_pages, Q, Kp, sel_out, ws, scores_out=None, cand_range
     Lq, H, d = Q.shape
     _check(load_library().hkv_select_pages(_p(kbar_pages), NP, _p(cand_range), _p(Q), Lq, H, d, Kp, _p(sel_out),
                                            _p(scores_out), _p(ws), ws.numel(), _stream(stream)), "hkv_select_pages")
+
+
+def hkv_page_scores(kbar_pages, Q, scores_out, ws, cand_range=None, stream=None):
+    """Page scores summed over the heads of Q / kbar_pages (one head group)."""
+    NP = kbar_pages.shape[0]
+    Lq, H, d = Q.shape
+    _check(load_library().hkv_page_scores(_p(kbar_pages), NP, _p(cand_range), _p(Q), Lq, H, d, _p(scores_out), _p(ws),
+                                          ws.numel(), _stream(stream)), "hkv_page_scores")
+
+
+def hkv_select_top(scores, Kp, sel_out, ws, cand_range=None, stream=None):
+    """Top-Kp pages of the (all-reduced) page scores, ascending."""
+    _check(load_library().hkv_select_top(_p(scores), scores.numel(), _p(cand_range), Kp, _p(sel_out), _p(ws),
+                                         ws.numel(), _stream(stream)), "hkv_select_top")
+
+
+def hkv_select_pages_policy(policy, kbar_pages, Q, Kp, sel_out, ws, scores_out=None, cand_range=None,
+                            rand_keys=None, stream=None):
+    """Page retrieval by policy: POLICY_SCORE (mean-key score), POLICY_RECENT, POLICY_RANDOM."""
+    NP = kbar_pages.shape[0]
+    Lq, H, d = Q.shape
+    _check(load_library().hkv_select_pages_policy(policy, _p(kbar_pages), NP, _p(cand_range), _p(Q), Lq, H, d, Kp,
+                                                  _p(rand_keys), _p(sel_out), _p(scores_out), _p(ws), ws.numel(),
+                                                  _stream(stream)), "hkv_select_pages_policy")
 
 
 def hkv_select_pages_noalloc(kbar_pages, Q, Kp, sel_out, scores_out=None, cand_range=None, status_out=None,

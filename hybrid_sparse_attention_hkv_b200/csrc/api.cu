@@ -79,7 +79,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 struct Layout {
   size_t status = 0, colpart = 0, q128 = 0, q64 = 0, kq64 = 0, kc128 = 0;
   size_t inter_idx = 0, inter_cnt = 0, intra_idx = 0, intra_cnt = 0;
-  size_t units = 0, n_units = 0, tile_done = 0, part_o = 0, part_ml = 0, lin_buf = 0, attn_end = 0;
+  size_t units = 0, n_units = 0, tile_done = 0, part_o = 0, part_ml = 0, part_lin = 0, attn_end = 0;
   int max_units = 0, max_slots = 0;
   size_t ekhi = 0, eklo = 0, fvhi = 0, fvlo = 0, projpart = 0, ekfv_hist = 0;
   size_t pages_end = 0;  // bytes needed by the page (HKV) calls
@@ -115,7 +115,7 @@ Layout make_layout(int H, int d, int Lq, long long Lc, int r) {
   L.tile_done = take((size_t)H * nQ128 * 4);
   L.part_o = take((size_t)L.max_slots * 128 * d * 4);
   L.part_ml = take((size_t)L.max_slots * 128 * 8);
-  L.lin_buf = take((size_t)Lq * H * d * 4);
+  L.part_lin = take((size_t)L.max_slots * 128 * d * 4);
   L.attn_end = off;
   const size_t hrd = (size_t)H * r * d;
   L.ekhi = take(hrd * 2);
@@ -374,6 +374,62 @@ hsa_status_t hkv_select_pages(const float* kbar_pages, int NP, const int32_t* ca
   return HSA_OK;
 }
 
+hsa_status_t hkv_page_scores(const float* kbar_pages, int NP, const int32_t* cand_range, const hsa_bf16* Q, int Lq,
+                             int H, int d, float* scores_out, void* ws, size_t ws_bytes, hsa_stream_t stream) {
+  const char* fn = __func__;
+  TRY(check_heads(fn, H, d));
+  if (NP < 1 || Lq < 1) return fail(HSA_ERR_INVALID_ARG, "%s: NP = %d, Lq = %d must be >= 1", fn, NP, Lq);
+  if ((size_t)H * d * 4 > 200 * 1024) return fail(HSA_ERR_UNSUPPORTED, "%s: H*d*4 bytes exceed shared memory", fn);
+  REQUIRE_PTR(kbar_pages);
+  REQUIRE_PTR(Q);
+  if (!scores_out) return fail(HSA_ERR_INVALID_ARG, "%s: scores_out is NULL", fn);
+  const Layout L = make_layout(H, d, 1, 0, 0);
+  const size_t need = 256 + align256((size_t)hsa::page_score_splits(Lq) * NP * 4);
+  TRY(check_ws(fn, ws, ws_bytes, need > L.pages_end ? need : L.pages_end));
+  float* part = at<float>(ws, 256);
+  HSA_LAUNCH("page_scores_partial", hsa::launch_page_scores_partial(Q, Lq, H * d, kbar_pages, NP, cand_range, part,
+                                                                    stream));
+  HSA_LAUNCH("page_scores_sum", hsa::launch_page_scores_sum(part, Lq, NP, cand_range, scores_out, stream));
+  return HSA_OK;
+}
+
+hsa_status_t hkv_select_top(const float* scores, int NP, const int32_t* cand_range, int Kp, int32_t* sel_out,
+                            void* ws, size_t ws_bytes, hsa_stream_t stream) {
+  const char* fn = __func__;
+  if (NP < 1) return fail(HSA_ERR_INVALID_ARG, "%s: NP = %d must be >= 1", fn, NP);
+  if (Kp < 1 || Kp > NP || Kp > 64) return fail(HSA_ERR_INVALID_ARG, "%s: Kp = %d must be in [1, min(NP, 64)]", fn, Kp);
+  REQUIRE_PTR(scores);
+  if (!sel_out) return fail(HSA_ERR_INVALID_ARG, "%s: sel_out is NULL", fn);
+  TRY(check_ws(fn, ws, ws_bytes, 256));
+  // the scores as one split of partial scores with "Lq" = 1: ranked as they are
+  HSA_LAUNCH("select_pages_final", hsa::launch_select_pages_final(scores, 1, NP, cand_range, Kp, sel_out, nullptr,
+                                                                  status_of(ws), stream));
+  return HSA_OK;
+}
+
+hsa_status_t hkv_select_pages_policy(int policy, const float* kbar_pages, int NP, const int32_t* cand_range,
+                                     const hsa_bf16* Q, int Lq, int H, int d, int Kp, const float* rand_keys,
+                                     int32_t* sel_out, float* scores_out, void* ws, size_t ws_bytes,
+                                     hsa_stream_t stream) {
+  const char* fn = __func__;
+  if (policy == hsa::kPolicyScore)
+    return hkv_select_pages(kbar_pages, NP, cand_range, Q, Lq, H, d, Kp, sel_out, scores_out, ws, ws_bytes, stream);
+  if (policy != hsa::kPolicyRecent && policy != hsa::kPolicyRandom)
+    return fail(HSA_ERR_INVALID_ARG, "%s: unknown policy %d", fn, policy);
+  if (NP < 1) return fail(HSA_ERR_INVALID_ARG, "%s: NP = %d must be >= 1", fn, NP);
+  if (Kp < 1 || Kp > NP || Kp > 64) return fail(HSA_ERR_INVALID_ARG, "%s: Kp = %d must be in [1, min(NP, 64)]", fn, Kp);
+  if (NP > (1 << 24)) return fail(HSA_ERR_UNSUPPORTED, "%s: NP = %d beyond 2^24 pages", fn, NP);
+  if (policy == hsa::kPolicyRandom) REQUIRE_PTR(rand_keys);
+  if (!sel_out) return fail(HSA_ERR_INVALID_ARG, "%s: sel_out is NULL", fn);
+  TRY(check_ws(fn, ws, ws_bytes, 256 + align256((size_t)NP * 4)));
+  float* part = at<float>(ws, 256);
+  HSA_LAUNCH("policy_keys", hsa::launch_policy_keys(policy, rand_keys, NP, part, stream));
+  // one split of keys, "Lq" = 1: the final pass ranks the keys as they are
+  HSA_LAUNCH("select_pages_final", hsa::launch_select_pages_final(part, 1, NP, cand_range, Kp, sel_out, scores_out,
+                                                                  status_of(ws), stream));
+  return HSA_OK;
+}
+
 hsa_status_t hkv_gather(const hsa_bf16* const* page_k, const hsa_bf16* const* page_v, int NP, const int32_t* sel,
                         int Kp, int P_tok, int H, int d, hsa_bf16* Kc, hsa_bf16* Vc, float* kbar128, void* ws,
                         size_t ws_bytes, hsa_stream_t stream) {
@@ -526,7 +582,6 @@ static hsa::AttnArgs attn_args(const hsa_config_t* cfg, const Layout& L, void* w
   a.status = status_of(ws);
   a.max_units = L.max_units;
   a.max_slots = L.max_slots;
-  a.lin_buf = at<float>(ws, L.lin_buf);
   return a;
 }
 
@@ -539,6 +594,7 @@ static hsa_status_t run_plan(const Layout& L, const hsa_selection_t& sel, void* 
   a.tile_done = at<int>(ws, L.tile_done);
   a.part_o = at<float>(ws, L.part_o);
   a.part_ml = at<float2>(ws, L.part_ml);
+  a.part_lin = at<float>(ws, L.part_lin);
   HSA_LAUNCH("attn_plan", hsa::launch_attn_plan(a, stream));
   return HSA_OK;
 }

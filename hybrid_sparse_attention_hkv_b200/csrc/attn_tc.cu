@@ -10,43 +10,36 @@
 //                 segment 0 only;
 //   cached tiles  one 128-row tile per kept inter block of the cached KV;
 //   chunk tiles   the union of the two 64-query halves' kept 64-row intra blocks,
-//                 each tagged with the halves that use it.
-// A segment takes the sparse tiles whose cumulative cost (2 per cached tile, 1 per
-// chunk tile) falls in its share of the list's cost.  A unit covering its whole
+//                 each tagged with the halves that use it; blocks with the same tag
+//                 are paired into 128-row tiles (two 64-row boxes in one slot), so
+//                 that a chunk block costs half a tile's fixed pipeline latency.
+// A segment takes the sparse tiles whose cumulative cost (2 per 128-row tile, 1 per
+// lone 64-row chunk tile) falls in its share of the list's cost.  A unit covering its whole
 // list writes the output; a segment of a split list writes its unnormalised O_s
-// with its running (max, sum) to a partial slot, and the CTA that finishes the
-// list's last segment merges the slots in segment order.
-//
-// Each query row is served by two softmax threads, one per half of every key tile
-// (its first and its second half of the columns).  Each half keeps its own running
-// max and sum and its own accumulator in TMEM (O_a, O_b); nothing is exchanged per
-// tile, and the two halves are combined only at the end:
-//   o = (2^m_a O_a + 2^m_b O_b) / (2^m_a l_a + 2^m_b l_b).
-// The linear tiles come first and use the same two accumulators; when they are
-// done the halves are combined, weighted by the gate and stashed in the workspace,
-// and the sparse tiles start the accumulators afresh.
-// 11 warps:
+// with its running (max, sum) to a partial slot (segment 0 adds the weighted
+// linear branch), and the CTA that finishes the list's last segment merges the
+// slots in segment order.
+// 7 warps:
 //   warp 0      TMA producer of the Q tile (once) and of each key tile's K part
 //               (K, or EK_hi + EK_lo) into a 3-slot ring of 128-byte-swizzled
 //               buffers (a slot frees when its S MMA ends);
-//   warp 10     TMA producer of the V parts (V, or FV_hi + FV_lo) into a 2-slot ring
-//               (a slot frees when its P.V MMAs end);
-//   warp 1      MMA issuer (one elected lane): S_j = Q K_j^T (+ Q EK_lo^T) into one
-//               of two TMEM S buffers, then, per half, O_x += P_x V_x with P_x read
-//               from TMEM (written over that half's S columns; for linear tiles
-//               P_hi FV_hi + P_lo FV_hi + P_hi FV_lo);
-//   warps 2-5   softmax of the first half of every tile's columns, one TMEM lane
-//               (= query row) per thread;
-//   warps 6-9   softmax of the second half (warp w + 4 serves the rows of warp w):
-//               exp2, row sums, P as packed bf16 back into TMEM; the running max is
-//               raised (and that half's O rescaled in TMEM) only when it grows by
-//               more than 2^8; finally the halves are combined, merged with the
-//               stashed linear branch, out = g o_s + (1 - g) o_l, and stored (each
-//               thread of a row stores half of its columns).
+//   warp 6      TMA producer of the V parts (V, or FV_hi + FV_lo) into a 2-slot
+//               ring (a slot frees when its P.V MMA ends);
+//   warp 1      MMA issuer (one elected lane): S_j = Q K_j^T (+ Q EK_lo^T) into one of two
+//               TMEM S buffers, then O += P_j V_j with P_j read from TMEM (written
+//               over S_j; for linear tiles P_hi FV_hi + P_lo FV_hi + P_hi FV_lo
+//               into a second accumulator O_l);
+//   warps 2-5   softmax, one TMEM lane (= query row) per thread, one running
+//               max / sum per branch: exp2, row sums, P as packed bf16 back into
+//               TMEM; the running max is raised (and that O rescaled in TMEM) only
+//               when it grows by more than 2^8; finally o_s = O_s / l_s,
+//               o_l = O_l / l_l, out = g o_s + (1 - g) o_l, stored.
 // The tensor core computes S_{j+1} while the softmax warps work on S_j.
-// Every wait is bounded (HSA_ERR_TIMEOUT in the workspace status on expiry); the
-// exchanges between the two halves of a row go through shared memory and mbarriers
-// (bounded waits), never through a named barrier that a timed-out warp would miss.
+// Every wait is bounded (HSA_ERR_TIMEOUT in the workspace status on expiry).  The
+// softmax warps' per-tile waits are per-lane (a warp-wide vote after each of them
+// cost 7% of the kernel's time); the MMA warp, which issues with elect.sync, and the
+// waits before the first and after the last tile, where the warps go on to
+// warp-collective TMEM access and teardown, take the warp's common answer.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -61,9 +54,7 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kTcThreads = 352;  // 11 warps
-constexpr int kWarpV = 10;       // V producer
-constexpr int kSoftThreads = 256;  // warps 2-9
+constexpr int kTcThreads = 224;  // 7 warps
 constexpr int kKStages = 3;      // K ring: a slot frees as soon as its S MMA completes
 constexpr int kVStages = 2;      // V ring: a slot frees when its P.V MMA completes
 constexpr int kRegionBytes = 128 * 128;  // one [128 rows x 64 bf16] swizzled region
@@ -72,10 +63,12 @@ struct TcMaps {
   CUtensorMap q, kc, vc, kq, vq, ekhi, eklo, fvhi, fvlo;
 };
 
-// Key-tile code: (first row << 4) | (type << 2) | half-mask.
+// Key-tile code: (first row << 4) | (type << 2) | half-mask; a pair of chunk blocks
+// ja < jb (64-row block ids < 8192): (ja << 17) | (jb << 4) | (type << 2) | half-mask.
 constexpr int kTileCached = 0;  // 128 rows of Kc / Vc
 constexpr int kTileChunk = 1;   // 64 rows of Kq / Vq
 constexpr int kTileLinear = 2;  // 64 rows of EK / FV (hi + lo)
+constexpr int kTilePair = 3;    // two 64-row blocks of Kq / Vq used by the same query halves
 
 template <int D>
 struct TcLayout {
@@ -89,7 +82,15 @@ __device__ __forceinline__ int tc_tile_code(long long start, int type, int mask)
 }
 __device__ __forceinline__ int tile_type(int code) { return (code >> 2) & 3; }
 __device__ __forceinline__ int tile_start(int code) { return code >> 4; }
-__device__ __forceinline__ int tile_rows(int code) { return tile_type(code) == kTileCached ? 128 : 64; }
+__device__ __forceinline__ int tile_rows(int code) {
+  const int t = tile_type(code);
+  return (t == kTileCached || t == kTilePair) ? 128 : 64;
+}
+__device__ __forceinline__ int pair_code(int ja, int jb, int mask) {
+  return (ja << 17) | (jb << 4) | (kTilePair << 2) | mask;
+}
+__device__ __forceinline__ int pair_first(int code) { return code >> 17; }
+__device__ __forceinline__ int pair_second(int code) { return (code >> 4) & 0x1FFF; }
 
 // 16 output values of row `grow`, head h, columns [16c, 16c + 16), fp32 or bf16.
 __device__ __forceinline__ void store_out16(const AttnArgs& a, int grow, int h, int D, int c, const float (&v)[16]) {
@@ -110,29 +111,29 @@ __device__ __forceinline__ void store_out16(const AttnArgs& a, int grow, int h, 
 }
 
 // ------------------------------------------------------------------ kernel
-// Online-softmax step of one query row over its half of one key tile: N raw scores
-// in sr[0..N) (N = 64 for a 128-row tile, 32 for a 64-row tile).  Updates the
-// running max m (raised only when it grows by more than 2^8, returning the factor
-// alpha for O), writes P = 2^(s*sl2 - m) as N/2 packed bf16 pairs at tS, and folds
-// the row sum into l.  MASKED: only the first `valid` keys exist.
+// Online-softmax step of one query row over one key tile of ROWS columns held in
+// sr[] (raw scores): update the running max m (raised only when it grows by more
+// than 2^8, returning the factor alpha for O), write P = 2^(s*sl2 - m) as packed
+// bf16 pairs over the first ROWS/2 columns of the S buffer, and fold the row sum
+// into l.  MASKED: only the first `valid` keys exist.
 __device__ __forceinline__ float fmax3f(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
 }
-template <int N, bool MASKED>
-__device__ __forceinline__ void softmax_half(const uint32_t (&sr)[64], int valid, float sl2, float& m, float& l,
+template <int ROWS, bool MASKED>
+__device__ __forceinline__ void softmax_tile(const uint32_t (&sr)[128], int valid, float sl2, float& m, float& l,
                                              float& alpha, bool& rescale, uint32_t tS) {
   float pm[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) pm[q] = -INFINITY;
   if (MASKED) {
 #pragma unroll
-    for (int k = 0; k < N; ++k)
+    for (int k = 0; k < ROWS; ++k)
       if (k < valid) pm[k & 7] = fmaxf(pm[k & 7], __uint_as_float(sr[k]));
   } else {
 #pragma unroll
-    for (int k = 0; k < N; k += 2) pm[(k >> 1) & 7] = fmax3f(pm[(k >> 1) & 7], __uint_as_float(sr[k]), __uint_as_float(sr[k + 1]));
+    for (int k = 0; k < ROWS; k += 2) pm[(k >> 1) & 7] = fmax3f(pm[(k >> 1) & 7], __uint_as_float(sr[k]), __uint_as_float(sr[k + 1]));
   }
   const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
   const float mn = mx * sl2;
@@ -148,7 +149,7 @@ __device__ __forceinline__ void softmax_half(const uint32_t (&sr)[64], int valid
 #pragma unroll
   for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int c = 0; c < N / 32; ++c) {
+  for (int c = 0; c < ROWS / 32; ++c) {
     uint32_t pk[16];
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
@@ -172,24 +173,23 @@ __device__ __forceinline__ void softmax_half(const uint32_t (&sr)[64], int valid
       acc[k & 3] = __fadd2_rn(acc[k & 3], make_float2(p0, p1));
       pk[k] = pack_bf16x2(p0, p1);
     }
-    tmem_st16(tS + c * 16, pk);  // P (bf16 pairs) over the first quarter of this half's S columns
+    tmem_st16(tS + c * 16, pk);  // P (bf16 pairs) over the first half of S
   }
   const float2 s01 = __fadd2_rn(acc[0], acc[1]), s23 = __fadd2_rn(acc[2], acc[3]);
   const float2 st = __fadd2_rn(s01, s23);
   l = l * alpha + (st.x + st.y);
 }
 
-// Linear-branch variant over this thread's 32 of a tile's 64 projected rows (no
-// masking): P is written as two bf16 parts, hi = bf16(p) over columns [0, 16) and
-// lo = bf16(p - hi) over [16, 32) of this half's S columns, so that P.FV keeps about
-// 16 significant bits.
-__device__ __forceinline__ void softmax_half_split(const uint32_t (&sr)[64], float sl2, float& m, float& l,
+// Linear-branch variant over 64 projected rows (no masking): P is written as two
+// bf16 parts, hi = bf16(p) over columns [0, 32) and lo = bf16(p - hi) over
+// [32, 64) of the S buffer, so that P.FV keeps about 16 significant bits.
+__device__ __forceinline__ void softmax_tile_split(const uint32_t (&sr)[64], float sl2, float& m, float& l,
                                                    float& alpha, bool& rescale, uint32_t tS) {
   float pm[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) pm[q] = -INFINITY;
 #pragma unroll
-  for (int k = 0; k < 32; ++k) pm[k & 7] = fmaxf(pm[k & 7], __uint_as_float(sr[k]));
+  for (int k = 0; k < 64; ++k) pm[k & 7] = fmaxf(pm[k & 7], __uint_as_float(sr[k]));
   const float mx = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])), fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7])));
   const float mn = mx * sl2;
   if (mn > m + 8.f) {
@@ -203,34 +203,27 @@ __device__ __forceinline__ void softmax_half_split(const uint32_t (&sr)[64], flo
   float2 acc[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
-  uint32_t hi[16], lo[16];
 #pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    const int i = 2 * k;
-    const float2 t = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), a2, b2);
-    const float p0 = ex2_approx(t.x), p1 = ex2_approx(t.y);
-    acc[k & 3] = __fadd2_rn(acc[k & 3], make_float2(p0, p1));
-    __nv_bfloat16 h0, l0, h1, l1;
-    split_bf16(p0, h0, l0);
-    split_bf16(p1, h1, l1);
-    hi[k] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
-    lo[k] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+  for (int c = 0; c < 2; ++c) {
+    uint32_t hi[16], lo[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const int i = c * 32 + 2 * k;
+      const float2 t = __ffma2_rn(make_float2(__uint_as_float(sr[i]), __uint_as_float(sr[i + 1])), a2, b2);
+      const float p0 = ex2_approx(t.x), p1 = ex2_approx(t.y);
+      acc[k & 3] = __fadd2_rn(acc[k & 3], make_float2(p0, p1));
+      __nv_bfloat16 h0, l0, h1, l1;
+      split_bf16(p0, h0, l0);
+      split_bf16(p1, h1, l1);
+      hi[k] = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+      lo[k] = (uint32_t)__bfloat16_as_ushort(l0) | ((uint32_t)__bfloat16_as_ushort(l1) << 16);
+    }
+    tmem_st16(tS + c * 16, hi);
+    tmem_st16(tS + 32 + c * 16, lo);
   }
-  tmem_st16(tS, hi);
-  tmem_st16(tS + 16, lo);
   const float2 s01 = __fadd2_rn(acc[0], acc[1]), s23 = __fadd2_rn(acc[2], acc[3]);
   const float2 st = __fadd2_rn(s01, s23);
   l = l * alpha + (st.x + st.y);
-}
-
-// Weights that combine the two halves of a row: w_x = 2^(m_x - M) with M the larger
-// max (0 for a half that saw no key); returns the combined sum 2^(m_a-M) l_a + ...
-__device__ __forceinline__ float combine_halves(float ma, float la, float mb, float lb, float& M, float& wa,
-                                                float& wb) {
-  M = fmaxf(ma, mb);
-  wa = (ma == -INFINITY) ? 0.f : exp2f(ma - M);
-  wb = (mb == -INFINITY) ? 0.f : exp2f(mb - M);
-  return wa * la + wb * lb;
 }
 
 // MMA issue by the whole MMA warp (one elected lane issues), every loop unrolled at
@@ -270,12 +263,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   unsigned char* sV = sK + kKStages * Lay::kKVBytes;          // [kVStages] V tiles
   int* tiles = reinterpret_cast<int*>(smem + Lay::kBytes);  // [r/64 + nKc + nKq]
   int* flags = tiles + (a.EKhi ? a.r / 64 : 0) + nKc + nKq; // [nKq]
+  int* scratch = flags + nKq;                                 // [nKq]
   __shared__ __align__(8) uint64_t bar_q, bar_k_full[kKStages], bar_k_empty[kKStages], bar_v_full[kVStages],
-      bar_v_empty[kVStages], bar_s_full[2], bar_p_full[2], bar_o_done, bar_final, bar_lin_done, bar_lin_free,
-      bar_ml_lin, bar_ml_fin;
-  __shared__ float2 s_ml_lin[2][128], s_ml_fin[2][128];  // (max, sum) of each half of each row
+      bar_v_empty[kVStages], bar_s_full[2], bar_p_full[2], bar_o_done, bar_final;
   __shared__ uint32_t s_tmem;
-  __shared__ int s_ntiles;
+  __shared__ int s_ntiles, s_n2;
+
   __shared__ int s_last;
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
@@ -312,14 +305,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bar_s_full[b], 1);
-      mbar_init(&bar_p_full[b], kSoftThreads);
+      mbar_init(&bar_p_full[b], 128);
     }
     mbar_init(&bar_o_done, 1);
     mbar_init(&bar_final, 1);
-    mbar_init(&bar_lin_done, 1);
-    mbar_init(&bar_lin_free, kSoftThreads);
-    mbar_init(&bar_ml_lin, kSoftThreads);
-    mbar_init(&bar_ml_fin, kSoftThreads);
     fence_barrier_init();
   }
 
@@ -358,26 +347,51 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
   __syncthreads();
   if (warp == 0) {
+    // chunk blocks by tag (both halves, half 0 only, half 1 only), ascending within a
+    // tag, paired; a tag's odd block out stays a 64-row tile at the end of the list.
+    // The partial last block (the largest id) is always the second of its pair.
     int base = n_lin + n_inter;
+    int single[3] = {-1, -1, -1};
     if (do_sparse) {
-      for (int b = 0; b < nKq; b += 32) {
-        const int j = b + lane;
-        const int f = j < nKq ? flags[j] : 0;
-        const unsigned bal = __ballot_sync(0xffffffffu, f != 0);
-        if (f) tiles[base + __popc(bal & ((1u << lane) - 1u))] = tc_tile_code((long long)j * 64, kTileChunk, f);
-        base += __popc(bal);
+      for (int c = 0; c < 3; ++c) {
+        const int tag = c == 0 ? 3 : c;
+        int cnt = 0;
+        for (int b = 0; b < nKq; b += 32) {
+          const int j = b + lane;
+          const bool in = j < nKq && flags[j] == tag;
+          const unsigned bal = __ballot_sync(0xffffffffu, in);
+          if (in) scratch[cnt + __popc(bal & ((1u << lane) - 1u))] = j;
+          cnt += __popc(bal);
+        }
+        __syncwarp();
+        for (int k = lane; k < cnt / 2; k += 32) tiles[base + k] = pair_code(scratch[2 * k], scratch[2 * k + 1], tag);
+        base += cnt / 2;
+        if (cnt & 1) single[c] = scratch[cnt - 1];
+        __syncwarp();
       }
     }
-    if (lane == 0) s_ntiles = base;
+    const int n2 = base - n_lin;  // 128-row sparse tiles: cached + pairs
+    for (int c = 0; c < 3; ++c) {
+      if (single[c] >= 0) {
+        if (lane == 0) tiles[base] = tc_tile_code((long long)single[c] * 64, kTileChunk, c == 0 ? 3 : c);
+        ++base;
+      }
+    }
+    if (lane == 0) {
+      s_ntiles = base;
+      s_n2 = n2;
+    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // this segment's share of the sparse tiles, by cost (a cached tile costs 2, a chunk tile 1)
-  const int n_chunk = s_ntiles - n_lin - n_inter;
-  const long long cost = 2LL * n_inter + n_chunk;
+  // this segment's share of the sparse tiles, by cost (a 128-row tile costs 2, a lone
+  // 64-row chunk tile 1; the 128-row tiles come first)
+  const int n2 = s_n2;
+  const int n1 = s_ntiles - n_lin - n2;
+  const long long cost = 2LL * n2 + n1;
   auto cut = [&](long long x) -> int {  // sparse tiles whose cumulative cost before them is < x
-    return x <= 2LL * n_inter ? (int)((x + 1) / 2) : n_inter + (int)(x - 2LL * n_inter);
+    return x <= 2LL * n2 ? (int)((x + 1) / 2) : n2 + (int)(x - 2LL * n2);
   };
   const int t0 = cut(cost * seg / nseg), t1 = cut(cost * (seg + 1) / nseg);
   const int T = n_lin + (t1 - t0);
@@ -385,7 +399,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   auto tile_at = [&](int j) -> int { return j < n_lin ? tiles[j] : tiles[j + t0]; };
   if (T == 0 && nseg == 1 && tid == 0) set_status(status, HSA_ERR_DEVICE);  // no key tile: empty selection
   const uint32_t tmem = s_tmem;
-  const uint32_t tOa = tmem + 256, tOb = tmem + 256 + D;  // accumulators of the two column halves
+  const uint32_t tOs = tmem + 256, tOl = tmem + 256 + D;
   constexpr int kHalfSlot = (D / 64) * 64 * 128;  // 64 rows x D bf16: hi part / lo part of a slot
 
   if (warp == 0) {
@@ -412,6 +426,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tma_load_2d(dK + c * 64 * 128, &maps.ekhi, &bar_k_full[s], c * 64, y);
             tma_load_2d(dK + kHalfSlot + c * 64 * 128, &maps.eklo, &bar_k_full[s], c * 64, y);
           }
+        } else if (type == kTilePair) {  // rows 0-63 and 64-127 of the slot from two blocks
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_2d(dK + c * 128 * 128, &maps.kq, &bar_k_full[s], h * D + c * 64, pair_first(code) * 64);
+            tma_load_2d(dK + c * 128 * 128 + 64 * 128, &maps.kq, &bar_k_full[s], h * D + c * 64,
+                        pair_second(code) * 64);
+          }
         } else {
           const CUtensorMap* mk = type == kTileChunk ? &maps.kq : &maps.kc;
 #pragma unroll
@@ -421,7 +442,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       __syncwarp();
     }
-  } else if (warp == kWarpV) {
+  } else if (warp == 6) {
     // ------------------------------------------------------------ V producer
     for (int j = 0; j < T; ++j) {
       const int s = j % kVStages;
@@ -438,6 +459,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int c = 0; c < D / 64; ++c) {
             tma_load_2d(dV + c * 64 * 128, &maps.fvhi, &bar_v_full[s], c * 64, y);
             tma_load_2d(dV + kHalfSlot + c * 64 * 128, &maps.fvlo, &bar_v_full[s], c * 64, y);
+          }
+        } else if (type == kTilePair) {
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_2d(dV + c * 128 * 128, &maps.vq, &bar_v_full[s], h * D + c * 64, pair_first(code) * 64);
+            tma_load_2d(dV + c * 128 * 128 + 64 * 128, &maps.vq, &bar_v_full[s], h * D + c * 64,
+                        pair_second(code) * 64);
           }
         } else {
           const CUtensorMap* mv = type == kTileChunk ? &maps.vq : &maps.vc;
@@ -478,9 +506,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (ok && T > 0) ok = issue_s(0);
     for (int j = 0; ok && j < T; ++j) {
       if (j + 1 < T && !issue_s(j + 1)) break;
-      // the first sparse P.V overwrites the accumulators: the linear branch must have
-      // been read out of them first
-      if (j == n_lin && n_lin > 0 && !mbar_wait_warp(&bar_lin_free, 0, status, wlim)) break;
       if (!mbar_wait_warp(&bar_p_full[j & 1], (j >> 1) & 1, status, wlim)) break;
       const int sv = j % kVStages;
       if (!mbar_wait_warp(&bar_v_full[sv], (j / kVStages) & 1, status, wlim)) break;
@@ -488,52 +513,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int code = tile_at(j);
       const uint32_t v_base = smem_u32(sV + sv * Lay::kKVBytes);
       const uint32_t tP = tmem + (j & 1) * 128;
-      const bool acc = !(j == 0 || j == n_lin);  // the first tile of each phase starts the accumulators
       if (tile_type(code) == kTileLinear) {
-        // per half x (projected rows 32x .. 32x + 31): O_x += P_hi FV_hi + P_lo FV_hi + P_hi FV_lo
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          const uint32_t tO = x ? tOb : tOa;
-          const uint64_t vhi = sdesc_sw128(v_base + x * 4096, 64 * 128, 1024);
-          const uint64_t vlo = sdesc_sw128(v_base + kHalfSlot + x * 4096, 64 * 128, 1024);
-          issue_pv<D, 32>(tO, tP + x * 32, vhi, acc);
-          issue_pv<D, 32>(tO, tP + x * 32 + 16, vhi, true);
-          issue_pv<D, 32>(tO, tP + x * 32, vlo, true);
-        }
-      } else if (tile_rows(code) == 128) {  // key rows 64x .. 64x + 63 of a cached tile
-#pragma unroll
-        for (int x = 0; x < 2; ++x)
-          issue_pv<D, 64>(x ? tOb : tOa, tP + x * 64, sdesc_sw128(v_base + x * 8192, 128 * 128, 1024), acc);
-      } else {  // key rows 32x .. 32x + 31 of a chunk tile
-#pragma unroll
-        for (int x = 0; x < 2; ++x)
-          issue_pv<D, 32>(x ? tOb : tOa, tP + x * 32, sdesc_sw128(v_base + x * 4096, 64 * 128, 1024), acc);
+        // O_l += P_hi FV_hi + P_lo FV_hi + P_hi FV_lo; first linear tile initialises O_l
+        const uint64_t vhi = sdesc_sw128(v_base, 64 * 128, 1024);
+        const uint64_t vlo = sdesc_sw128(v_base + kHalfSlot, 64 * 128, 1024);
+        issue_pv<D, 64>(tOl, tP, vhi, j > 0);
+        issue_pv<D, 64>(tOl, tP + 32, vhi, true);
+        issue_pv<D, 64>(tOl, tP, vlo, true);
+      } else if (tile_rows(code) == 128) {  // the first sparse tile initialises O_s
+        issue_pv<D, 128>(tOs, tP, sdesc_sw128(v_base, 128 * 128, 1024), j > n_lin);
+      } else {
+        issue_pv<D, 64>(tOs, tP, sdesc_sw128(v_base, 64 * 128, 1024), j > n_lin);
       }
       mma_commit_elect(&bar_v_empty[sv]);
       mma_commit_elect(&bar_o_done);
-      // one-shot barriers: every MMA of the linear phase / of the unit has completed
-      if (j == n_lin - 1) mma_commit_elect(&bar_lin_done);
+      // one-shot: completes once every MMA of the unit has completed
       if (j == T - 1) mma_commit_elect(&bar_final);
     }
-  } else {
-    // ------------------------------------------------------------ softmax + epilogue (warps 2-9)
-    const int hf = warp >= 6 ? 1 : 0;  // column half of every key tile
+  } else if (warp >= 2 && warp <= 5) {
+    // ------------------------------------------------------------ softmax + epilogue
     const int wq = warp & 3;
     const int row = 32 * wq + lane;
-    const int half_bit = wq < 2 ? 1 : 2;  // warp-uniform: rows 0..63 are query half 0
+    const int half_bit = wq < 2 ? 1 : 2;  // warp-uniform: rows 0..63 are half 0
     const uint32_t loff = (uint32_t)(32 * wq) << 16;
-    const uint32_t tO = (hf ? tOb : tOa) + loff;
     const float sl2 = a.scale * 1.4426950408889634f;
-    const int grow = q0 + row;
-    const bool valid_row = grow < a.Lq;
-    // out = g o_s + (1 - g) o_l with g = sigmoid(gate logit) when both branches run
-    const float g = (do_sparse && any_lin && a.gate_logit) ? 1.f / (1.f + expf(-a.gate_logit[h])) : 1.f;
-    float ms = -INFINITY, ls = 0.f;  // sparse branch running max / sum of this half
-    float ml = -INFINITY, ll = 0.f;  // linear branch running max / sum of this half
+    float ms = -INFINITY, ls = 0.f;  // sparse branch running max / sum
+    float ml = -INFINITY, ll = 0.f;  // linear branch running max / sum
     bool ok = true;
-    auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {  // bounded, warp-uniform answer
-      return mbar_wait_warp(bar, par, status, wlim);
-    };
     for (int j = 0; j < T; ++j) {
       const int b = j & 1;
       if (!mbar_wait(&bar_s_full[b], (j >> 1) & 1, status, wlim)) {
@@ -544,165 +550,128 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const int code = tile_at(j);
       const int type = tile_type(code);
       const int rows = tile_rows(code);
-      const long long nrows = type == kTileChunk ? (long long)a.Lq : a.Lc;
-      const int valid = type == kTileLinear ? 64 : (int)min((long long)rows, nrows - tile_start(code));
-      const int hcols = type == kTileCached ? 64 : 32;  // this thread's columns of the tile
-      const int my_valid = min(max(valid - hf * hcols, 0), hcols);
+      const long long nrows = (type == kTileChunk || type == kTilePair) ? (long long)a.Lq : a.Lc;
+      const int valid = type == kTileLinear ? 64
+                        : type == kTilePair ? 64 + (int)min(64LL, nrows - 64LL * pair_second(code))
+                                            : (int)min((long long)rows, nrows - tile_start(code));
       const bool used = (code & half_bit) != 0;
-      const uint32_t tS = tmem + b * 128 + loff + hf * hcols;
+      const uint32_t tS = tmem + b * 128 + loff;
       float alpha = 1.f;
       bool rescale = false;
-      uint32_t sr[64];
       if (type == kTileLinear) {  // tile-uniform
-        tmem_ld32_sync(tS, sr);
-        softmax_half_split(sr, sl2, ml, ll, alpha, rescale, tS);
+        uint32_t h64[64];
+        tmem_ld64_sync(tS, h64);
+        softmax_tile_split(h64, sl2, ml, ll, alpha, rescale, tS);
       } else if (used) {  // warp-uniform (a warp's 32 rows lie in one 64-row half)
-        if (hcols == 64) {
-          tmem_ld64_sync(tS, sr);
-          if (my_valid == 64) softmax_half<64, false>(sr, my_valid, sl2, ms, ls, alpha, rescale, tS);
-          else softmax_half<64, true>(sr, my_valid, sl2, ms, ls, alpha, rescale, tS);
+        uint32_t sr[128];
+        if (rows == 128) {
+          tmem_ld128_sync(tS, sr);
+          if (valid == 128) softmax_tile<128, false>(sr, valid, sl2, ms, ls, alpha, rescale, tS);
+          else softmax_tile<128, true>(sr, valid, sl2, ms, ls, alpha, rescale, tS);
         } else {
-          tmem_ld32_sync(tS, sr);
-          if (my_valid == 32) softmax_half<32, false>(sr, my_valid, sl2, ms, ls, alpha, rescale, tS);
-          else softmax_half<32, true>(sr, my_valid, sl2, ms, ls, alpha, rescale, tS);
+          uint32_t h64[64];
+          tmem_ld64_sync(tS, h64);
+#pragma unroll
+          for (int k = 0; k < 64; ++k) sr[k] = h64[k];
+          if (valid == 64) softmax_tile<64, false>(sr, valid, sl2, ms, ls, alpha, rescale, tS);
+          else softmax_tile<64, true>(sr, valid, sl2, ms, ls, alpha, rescale, tS);
         }
       } else {
         uint32_t zero[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) zero[k] = 0u;
-        tmem_st16(tS, zero);
-        if (hcols == 64) tmem_st16(tS + 16, zero);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (c * 32 < rows) tmem_st16(tS + c * 16, zero);
       }
       tmem_st_wait();
       if (__any_sync(0xffffffffu, rescale)) {
         // O holds the P.V products of tiles 0..j-1 once the last of them has completed
-        // (P.V of tile j cannot have started: it waits for this P; S_j was issued
-        // after P.V of tile j - 2, so the barrier is at most one phase behind).
+        // (P.V of tile j cannot have started: it waits for this P).  Without a rescale
+        // nothing here touches O, and the wait is skipped.
         if (j > 0 && !mbar_wait(&bar_o_done, (j - 1) & 1, status, wlim)) {
           ok = false;
           break;
         }
         tc_fence_after();
+        const uint32_t tO = type == kTileLinear ? tOl : tOs;
 #pragma unroll
         for (int c = 0; c < D / 16; ++c) {
           uint32_t r[16];
-          tmem_ld16_sync(tO + c * 16, r);
+          tmem_ld16_sync(tO + loff + c * 16, r);
 #pragma unroll
           for (int k = 0; k < 16; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
-          tmem_st16(tO + c * 16, r);
+          tmem_st16(tO + loff + c * 16, r);
         }
         tmem_st_wait();
       }
       tc_fence_before();
       mbar_arrive(&bar_p_full[b]);
-      if (j == n_lin - 1) {
-        // ---- end of the linear phase: combine the halves, weight by 1 - g (or 1),
-        // and stash (or, without a sparse branch, store) this thread's half of the
-        // row's columns; then hand the accumulators back to the sparse tiles
-        s_ml_lin[hf][row] = make_float2(ml, ll);
-        mbar_arrive(&bar_ml_lin);
-        if (!wait_all(&bar_ml_lin, 0) || !wait_all(&bar_lin_done, 0)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const float2 pa = s_ml_lin[0][row], pb = s_ml_lin[1][row];
-        float M, wa, wb;
-        const float L = combine_halves(pa.x, pa.y, pb.x, pb.y, M, wa, wb);
-        const float wl = (do_sparse ? 1.f - g : 1.f) / L;
-        wa *= wl;
-        wb *= wl;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          const int cc = hf * (D / 32) + c;  // 16-column group of the row
-          uint32_t ra[16], rb[16];
-          tmem_ld16_sync(tOa + loff + cc * 16, ra);
-          tmem_ld16_sync(tOb + loff + cc * 16, rb);
-          if (valid_row) {
-            float v[16];
-#pragma unroll
-            for (int k = 0; k < 16; ++k) v[k] = __uint_as_float(ra[k]) * wa + __uint_as_float(rb[k]) * wb;
-            if (do_sparse) {
-              float* dst = a.lin_buf + ((long long)grow * a.H + h) * D + cc * 16;
-#pragma unroll
-              for (int k = 0; k < 16; k += 4) *reinterpret_cast<float4*>(dst + k) = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
-            } else {
-              store_out16(a, grow, h, D, cc, v);
-            }
-          }
-        }
-        if (do_sparse) __threadfence();  // a merging CTA may read the stash
-        tc_fence_before();
-        mbar_arrive(&bar_lin_free);
-      }
     }
-    // ---- epilogue of the sparse branch: wait for every P.V product of the unit on
-    // the one-shot barrier the MMA warp commits after its last P.V (phase 0, so its
-    // parity names it unambiguously), combine the two halves of the row and store
-    if (ok && do_sparse && T > 0) ok = wait_all(&bar_final, 0);
-    if (ok && do_sparse) {
-      s_ml_fin[hf][row] = make_float2(ms, ls);
-      mbar_arrive(&bar_ml_fin);
-      ok = wait_all(&bar_ml_fin, 0);
-    }
-    if (ok && do_sparse) {
+    // Wait for every P.V product of the unit on the one-shot barrier the MMA warp
+    // commits after its last P.V (phase 0, so the parity names it unambiguously; the
+    // per-tile barrier can be up to two phases ahead or behind here).  The wait polls
+    // (bounded): the softmax warps have no other work left, and sleeping waits here
+    // cost 1 % of the kernel's time.
+    auto wait_poll = [&](uint64_t* bar, uint32_t par) -> bool {
+      bool r = false;
+      for (uint32_t i = 0; i < kSpinLimit && !r; ++i) r = mbar_try_wait(bar, par);
+      if (!r) set_status(status, HSA_ERR_TIMEOUT);
+      return __all_sync(0xffffffffu, r);
+    };
+    if (ok && (T == 0 || wait_poll(&bar_final, 0))) {
       tc_fence_after();
-      const float2 pa = s_ml_fin[0][row], pb = s_ml_fin[1][row];
-      float M, wa, wb;
-      const float L = combine_halves(pa.x, pa.y, pb.x, pb.y, M, wa, wb);
-      const bool had_sparse = T > n_lin;
+      const int grow = q0 + row;
+      const bool valid_row = grow < a.Lq;
+      // out = g o_s + (1 - g) o_l with g = sigmoid(gate logit) when both branches run
+      const float g = (do_sparse && any_lin && a.gate_logit) ? 1.f / (1.f + expf(-a.gate_logit[h])) : 1.f;
+      const float wl = do_lin ? (do_sparse ? 1.f - g : 1.f) / ll : 0.f;
       if (nseg == 1) {
-        if (valid_row && !(L > 0.f)) set_status(status, HSA_ERR_DEVICE);
-        const float ws = L > 0.f ? g / L : 0.f;
+        if (do_sparse && valid_row && !(ls > 0.f)) set_status(status, HSA_ERR_DEVICE);
+        const float ws = (do_sparse && ls > 0.f) ? g / ls : 0.f;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          const int cc = hf * (D / 32) + c;
-          uint32_t ra[16], rb[16];
-          tmem_ld16_sync(tOa + loff + cc * 16, ra);
-          tmem_ld16_sync(tOb + loff + cc * 16, rb);
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t rs[16], rl[16];
+          if (do_sparse) tmem_ld16_sync(tOs + loff + c * 16, rs);
+          if (do_lin) tmem_ld16_sync(tOl + loff + c * 16, rl);
           if (valid_row) {
             float v[16];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) v[k] = (__uint_as_float(ra[k]) * wa + __uint_as_float(rb[k]) * wb) * ws;
-            if (do_lin) {
-              const float* src = a.lin_buf + ((long long)grow * a.H + h) * D + cc * 16;
-#pragma unroll
-              for (int k = 0; k < 16; k += 4) {
-                const float4 l4 = *reinterpret_cast<const float4*>(src + k);
-                v[k] += l4.x; v[k + 1] += l4.y; v[k + 2] += l4.z; v[k + 3] += l4.w;
-              }
+            for (int k = 0; k < 16; ++k) {
+              const float vs = do_sparse ? __uint_as_float(rs[k]) * ws : 0.f;
+              const float vl = do_lin ? __uint_as_float(rl[k]) * wl : 0.f;
+              v[k] = vs + vl;
             }
-            store_out16(a, grow, h, D, cc, v);
+            store_out16(a, grow, h, D, c, v);
           }
         }
       } else {
-        // one segment of a split list: the combined unnormalised O_s (relative to M)
-        // and (M, L); the linear branch, if any, is in the stash
+        // one segment of a split list: unnormalised O_s and (max, sum); segment 0
+        // also leaves the weighted linear branch at the list's first slot
         const int slot = slot0 + seg;
         float* po = a.part_o + ((long long)slot * 128 + row) * D;
+        float* pl = a.part_lin + ((long long)slot0 * 128 + row) * D;
+        const bool had_sparse = T > n_lin;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          const int cc = hf * (D / 32) + c;
-          uint32_t ra[16], rb[16];
-          if (had_sparse) {
-            tmem_ld16_sync(tOa + loff + cc * 16, ra);
-            tmem_ld16_sync(tOb + loff + cc * 16, rb);
-          }
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t rs[16], rl[16];
+          if (had_sparse) tmem_ld16_sync(tOs + loff + c * 16, rs);
+          if (do_lin) tmem_ld16_sync(tOl + loff + c * 16, rl);
           if (valid_row) {
 #pragma unroll
             for (int k = 0; k < 16; k += 4) {
-              float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
-              if (had_sparse)
-                o4 = make_float4(__uint_as_float(ra[k]) * wa + __uint_as_float(rb[k]) * wb,
-                                 __uint_as_float(ra[k + 1]) * wa + __uint_as_float(rb[k + 1]) * wb,
-                                 __uint_as_float(ra[k + 2]) * wa + __uint_as_float(rb[k + 2]) * wb,
-                                 __uint_as_float(ra[k + 3]) * wa + __uint_as_float(rb[k + 3]) * wb);
-              *reinterpret_cast<float4*>(po + cc * 16 + k) = o4;
+              *reinterpret_cast<float4*>(po + c * 16 + k) =
+                  had_sparse ? make_float4(__uint_as_float(rs[k]), __uint_as_float(rs[k + 1]),
+                                           __uint_as_float(rs[k + 2]), __uint_as_float(rs[k + 3]))
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+              if (do_lin)
+                *reinterpret_cast<float4*>(pl + c * 16 + k) =
+                    make_float4(__uint_as_float(rl[k]) * wl, __uint_as_float(rl[k + 1]) * wl,
+                                __uint_as_float(rl[k + 2]) * wl, __uint_as_float(rl[k + 3]) * wl);
             }
           }
         }
-        if (valid_row && hf == 0)
-          a.part_ml[(long long)slot * 128 + row] = make_float2(had_sparse && L > 0.f ? M : -INFINITY, L);
+        if (valid_row) a.part_ml[(long long)slot * 128 + row] = make_float2(had_sparse && ls > 0.f ? ms : -INFINITY, ls);
         __threadfence();
       }
     }
@@ -732,7 +701,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (!(L > 0.f)) set_status(status, HSA_ERR_DEVICE);
         const float g = (any_lin && a.gate_logit) ? 1.f / (1.f + expf(-a.gate_logit[h])) : 1.f;
         const float ws = L > 0.f ? g / L : 0.f;
-        const float* pl = a.lin_buf + ((long long)grow * a.H + h) * D;
+        const float* pl = a.part_lin + ((long long)slot0 * 128 + row) * D;
 #pragma unroll 1
         for (int c = 0; c < D / 16; ++c) {
           float v[16];
@@ -814,7 +783,7 @@ cudaError_t launch_tc(const AttnArgs& a, cudaStream_t s) {
   if ((e = make_map(&maps.fvhi, lin ? a.FVhi : a.Vq, lin ? pr : a.Lq, lin ? D : HD, 64)) != cudaSuccess) return e;
   if ((e = make_map(&maps.fvlo, lin ? a.FVlo : a.Vq, lin ? pr : a.Lq, lin ? D : HD, 64)) != cudaSuccess) return e;
   const int n_lin = lin ? a.r / 64 : 0;
-  const size_t smem = 1024 + TcLayout<D>::kBytes + (size_t)(n_lin + nKc + 2 * nKq) * 4;
+  const size_t smem = 1024 + TcLayout<D>::kBytes + (size_t)(n_lin + nKc + 3 * nKq) * 4;
   if (smem > 232448) return cudaErrorInvalidConfiguration;
   e = cudaFuncSetAttribute(sparse_attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -232,6 +232,28 @@ __global__ void __launch_bounds__(kFinalThreads) select_pages_final_kernel(
   }
 }
 
+// s_p = (sum over the splits of part[q][p]) / Lq for the candidates, -inf elsewhere
+// (the page scores of this call's heads, before any ranking).
+__global__ void page_scores_sum_kernel(const float* __restrict__ part, int splits, long long Lq, int NP,
+                                       const int32_t* __restrict__ cand_range, float* __restrict__ scores) {
+  const int p = blockIdx.x * blockDim.x + threadIdx.x;
+  if (p >= NP) return;
+  int first = 0, end = NP;
+  if (cand_range) {
+    first = cand_range[0];
+    end = cand_range[1];
+  }
+  float s = 0.f;
+  for (int q = 0; q < splits; ++q) s += part[(long long)q * NP + p];
+  scores[p] = (p >= first && p < end) ? s / (float)Lq : -INFINITY;
+}
+
+cudaError_t launch_page_scores_sum(const float* part, long long Lq, int NP, const int32_t* cand_range, float* scores,
+                                   cudaStream_t s) {
+  page_scores_sum_kernel<<<(NP + 255) / 256, 256, 0, s>>>(part, page_score_splits(Lq), Lq, NP, cand_range, scores);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_page_scores_partial(const uint16_t* Q, long long Lq, int C, const float* kbar_pages, int NP,
                                        const int32_t* cand_range, float* part, cudaStream_t s) {
   const int splits = page_score_splits(Lq);
@@ -256,6 +278,23 @@ cudaError_t launch_select_pages_final(const float* part, long long Lq, int NP, c
   }
   select_pages_final_kernel<<<1, kFinalThreads, smem, s>>>(part, page_score_splits(Lq), Lq, NP, cand_range, Kp,
                                                            sel_out, scores_out, status);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ retrieval policies
+// The retrieval ablations of the method's evaluation rank the candidate pages by
+// something other than the mean-key score: by recency (the page id: the most recent
+// pages) or by caller-drawn random keys (a uniform random subset).  One split of
+// "partial scores" holds those keys; select_pages_final then ranks them exactly as
+// it ranks page scores (ties -> lower page id) and writes the top Kp ascending.
+__global__ void policy_keys_kernel(int policy, const float* __restrict__ rand_keys, int NP, float* __restrict__ part) {
+  const int p = blockIdx.x * blockDim.x + threadIdx.x;
+  if (p >= NP) return;
+  part[p] = policy == kPolicyRecent ? (float)p : rand_keys[p];
+}
+
+cudaError_t launch_policy_keys(int policy, const float* rand_keys, int NP, float* part, cudaStream_t s) {
+  policy_keys_kernel<<<(NP + 255) / 256, 256, 0, s>>>(policy, rand_keys, NP, part);
   return cudaGetLastError();
 }
 

@@ -25,8 +25,16 @@ cudaError_t launch_page_summary_final(const float* part, long long n, int C, flo
 int page_score_splits(long long Lq);  // row splits of pass 1 (<= kColMaxSplits)
 cudaError_t launch_page_scores_partial(const uint16_t* Q, long long Lq, int C, const float* kbar_pages, int NP,
                                        const int32_t* cand_range, float* part, cudaStream_t s);
+cudaError_t launch_page_scores_sum(const float* part, long long Lq, int NP, const int32_t* cand_range, float* scores,
+                                   cudaStream_t s);
 cudaError_t launch_select_pages_final(const float* part, long long Lq, int NP, const int32_t* cand_range, int Kp,
                                       int32_t* sel_out, float* scores_out, int* status, cudaStream_t s);
+// Retrieval policies other than the mean-key score (hkv_select_pages_policy).
+constexpr int kPolicyScore = 0;
+constexpr int kPolicyRecent = 1;
+constexpr int kPolicyRandom = 2;
+// part[p] = the policy's ranking key of page p (its id, or rand_keys[p]); one split.
+cudaError_t launch_policy_keys(int policy, const float* rand_keys, int NP, float* part, cudaStream_t s);
 cudaError_t launch_select_prompt(const float* e_cur, const float* e_seg, int n_seg, int dim,
                                  const int32_t* seg_begin, int32_t* seg_out, int32_t* cand_range_out,
                                  cudaStream_t s);
@@ -107,7 +115,7 @@ struct AttnArgs {
   int* tile_done;    // [H * nQ128] segments finished (zeroed by the plan)
   float* part_o;     // [max_slots][128][d] unnormalised O_s of a segment
   float2* part_ml;   // [max_slots][128] running max (log2 units) and sum of a segment
-  float* lin_buf;    // [Lq][H][d] the linear branch weighted by 1 - g, stashed between the two phases
+  float* part_lin;   // [max_slots][128][d] weighted linear branch of a split list (at its first slot)
 };
 // Sparse and/or linear branch with the gated merge, on tcgen05 / TMEM / TMA.
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s);

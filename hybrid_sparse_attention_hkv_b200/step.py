@@ -53,6 +53,11 @@ class HkvHsaStep:
         for p in range(self.NP):
             hkv_page_summary(pages_k[p], self.kbar_pages[p], self.ws)
 
+    def _retrieve(self, Q, cand):
+        """Page-level retrieval into self.sel (self.scores: the page scores)."""
+        hkv_select_pages(self.kbar_pages, Q, self.Kp, self.sel, self.ws, self.scores, cand)
+        return self.sel
+
     def __call__(self, Q, Kq, Vq, tau, gate_logit, E, F, e_cur=None, e_seg=None, seg_begin=None,
                  ef_head_stride=0, out=None):
         """One step on the current stream; the result goes to `out` (same shape and
@@ -62,7 +67,7 @@ class HkvHsaStep:
         if e_cur is not None:
             hkv_select_prompt(e_cur, e_seg, seg_begin, self.seg, self.cand_range)
             cand = self.cand_range
-        hkv_select_pages(self.kbar_pages, Q, self.Kp, self.sel, self.ws, self.scores, cand)
+        self._retrieve(Q, cand)
         if self.store is not None:
             self.store.fetch(self.sel, self.ws)
         hkv_gather(self.page_k_ptrs, self.page_v_ptrs, self.sel, self.Kp, self.P_tok, self.H, self.d,
@@ -79,7 +84,7 @@ class HkvHsaStep:
         if e_cur is not None:
             hkv_select_prompt(e_cur, e_seg, seg_begin, self.seg, self.cand_range)
             cand = self.cand_range
-        hkv_select_pages(self.kbar_pages, Q, self.Kp, self.sel, self.ws, self.scores, cand)
+        self._retrieve(Q, cand)
         if self.store is not None:
             self.store.fetch(self.sel, self.ws)
         hkv_gather(self.page_k_ptrs, self.page_v_ptrs, self.sel, self.Kp, self.P_tok, self.H, self.d,

@@ -160,6 +160,44 @@ hsa_status_t hkv_select_pages(const float* kbar_pages, int NP, const int32_t* ca
                               int32_t* sel_out, float* scores_out,
                               void* ws, size_t ws_bytes, hsa_stream_t stream);
 
+/* Page-level retrieval in two calls, for a step whose heads are spread over
+ * several GPUs (the page score is a sum over heads, the only quantity of the step
+ * that mixes heads):
+ *   hkv_page_scores  scores_out[p] = sum over the heads of this call of
+ *                    qbar[h] . kbar_pages[p, h, :] (as hkv_select_pages), -inf
+ *                    outside cand_range; Q, kbar_pages hold these heads only;
+ *   (the caller adds the scores of all head groups: an all-reduce)
+ *   hkv_select_top   the Kp largest of scores[NP] within cand_range (ties -> lower
+ *                    page id), ascending, as hkv_select_pages ranks them.
+ * With one head group the two calls select exactly what hkv_select_pages
+ * selects.  Both use the workspace. */
+hsa_status_t hkv_page_scores(const float* kbar_pages, int NP, const int32_t* cand_range, const hsa_bf16* Q, int Lq,
+                             int H, int d, float* scores_out, void* ws, size_t ws_bytes, hsa_stream_t stream);
+hsa_status_t hkv_select_top(const float* scores, int NP, const int32_t* cand_range, int Kp, int32_t* sel_out,
+                            void* ws, size_t ws_bytes, hsa_stream_t stream);
+
+/* Retrieval policies of the method's retrieval ablations ([NEWS] HKV paragraph,
+ * Table 6: page-only, prompt-only, recent-page and random-page retrieval under the
+ * same budget of Kp pages; Table 5: the sliding-window cache):
+ *   HKV_POLICY_SCORE   the mean-key score of hkv_select_pages (page-only retrieval
+ *                      with cand_range NULL, two-stage with the prompt stage's range)
+ *   HKV_POLICY_RECENT  the Kp most recent candidates (largest page ids): over all
+ *                      pages the sliding window over the history, within the prompt
+ *                      stage's range prompt-only retrieval
+ *   HKV_POLICY_RANDOM  the Kp candidates with the largest rand_keys[p] (device fp32
+ *                      [NP], drawn by the caller, e.g. uniform): a uniform random
+ *                      subset; ties -> lower page id
+ * Output as hkv_select_pages: sel_out[0..Kp) ascending; scores_out (optional) gets
+ * each candidate's ranking key (score, page id or random key), -inf outside the
+ * range.  Q is read only by HKV_POLICY_SCORE.  Uses the workspace. */
+#define HKV_POLICY_SCORE 0
+#define HKV_POLICY_RECENT 1
+#define HKV_POLICY_RANDOM 2
+hsa_status_t hkv_select_pages_policy(int policy, const float* kbar_pages, int NP, const int32_t* cand_range,
+                                     const hsa_bf16* Q, int Lq, int H, int d, int Kp, const float* rand_keys,
+                                     int32_t* sel_out, float* scores_out, void* ws, size_t ws_bytes,
+                                     hsa_stream_t stream);
+
 /* Active-cache assembly ([NEWS] HKV and kernel paragraphs: KV-cache
  * reorganisation into contiguous memory): for i < Kp,
  *   Kc[i*P_tok + t] = page_k[sel[i]][t],  Vc[i*P_tok + t] = page_v[sel[i]][t]

@@ -50,7 +50,7 @@ from dataclasses import dataclass
 import numpy as np
 
 __all__ = [
-    "widen", "prompt_top1", "page_summary", "pooled_query", "page_scores", "select_pages",
+    "widen", "prompt_top1", "page_summary", "pooled_query", "page_scores", "select_pages", "select_pages_policy",
     "gather_pages", "block_means", "block_probs", "keep_blocks", "Selection", "block_select",
     "sparse_attention", "linear_projection", "linear_attention", "gate", "gated_merge",
     "hsa_step", "hkv_hsa_step",
@@ -112,6 +112,28 @@ def select_pages(kbar_pages, Q, Kp, cand=None, dtype=np.float32):
         raise ValueError("need 1 <= Kp <= number of candidates")
     ranked = sorted(cand, key=lambda p: (-s[p], p))
     return np.array(sorted(ranked[:Kp]), dtype=np.int32), s
+
+
+def select_pages_policy(policy, kbar_pages, Q, Kp, cand=None, rand_keys=None, dtype=np.float32):
+    """The retrieval ablations ([NEWS] HKV paragraph, Table 6: page-only, prompt-only,
+    recent-page and random-page retrieval under one budget of Kp pages; Table 5: the
+    sliding window).  "score": the mean-key score (select_pages); "recent": the Kp
+    candidates with the largest page ids (the most recent pages); "random": the Kp
+    candidates with the largest caller-drawn keys rand_keys[p], ties -> lower page id.
+    Returns the kept page ids ascending."""
+    if policy == "score":
+        return select_pages(kbar_pages, Q, Kp, cand, dtype)[0]
+    NP = np.asarray(kbar_pages).shape[0]
+    cand = list(range(NP)) if cand is None else [int(c) for c in cand]
+    if not 1 <= Kp <= len(cand):
+        raise ValueError("need 1 <= Kp <= number of candidates")
+    if policy == "recent":
+        return np.array(sorted(cand)[-Kp:], dtype=np.int32)
+    if policy == "random":
+        keys = np.asarray(rand_keys, dtype=np.float64)
+        ranked = sorted(cand, key=lambda p: (-keys[p], p))
+        return np.array(sorted(ranked[:Kp]), dtype=np.int32)
+    raise ValueError(f"unknown policy {policy!r}")
 
 
 def gather_pages(pages, sel) -> np.ndarray:

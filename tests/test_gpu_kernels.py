@@ -435,3 +435,81 @@ def test_multi_step_reuse(shape):
         assert hsa.hsa_status_read(st.ws) == 0
     finally:
         ds.close()
+
+
+# ----------------------------------------------------------------- retrieval policies
+
+def test_retrieval_policies_match_the_oracle():
+    """Page-only, prompt-only (recent pages of a candidate range), recent-page (sliding
+    window) and random-page retrieval: the GPU's page ids equal the oracle's exactly."""
+    H, d, Lq, NP, Kp = 4, 128, 520, 16, 4
+    kbar = torch.from_numpy(synth.normal_f32((NP, H, d), 71, 1, sigma=0.5)).cuda()
+    Qb = synth.normal_bf16((Lq, H, d), 71, 2)
+    Q = to_dev(Qb)
+    keys = synth.normal_f32((NP,), 71, 3)
+    keys[5] = keys[9]  # a tie: the lower page id ranks first
+    cfg = make_config(H, d, Lq, 0, 64)
+    ws = hsa.workspace(cfg)
+    kb = kbar.cpu().numpy()
+    for cand in (None, (3, 11)):
+        rng_t = None if cand is None else torch.tensor(cand, dtype=torch.int32, device="cuda")
+        cl = None if cand is None else range(*cand)
+        for pol, name in ((hsa.POLICY_SCORE, "score"), (hsa.POLICY_RECENT, "recent"), (hsa.POLICY_RANDOM, "random")):
+            sel = torch.full((Kp,), -7, dtype=torch.int32, device="cuda")
+            sc = torch.zeros(NP, dtype=torch.float32, device="cuda")
+            hsa.hkv_select_pages_policy(pol, kbar, Q, Kp, sel, ws, sc, rng_t, torch.from_numpy(keys).cuda())
+            torch.cuda.synchronize()
+            want = oracle.select_pages_policy(name, kb, Qb, Kp, cand=cl, rand_keys=keys)
+            if name == "score":
+                _, scores = oracle.select_pages(kb, Qb, Kp, cl)
+                check_pages(sel.cpu().numpy(), want, scores, Kp)
+            else:
+                assert sel.cpu().tolist() == want.tolist(), (name, cand)
+    assert hsa.hsa_status_read(ws) == 0
+
+
+# ----------------------------------------------------------------- head-sharded step
+
+def test_head_groups_emulated_on_one_gpu():
+    """The step of two head groups, one after the other on one GPU (no group waits for
+    another): the partial page scores of the groups, added, select the pages the
+    unsharded retrieval selects; each group's output equals the unsharded output of
+    its heads."""
+    from hybrid_sparse_attention_hkv_b200.sharded import head_range
+    from hybrid_sparse_attention_hkv_b200.step import HkvHsaStep, page_pointers
+    shape = SMALL[2]
+    ds = DeviceStep(shape, 81)
+    x, st = ds.x, ds.step
+    H, Kp, NP = shape.H, shape.Kp, shape.NP
+    full_out = ds.run().clone()
+    torch.cuda.synchronize()
+    total = torch.zeros(NP, dtype=torch.float32, device="cuda")
+    groups = [head_range(H, r, 2) for r in range(2)]
+    steps = []
+    for h0, h1 in groups:
+        pk = to_dev(np.ascontiguousarray(x.pages_k[:, :, h0:h1]))
+        pv = to_dev(np.ascontiguousarray(x.pages_v[:, :, h0:h1]))
+        g = HkvHsaStep(h1 - h0, shape.d, shape.Lq, shape.P_tok, NP, Kp, shape.r, page_pointers(pk),
+                       page_pointers(pv))
+        g.seal_pages(pk)
+        Qg = to_dev(np.ascontiguousarray(x.Q[:, h0:h1]))
+        hsa.hkv_page_scores(g.kbar_pages, Qg, g.scores, g.ws)
+        total += g.scores
+        steps.append((g, pk, pv, Qg))
+    sel = torch.zeros(Kp, dtype=torch.int32, device="cuda")
+    hsa.hkv_select_top(total, Kp, sel, steps[0][0].ws)
+    torch.cuda.synchronize()
+    check_pages(sel.cpu().numpy(), st.sel.cpu().numpy(), st.scores.cpu().numpy(), Kp)
+    assert sel.cpu().tolist() == st.sel.cpu().tolist()
+    for (h0, h1), (g, pk, pv, Qg) in zip(groups, steps):
+        sl = slice(h0, h1)
+        g.sel.copy_(sel)
+        hsa.hkv_gather(g.page_k_ptrs, g.page_v_ptrs, g.sel, Kp, shape.P_tok, h1 - h0, shape.d, g.Kc, g.Vc, g.ws,
+                       g.kbar128)
+        hsa.hsa_forward(g.cfg, Qg, g.Kc, g.Vc, to_dev(np.ascontiguousarray(x.Kq[:, sl])),
+                        to_dev(np.ascontiguousarray(x.Vq[:, sl])), ds.tau[sl].contiguous(), ds.z[sl].contiguous(),
+                        ds.E, ds.F, g.out, g.ws, g.kbar128, g.selection)
+        torch.cuda.synchronize()
+        assert torch.equal(g.selection.inter_cnt, st.selection.inter_cnt[sl])
+        assert torch.equal(g.selection.intra_cnt, st.selection.intra_cnt[sl])
+        assert float((g.out - full_out[:, sl]).abs().max()) <= 1e-4

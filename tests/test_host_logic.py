@@ -106,3 +106,62 @@ def test_reference_arm_two_ranks_prints_one_line():
     res = json.loads(lines[0])
     assert res["impl"] == "reference" and res["unit"] == "query-tokens/s" and res["value"] > 0
     assert res["cpu_baseline"]["kind"] == "oracle" and res["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _sharded_worker(rank, world, port, q):
+    """A head-sharded retrieval over gloo: each rank's partial page scores are the
+    oracle's scores of its heads; the plumbing sums them over the ranks and ranks."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import oracle
+    import synth
+    from hybrid_sparse_attention_hkv_b200.sharded import head_range, sharded_retrieval
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    H, d, Lq, NP, Kp = 5, 16, 96, 12, 3
+    kbar = synth.normal_f32((NP, H, d), 5, 1, sigma=0.5).astype(np.float64)
+    Q = synth.normal_bf16((Lq, H, d), 5, 2, offset=synth.normal_f32((H, d), 5, 3))
+    h0, h1 = head_range(H, rank, world)
+    qbar = oracle.pooled_query(Q[:, h0:h1])
+
+    def partial():
+        return torch.from_numpy(oracle.page_scores(kbar[:, h0:h1], qbar).copy())
+
+    def select(s):
+        s = s.numpy()
+        return sorted(sorted(range(NP), key=lambda p: (-s[p], p))[:Kp])
+
+    sel = sharded_retrieval(partial, lambda t: dist.all_reduce(t, op=dist.ReduceOp.SUM), select)
+    full, _ = oracle.select_pages(kbar, Q, Kp, dtype=np.float64)
+    q.put((rank, (h0, h1), sel, full.tolist()))
+    dist.destroy_process_group()
+
+
+def test_head_sharded_retrieval_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = free_port()
+    procs = [ctx.Process(target=_sharded_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    (r0, hr0, s0, full0), (r1, hr1, s1, full1) = out
+    assert hr0 == (0, 3) and hr1 == (3, 5)  # 5 heads over 2 ranks
+    assert s0 == s1 == full0 == full1  # every rank selects the unsharded pages
+
+
+def test_head_ranges_cover_every_head_once():
+    from hybrid_sparse_attention_hkv_b200.sharded import head_range
+    for H in (1, 2, 5, 12, 40):
+        for world in (1, 2, 3, 4, 8):
+            if world > H:
+                continue
+            r = [head_range(H, k, world) for k in range(world)]
+            assert r[0][0] == 0 and r[-1][1] == H
+            assert all(a[1] == b[0] for a, b in zip(r, r[1:]))
+            assert max(b - a for a, b in r) - min(b - a for a, b in r) <= 1

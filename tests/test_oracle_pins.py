@@ -474,3 +474,23 @@ def test_block_select_golden_rejects_plausible_mistakes(golden_dir):
     swapped[:, 1] = Kc[:, 0]
     assert [r.tolist() for r in oracle.block_select(Q, swapped, Kq, tau, scale=sc, dtype=np.float64).inter[1]] \
         != want_inter[1]
+
+
+def test_retrieval_policies_closed_forms():
+    """Recent pages are the last Kp candidates; random pages are the Kp largest keys
+    (ties -> lower page id), checked against a plain stable sort; 'score' is select_pages."""
+    rng = np.random.default_rng(11)
+    kb = rng.normal(size=(12, 2, 8))
+    Q = bf16(rng.normal(size=(16, 2, 8)))
+    assert oracle.select_pages_policy("recent", kb, Q, 3).tolist() == [9, 10, 11]
+    assert oracle.select_pages_policy("recent", kb, Q, 2, cand=range(3, 7)).tolist() == [5, 6]
+    keys = np.array([0.5, 0.9, 0.1, 0.9, 0.3, 0.7, 0.2, 0.0, 0.8, 0.6, 0.4, 0.95])
+    # ranked: 11 (.95), 1 and 3 tie at .9 (1 first), 8 (.8) ...
+    assert oracle.select_pages_policy("random", kb, Q, 3, rand_keys=keys).tolist() == [1, 3, 11]
+    assert oracle.select_pages_policy("random", kb, Q, 2, cand=[0, 2, 4, 6], rand_keys=keys).tolist() == [0, 4]
+    for _ in range(50):
+        k = rng.integers(0, 5, size=12).astype(float)  # many ties
+        Kp = int(rng.integers(1, 12))
+        order = np.argsort(-k, kind="stable")  # stable: ties keep the lower index first
+        assert oracle.select_pages_policy("random", kb, Q, Kp, rand_keys=k).tolist() == sorted(order[:Kp].tolist())
+    assert np.array_equal(oracle.select_pages_policy("score", kb, Q, 3), oracle.select_pages(kb, Q, 3)[0])
