@@ -28,6 +28,7 @@ EXPORTED = [
     "hsa_thread_release", "hsa_prepare_history", "hsa_forward_reuse",
     "hkv_store_state_size", "hkv_store_init", "hkv_store_tables", "hkv_store_seal", "hkv_store_fetch",
     "hkv_store_prefetch", "hkv_store_residency", "hkv_select_pages_policy", "hkv_page_scores", "hkv_select_top",
+    "hsa_sparse_attn_lse", "hsa_fidelity",
 ]
 
 POLICY_SCORE, POLICY_RECENT, POLICY_RANDOM = 0, 1, 2
@@ -93,6 +94,8 @@ def load_library(path: str = LIB_PATH):
                                   P]),
         "hkv_select_pages_policy": (I, [I, P, I, P, P, I, I, I, I, P, P, P, P, S, P]),
         "hkv_page_scores": (I, [P, I, P, P, I, I, I, P, P, S, P]),
+        "hsa_sparse_attn_lse": (I, [CP, P, P, P, P, P, _Selection, P, P, P, S, P]),
+        "hsa_fidelity": (I, [CP, P, P, P, P, P, P, P, S, P]),
         "hkv_select_top": (I, [P, I, P, I, P, P, S, P]),
         "hkv_store_state_size": (S, [I, I]),
         "hkv_store_init": (I, [ctypes.POINTER(StoreDesc), P]),
@@ -260,6 +263,36 @@ def hsa_block_select(cfg, Q, Kc, Kq, tau, sel: SelectionBuffers, ws, kbar128=Non
 def hsa_sparse_attn(cfg, Q, Kc, Vc, Kq, Vq, sel: SelectionBuffers, o_sparse, ws, stream=None):
     _check(load_library().hsa_sparse_attn(ctypes.byref(cfg), _p(Q), _p(Kc), _p(Vc), _p(Kq), _p(Vq), sel.c(),
                                           _p(o_sparse), _p(ws), ws.numel(), _stream(stream)), "hsa_sparse_attn")
+
+
+def hsa_sparse_attn_lse(cfg, Q, Kc, Vc, Kq, Vq, sel: SelectionBuffers, o_sparse, lse, ws, stream=None):
+    _check(load_library().hsa_sparse_attn_lse(ctypes.byref(cfg), _p(Q), _p(Kc), _p(Vc), _p(Kq), _p(Vq), sel.c(),
+                                              _p(o_sparse), _p(lse), _p(ws), ws.numel(), _stream(stream)),
+           "hsa_sparse_attn_lse")
+
+
+def hsa_fidelity(cfg, o_ref, lse_ref, o_sparse, lse_sparse, o_linear, report, ws, stream=None):
+    """report: device float64 [H, 5] (see include/hsa.h)."""
+    _check(load_library().hsa_fidelity(ctypes.byref(cfg), _p(o_ref), _p(lse_ref), _p(o_sparse), _p(lse_sparse),
+                                       _p(o_linear), _p(report), _p(ws), ws.numel(), _stream(stream)), "hsa_fidelity")
+
+
+def fidelity_report(cfg, Q, Kc, Vc, Kq, Vq, E, F, sel: SelectionBuffers, ws, ef_head_stride=0):
+    """Both branches of one step against dense attention (the sparse branch with every
+    block kept): float64 [H, 5] on the device (include/hsa.h, hsa_fidelity)."""
+    dense = SelectionBuffers.empty(cfg)
+    ones = torch.ones(cfg.H, dtype=torch.float32, device=Q.device)
+    hsa_block_select(cfg, Q, Kc, Kq, ones, dense, ws)
+    shape = (cfg.Lq, cfg.H, cfg.d)
+    o_ref, o_sp, o_lin = (torch.empty(shape, dtype=torch.float32, device=Q.device) for _ in range(3))
+    lse_ref = torch.empty(cfg.Lq, cfg.H, dtype=torch.float32, device=Q.device)
+    lse_sp = torch.empty_like(lse_ref)
+    hsa_sparse_attn_lse(cfg, Q, Kc, Vc, Kq, Vq, dense, o_ref, lse_ref, ws)
+    hsa_sparse_attn_lse(cfg, Q, Kc, Vc, Kq, Vq, sel, o_sp, lse_sp, ws)
+    hsa_linear_attn(cfg, Q, Kc, Vc, Kq, Vq, E, F, o_lin, ws, ef_head_stride)
+    report = torch.empty(cfg.H, 5, dtype=torch.float64, device=Q.device)
+    hsa_fidelity(cfg, o_ref, lse_ref, o_sp, lse_sp, o_lin, report, ws)
+    return report
 
 
 def hsa_linear_attn(cfg, Q, Kc, Vc, Kq, Vq, E, F, o_linear, ws, ef_head_stride=0, stream=None):

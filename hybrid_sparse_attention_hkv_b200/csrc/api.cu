@@ -667,6 +667,43 @@ hsa_status_t hsa_sparse_attn(const hsa_config_t* cfg, const hsa_bf16* Q, const h
   return HSA_OK;
 }
 
+hsa_status_t hsa_sparse_attn_lse(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc, const hsa_bf16* Vc,
+                                 const hsa_bf16* Kq, const hsa_bf16* Vq, hsa_selection_t sel, float* o_sparse,
+                                 float* lse_out, void* ws, size_t ws_bytes, hsa_stream_t stream) {
+  const char* fn = __func__;
+  TRY(check_cfg(fn, cfg, false));
+  TRY(check_tensors(fn, cfg, Q, Kc, Vc, Kq, Vq, true));
+  TRY(check_sel(fn, sel));
+  REQUIRE_PTR(o_sparse);
+  REQUIRE_PTR(lse_out);
+  const Layout L = make_layout(cfg->H, cfg->d, cfg->Lq, cfg->Lc, 0);
+  TRY(check_ws(fn, ws, ws_bytes, L.attn_end));
+  hsa::AttnArgs a = attn_args(cfg, L, ws, Q, Kc, Vc, Kq, Vq);
+  TRY(run_plan(L, sel, ws, a, stream));
+  a.out_f32 = o_sparse;
+  a.lse_out = lse_out;
+  HSA_LAUNCH("attention", hsa::launch_attn_tc(a, stream));
+  return HSA_OK;
+}
+
+hsa_status_t hsa_fidelity(const hsa_config_t* cfg, const float* o_ref, const float* lse_ref, const float* o_sparse,
+                          const float* lse_sparse, const float* o_linear, double* report, void* ws, size_t ws_bytes,
+                          hsa_stream_t stream) {
+  const char* fn = __func__;
+  TRY(check_cfg(fn, cfg, false));
+  REQUIRE_PTR(o_ref);
+  REQUIRE_PTR(lse_ref);
+  REQUIRE_PTR(o_sparse);
+  REQUIRE_PTR(lse_sparse);
+  REQUIRE_PTR(o_linear);
+  REQUIRE_PTR(report);
+  const size_t need = 256 + (size_t)cfg->H * hsa::kFidelitySplits * 8 * sizeof(double);
+  TRY(check_ws(fn, ws, ws_bytes, need));
+  HSA_LAUNCH("fidelity", hsa::launch_fidelity(o_ref, lse_ref, o_sparse, lse_sparse, o_linear, cfg->Lq, cfg->H, cfg->d,
+                                              at<double>(ws, 256), report, stream));
+  return HSA_OK;
+}
+
 hsa_status_t hsa_linear_attn(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc, const hsa_bf16* Vc,
                              const hsa_bf16* Kq, const hsa_bf16* Vq, const hsa_bf16* E, const hsa_bf16* F,
                              long long ef_head_stride, float* o_linear, void* ws, size_t ws_bytes,

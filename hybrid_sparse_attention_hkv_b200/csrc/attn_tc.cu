@@ -629,6 +629,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (nseg == 1) {
         if (do_sparse && valid_row && !(ls > 0.f)) set_status(status, HSA_ERR_DEVICE);
         const float ws = (do_sparse && ls > 0.f) ? g / ls : 0.f;
+        if (do_sparse && valid_row && a.lse_out)  // ln sum_k exp(q.k * scale) = (m + log2 l) ln 2
+          a.lse_out[(long long)grow * a.H + h] = ls > 0.f ? (ms + log2f(ls)) * 0.6931471805599453f : -INFINITY;
 #pragma unroll
         for (int c = 0; c < D / 16; ++c) {
           uint32_t rs[16], rl[16];
@@ -699,6 +701,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (m_l.x != -INFINITY) L += m_l.y * exp2f(m_l.x - M);
         }
         if (!(L > 0.f)) set_status(status, HSA_ERR_DEVICE);
+        if (a.lse_out) a.lse_out[(long long)grow * a.H + h] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
         const float g = (any_lin && a.gate_logit) ? 1.f / (1.f + expf(-a.gate_logit[h])) : 1.f;
         const float ws = L > 0.f ? g / L : 0.f;
         const float* pl = a.part_lin + ((long long)slot0 * 128 + row) * D;

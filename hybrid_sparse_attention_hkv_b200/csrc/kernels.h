@@ -107,6 +107,7 @@ struct AttnArgs {
   float* out_f32;
   uint16_t* out_bf16;
   int* status;  // workspace status word (may be NULL)
+  float* lse_out;  // optional [Lq][H]: natural-log log-sum-exp of the sparse branch's scaled scores
   // work plan (workspace; sparse branch only -- without it, unit u is query tile u whole)
   int max_units;     // capacity of units (grid size of the attention launch)
   int max_slots;     // capacity of the partial-result slots
@@ -143,6 +144,14 @@ cudaError_t launch_proj_tc(const uint16_t* E, const uint16_t* F, long long ef_he
 cudaError_t launch_proj_reduce(const float* part, int splits, int H, int d, int r, const float* add,
                                float* sum_out, uint16_t* EKhi, uint16_t* EKlo, uint16_t* FVhi, uint16_t* FVlo,
                                cudaStream_t s);
+
+// ---------------------------------------------------------------- fidelity.cu
+// Per-head comparison of the two branches with dense attention (fp64 sums, fixed
+// order): report[h][0..5) = cos(o_lin, o_ref), cos(o_sp, o_ref), mean kept mass
+// exp(lse_sp - lse_ref), |o_lin - o_ref| / |o_ref|, |o_sp - o_ref| / |o_ref|.
+constexpr int kFidelitySplits = 64;
+cudaError_t launch_fidelity(const float* o_ref, const float* lse_ref, const float* o_sp, const float* lse_sp,
+                            const float* o_lin, int Lq, int H, int d, double* part, double* report, cudaStream_t s);
 
 // ---------------------------------------------------------------- waits.cu
 // Write the wait limit (microseconds; 0 = the 2 s default) into a workspace header.

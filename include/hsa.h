@@ -334,6 +334,33 @@ hsa_status_t hsa_sparse_attn(const hsa_config_t* cfg, const hsa_bf16* Q, const h
                              hsa_selection_t sel, float* o_sparse,
                              void* ws, size_t ws_bytes, hsa_stream_t stream);
 
+/* hsa_sparse_attn that also writes, per query row and head, the natural-log
+ * log-sum-exp of the scaled scores over the keys the row attends to:
+ *   lse_out[t * H + h] = ln sum_k exp(q_t . k * scale)                  (fp32 [Lq, H])
+ * With a selection that keeps every block this is dense attention's, and
+ * exp(lse_sparse - lse_dense) is the share of dense attention's softmax mass that
+ * falls inside the kept blocks. */
+hsa_status_t hsa_sparse_attn_lse(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc,
+                                 const hsa_bf16* Vc, const hsa_bf16* Kq, const hsa_bf16* Vq,
+                                 hsa_selection_t sel, float* o_sparse, float* lse_out,
+                                 void* ws, size_t ws_bytes, hsa_stream_t stream);
+
+/* Fidelity of the two branches against dense attention ([NEWS] HSA paragraph,
+ * Figure 6: how much of full attention's global mass and output the linear branch
+ * keeps), a diagnostic on any inputs.  o_ref / lse_ref: dense attention (the
+ * sparse branch with every block kept), o_sparse / lse_sparse: the sparse branch,
+ * o_linear: the linear branch, all [Lq, H, d] fp32 (lse [Lq, H]).  Writes, per head
+ * h, report[5h + k] (device fp64):
+ *   k = 0  cos(o_linear, o_ref)   over the head's rows and columns
+ *   k = 1  cos(o_sparse, o_ref)
+ *   k = 2  mean over rows of exp(lse_sparse - lse_ref): dense mass kept by the blocks
+ *   k = 3  |o_linear - o_ref| / |o_ref|
+ *   k = 4  |o_sparse - o_ref| / |o_ref|
+ * fp64 sums in a fixed order.  Uses the workspace. */
+hsa_status_t hsa_fidelity(const hsa_config_t* cfg, const float* o_ref, const float* lse_ref, const float* o_sparse,
+                          const float* lse_sparse, const float* o_linear, double* report,
+                          void* ws, size_t ws_bytes, hsa_stream_t stream);
+
 /* Linear branch ([NEWS] HSA paragraph, Linformer-style low rank):
  *   EK_h = E_h [Kc; Kq]_h,  FV_h = F_h [Vc; Vq]_h   (E_h, F_h: [r, L], L = Lc+Lq)
  *   o_linear[t, h, :] = softmax_j(q_t . EK_h[j] * scale) FV_h        (fp32 out)

@@ -52,7 +52,7 @@ import numpy as np
 __all__ = [
     "widen", "prompt_top1", "page_summary", "pooled_query", "page_scores", "select_pages", "select_pages_policy",
     "gather_pages", "block_means", "block_probs", "keep_blocks", "Selection", "block_select",
-    "sparse_attention", "linear_projection", "linear_attention", "gate", "gated_merge",
+    "sparse_attention", "linear_projection", "linear_attention", "fidelity", "gate", "gated_merge",
     "hsa_step", "hkv_hsa_step",
 ]
 
@@ -279,6 +279,42 @@ def linear_attention(Q, EK, FV, scale=None, rows=None):
         s -= s.max(axis=1, keepdims=True)
         w = np.exp(s)
         out[:, h] = (w @ FV[h]) / w.sum(axis=1, keepdims=True)
+    return out
+
+
+# --------------------------------------------------------------------------- fidelity diagnostic
+
+def fidelity(Q, Kc, Vc, Kq, Vq, inter, intra, EK, FV, scale=None, Binter=128, Bintra=64):
+    """How close each branch comes to dense attention ([NEWS] HSA paragraph, Figure 6:
+    the linear branch's fidelity to full attention in global mass and in output).
+    Per head h, over all rows t and columns:
+      [0] cos(o_lin, o_dense), [1] cos(o_sparse, o_dense),
+      [2] mean over t of the dense softmax mass of the keys the sparse branch keeps,
+      [3] |o_lin - o_dense| / |o_dense|, [4] |o_sparse - o_dense| / |o_dense|.
+    Dense attention = every key of [Kc; Kq].  Returns [H, 5] float64."""
+    Lq, H, d = Q.shape
+    Lc, Lk = Kc.shape[0], Kq.shape[0]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    all_inter = [[np.arange(-(-Lc // Binter))] * (-(-Lq // Binter))] * H
+    all_intra = [[np.arange(-(-Lk // Bintra))] * (-(-Lq // Bintra))] * H
+    o_ref = sparse_attention(Q, Kc, Vc, Kq, Vq, all_inter, all_intra, scale, Binter, Bintra)
+    o_sp = sparse_attention(Q, Kc, Vc, Kq, Vq, inter, intra, scale, Binter, Bintra)
+    o_lin = linear_attention(Q, EK, FV, scale)
+    out = np.zeros((H, 5))
+    for h in range(H):
+        K = np.concatenate([widen(Kc[:, h]), widen(Kq[:, h])], axis=0)
+        s = (widen(Q[:, h]) @ K.T) * scale
+        s -= s.max(axis=1, keepdims=True)
+        p = np.exp(s)
+        p /= p.sum(axis=1, keepdims=True)
+        mass = np.empty(Lq)
+        for t in range(Lq):
+            kept = np.concatenate([_block_rows(inter[h][t // Binter], Binter, Lc),
+                                   Lc + _block_rows(intra[h][t // Bintra], Bintra, Lk)])
+            mass[t] = p[t, kept].sum()
+        r, sp, li = o_ref[:, h].ravel(), o_sp[:, h].ravel(), o_lin[:, h].ravel()
+        out[h] = [li @ r / np.sqrt((li @ li) * (r @ r)), sp @ r / np.sqrt((sp @ sp) * (r @ r)), mass.mean(),
+                  np.linalg.norm(li - r) / np.linalg.norm(r), np.linalg.norm(sp - r) / np.linalg.norm(r)]
     return out
 
 

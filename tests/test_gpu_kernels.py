@@ -513,3 +513,33 @@ def test_head_groups_emulated_on_one_gpu():
         assert torch.equal(g.selection.inter_cnt, st.selection.inter_cnt[sl])
         assert torch.equal(g.selection.intra_cnt, st.selection.intra_cnt[sl])
         assert float((g.out - full_out[:, sl]).abs().max()) <= 1e-4
+
+
+# ----------------------------------------------------------------- fidelity diagnostic
+
+def test_fidelity_report_matches_the_oracle(small):
+    """Per-head cosine and relative error of both branches against dense attention and
+    the kept dense mass (through the kernel's log-sum-exp), against the oracle's
+    definitions; and the lse of dense attention equals a library log-sum-exp."""
+    x, st, shape = small.x, small.step, small.shape
+    rep = hsa.fidelity_report(st.cfg, small.Q, st.Kc, st.Vc, small.Kq, small.Vq, small.E, small.F, st.selection,
+                              st.ws).cpu().numpy()
+    Kc, Vc = bits_of(st.Kc), bits_of(st.Vc)
+    sb = st.selection
+    inter = selection_lists(sb.inter_idx.cpu().numpy(), sb.inter_cnt.cpu().numpy())
+    intra = selection_lists(sb.intra_idx.cpu().numpy(), sb.intra_cnt.cpu().numpy())
+    EK, FV = oracle.linear_projection(x.E, x.F, Kc, x.Kq, Vc, x.Vq)
+    ref = oracle.fidelity(x.Q, Kc, Vc, x.Kq, x.Vq, inter, intra, EK, FV)
+    np.testing.assert_allclose(rep[:, [0, 1, 2]], ref[:, [0, 1, 2]], atol=2e-3)
+    np.testing.assert_allclose(rep[:, [3, 4]], ref[:, [3, 4]], atol=5e-3, rtol=5e-2)
+    # the dense log-sum-exp itself
+    dense = SelectionBuffers.empty(st.cfg)
+    hsa.hsa_block_select(st.cfg, small.Q, st.Kc, small.Kq, torch.ones(shape.H, device="cuda"), dense, st.ws)
+    o = torch.empty_like(st.out)
+    lse = torch.empty(shape.Lq, shape.H, dtype=torch.float32, device="cuda")
+    hsa.hsa_sparse_attn_lse(st.cfg, small.Q, st.Kc, st.Vc, small.Kq, small.Vq, dense, o, lse, st.ws)
+    torch.cuda.synchronize()
+    K = torch.from_numpy(np.concatenate([oracle.widen(Kc), oracle.widen(x.Kq)]))
+    s = torch.einsum("thc,khc->htk", torch.from_numpy(oracle.widen(x.Q)), K) / math.sqrt(shape.d)
+    want = torch.logsumexp(s, dim=2).T.numpy()
+    np.testing.assert_allclose(lse.cpu().numpy(), want, atol=2e-3)

@@ -494,3 +494,36 @@ def test_retrieval_policies_closed_forms():
         order = np.argsort(-k, kind="stable")  # stable: ties keep the lower index first
         assert oracle.select_pages_policy("random", kb, Q, Kp, rand_keys=k).tolist() == sorted(order[:Kp].tolist())
     assert np.array_equal(oracle.select_pages_policy("score", kb, Q, 3), oracle.select_pages(kb, Q, 3)[0])
+
+
+def test_fidelity_closed_forms():
+    """Keeping every block: the sparse branch is dense attention (cos 1, error 0, mass 1);
+    E = F = I with r = L: the linear branch is dense attention too; the kept mass equals
+    exp(lse_kept - lse_all) computed with a library log-sum-exp."""
+    from scipy.special import logsumexp
+    H, d, Lq, Lc = 2, 8, 128, 256
+    L = Lq + Lc
+    Q = rand_bf16((Lq, H, d), 31, 1)
+    Kc, Vc = rand_bf16((Lc, H, d), 31, 2), rand_bf16((Lc, H, d), 31, 3)
+    Kq, Vq = rand_bf16((Lq, H, d), 31, 4), rand_bf16((Lq, H, d), 31, 5)
+    I = bf16(np.eye(L))
+    EK, FV = oracle.linear_projection(I, I, Kc, Kq, Vc, Vq)
+    full_i = [[np.arange(2)] * 1] * H
+    full_q = [[np.arange(2)] * 2] * H
+    rep = oracle.fidelity(Q, Kc, Vc, Kq, Vq, full_i, full_q, EK, FV)
+    np.testing.assert_allclose(rep[:, [0, 1, 2]], 1.0, atol=1e-12)
+    np.testing.assert_allclose(rep[:, [3, 4]], 0.0, atol=1e-12)
+    inter = [[np.array([1])], [np.array([0])]]
+    intra = [[np.array([0]), np.array([0, 1])], [np.array([1]), np.array([1])]]
+    rep = oracle.fidelity(Q, Kc, Vc, Kq, Vq, inter, intra, EK, FV)
+    scale = 1 / math.sqrt(d)
+    for h in range(H):
+        K = np.concatenate([oracle.widen(Kc[:, h]), oracle.widen(Kq[:, h])])
+        s = oracle.widen(Q[:, h]) @ K.T * scale
+        m = []
+        for t in range(Lq):
+            kept = [k for k in range(L) if (k < Lc and k // 128 in inter[h][0]) or
+                    (k >= Lc and (k - Lc) // 64 in intra[h][t // 64])]
+            m.append(np.exp(logsumexp(s[t, kept]) - logsumexp(s[t])))
+        assert abs(rep[h, 2] - np.mean(m)) < 1e-12
+        assert 0 < rep[h, 2] < 1 and rep[h, 1] < 1 and rep[h, 4] > 0
