@@ -28,7 +28,8 @@ EXPORTED = [
     "hsa_thread_release", "hsa_prepare_history", "hsa_forward_reuse",
     "hkv_store_state_size", "hkv_store_init", "hkv_store_tables", "hkv_store_seal", "hkv_store_fetch",
     "hkv_store_prefetch", "hkv_store_residency", "hkv_select_pages_policy", "hkv_page_scores", "hkv_select_top",
-    "hsa_sparse_attn_lse", "hsa_fidelity",
+    "hsa_sparse_attn_lse", "hsa_fidelity", "hkv_page_block_sums", "hkv_block_means_from_pages",
+    "hsa_forward_selected",
 ]
 
 POLICY_SCORE, POLICY_RECENT, POLICY_RANDOM = 0, 1, 2
@@ -43,7 +44,10 @@ class HsaError(RuntimeError):
 class Config(ctypes.Structure):
     _fields_ = [("H", ctypes.c_int), ("d", ctypes.c_int), ("Lq", ctypes.c_int), ("Lc", ctypes.c_int),
                 ("block_inter", ctypes.c_int), ("block_intra", ctypes.c_int), ("rank", ctypes.c_int),
-                ("scale", ctypes.c_float)]
+                ("scale", ctypes.c_float), ("select_mode", ctypes.c_int)]
+
+
+SELECT_SEPARATE, SELECT_JOINT = 0, 1
 
 
 class StoreDesc(ctypes.Structure):
@@ -95,6 +99,9 @@ def load_library(path: str = LIB_PATH):
         "hkv_select_pages_policy": (I, [I, P, I, P, P, I, I, I, I, P, P, P, P, S, P]),
         "hkv_page_scores": (I, [P, I, P, P, I, I, I, P, P, S, P]),
         "hsa_sparse_attn_lse": (I, [CP, P, P, P, P, P, _Selection, P, P, P, S, P]),
+        "hkv_page_block_sums": (I, [P, I, I, I, P, P]),
+        "hkv_block_means_from_pages": (I, [P, I, P, I, I, I, I, P, P, S, P]),
+        "hsa_forward_selected": (I, [CP, P, P, P, P, P, P, P, P, L, ctypes.POINTER(_Selection), P, I, P, S, P]),
         "hsa_fidelity": (I, [CP, P, P, P, P, P, P, P, S, P]),
         "hkv_select_top": (I, [P, I, P, I, P, P, S, P]),
         "hkv_store_state_size": (S, [I, I]),
@@ -131,8 +138,8 @@ def _stream(stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def make_config(H, d, Lq, Lc, rank=0, scale=0.0, block_inter=128, block_intra=64) -> Config:
-    return Config(H, d, Lq, Lc, block_inter, block_intra, rank, scale)
+def make_config(H, d, Lq, Lc, rank=0, scale=0.0, block_inter=128, block_intra=64, select_mode=0) -> Config:
+    return Config(H, d, Lq, Lc, block_inter, block_intra, rank, scale, select_mode)
 
 
 def hsa_workspace_size(cfg: Config, NP: int = 0, P_tok: int = 0) -> int:
@@ -180,7 +187,10 @@ class SelectionBuffers:
 
     @staticmethod
     def empty(cfg: Config, device="cuda") -> "SelectionBuffers":
+        """Buffers of one selection; in joint mode the inter rows are per 64-row query block."""
         nQ128, nQ64 = -(-cfg.Lq // 128), -(-cfg.Lq // 64)
+        if cfg.select_mode == SELECT_JOINT:
+            nQ128 = nQ64
         nKc = -(-cfg.Lc // 128)
         i32 = dict(dtype=torch.int32, device=device)
         return SelectionBuffers(torch.zeros(cfg.H, nQ128, max(nKc, 1), **i32), torch.zeros(cfg.H, nQ128, **i32),
@@ -246,6 +256,20 @@ def hkv_select_pages_noalloc(kbar_pages, Q, Kp, sel_out, scores_out=None, cand_r
            "hkv_select_pages_noalloc")
 
 
+def hkv_page_block_sums(K_page, sums64, stream=None):
+    """64-row key sums of one page ([ceil(P_tok/64), H, d] fp32)."""
+    P_tok, H, d = K_page.shape
+    _check(load_library().hkv_page_block_sums(_p(K_page), P_tok, H, d, _p(sums64), _stream(stream)),
+           "hkv_page_block_sums")
+
+
+def hkv_block_means_from_pages(sums64_pages, sel, Kp, P_tok, H, d, kbar128, ws, stream=None):
+    NP = sums64_pages.shape[0]
+    _check(load_library().hkv_block_means_from_pages(_p(sums64_pages), NP, _p(sel), Kp, P_tok, H, d, _p(kbar128),
+                                                     _p(ws), ws.numel(), _stream(stream)),
+           "hkv_block_means_from_pages")
+
+
 def hkv_gather(page_k_ptrs, page_v_ptrs, sel, Kp, P_tok, H, d, Kc, Vc, ws, kbar128=None, stream=None):
     """page_k_ptrs / page_v_ptrs: device int64 tensors [NP] of page base addresses."""
     NP = page_k_ptrs.numel()
@@ -309,6 +333,15 @@ def hsa_forward(cfg, Q, Kc, Vc, Kq, Vq, tau, gate_logit, E, F, out, ws, kbar128=
                                       _p(tau), _p(gate_logit), _p(E), _p(F), ef_head_stride, _p(out),
                                       1 if out.dtype == torch.bfloat16 else 0, csel, _p(ws), ws.numel(),
                                       _stream(stream)), "hsa_forward")
+
+
+def hsa_forward_selected(cfg, Q, Kc, Vc, Kq, Vq, gate_logit, E, F, sel: SelectionBuffers, out, ws, ef_head_stride=0,
+                         stream=None):
+    """hsa_forward with the selection `sel` already made (input)."""
+    _check(load_library().hsa_forward_selected(ctypes.byref(cfg), _p(Q), _p(Kc), _p(Vc), _p(Kq), _p(Vq),
+                                               _p(gate_logit), _p(E), _p(F), ef_head_stride, ctypes.byref(sel.c()),
+                                               _p(out), 1 if out.dtype == torch.bfloat16 else 0, _p(ws), ws.numel(),
+                                               _stream(stream)), "hsa_forward_selected")
 
 
 def hsa_prepare_history(cfg, Kc, Vc, E, F, ws, ef_head_stride=0, stream=None):

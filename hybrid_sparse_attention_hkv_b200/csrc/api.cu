@@ -103,8 +103,8 @@ Layout make_layout(int H, int d, int Lq, long long Lc, int r) {
   L.q64 = take(nQ64 * hd * 4);
   L.kq64 = take(nQ64 * hd * 4);
   L.kc128 = take(nKc * hd * 4);
-  L.inter_idx = take((size_t)H * nQ128 * nKc * 4);
-  L.inter_cnt = take((size_t)H * nQ128 * 4);
+  L.inter_idx = take((size_t)H * nQ64 * nKc * 4);  // nQ64 rows: room for the joint mode's per-64-row lists
+  L.inter_cnt = take((size_t)H * nQ64 * 4);
   L.intra_idx = take((size_t)H * nQ64 * nQ64 * 4);
   L.intra_cnt = take((size_t)H * nQ64 * 4);
   // attention work plan and the partial results of split lists
@@ -155,6 +155,10 @@ hsa_status_t check_cfg(const char* fn, const hsa_config_t* c, bool need_rank) {
   if ((c->Lc + 127) / 128 > hsa::kMaxSelBlocks || (c->Lq + 63) / 64 > hsa::kMaxSelBlocks)
     return fail(HSA_ERR_UNSUPPORTED, "%s: more than %d blocks in a selection row", fn, hsa::kMaxSelBlocks);
   if (!(c->scale >= 0.f) || isinf(c->scale)) return fail(HSA_ERR_INVALID_ARG, "%s: scale must be finite and >= 0", fn);
+  if (c->select_mode != HSA_SELECT_SEPARATE && c->select_mode != HSA_SELECT_JOINT)
+    return fail(HSA_ERR_INVALID_ARG, "%s: select_mode = %d", fn, c->select_mode);
+  if (c->select_mode == HSA_SELECT_JOINT && (c->Lc + 127) / 128 + (c->Lq + 63) / 64 > 2 * hsa::kMaxSelBlocks)
+    return fail(HSA_ERR_UNSUPPORTED, "%s: more than %d blocks in a joint selection row", fn, 2 * hsa::kMaxSelBlocks);
   if (need_rank && (c->rank < 64 || c->rank > 1024 || c->rank % 64 != 0))
     return fail(HSA_ERR_UNSUPPORTED, "%s: rank = %d (supported: multiples of 64 in [64, 1024])", fn, c->rank);
   return HSA_OK;
@@ -448,6 +452,32 @@ hsa_status_t hkv_gather(const hsa_bf16* const* page_k, const hsa_bf16* const* pa
   return HSA_OK;
 }
 
+hsa_status_t hkv_page_block_sums(const hsa_bf16* K_page, int P_tok, int H, int d, float* sums64, hsa_stream_t stream) {
+  const char* fn = __func__;
+  TRY(check_heads(fn, H, d));
+  if (P_tok < 1) return fail(HSA_ERR_INVALID_ARG, "%s: P_tok = %d must be >= 1", fn, P_tok);
+  REQUIRE_PTR(K_page);
+  REQUIRE_PTR(sums64);
+  HSA_LAUNCH("block_sums64", hsa::launch_block_sums64(K_page, P_tok, H * d, sums64, stream));
+  return HSA_OK;
+}
+
+hsa_status_t hkv_block_means_from_pages(const float* sums64_pages, int NP, const int32_t* sel, int Kp, int P_tok,
+                                        int H, int d, float* kbar128, void* ws, size_t ws_bytes, hsa_stream_t stream) {
+  const char* fn = __func__;
+  TRY(check_heads(fn, H, d));
+  if (NP < 1 || P_tok < 1) return fail(HSA_ERR_INVALID_ARG, "%s: NP = %d, P_tok = %d must be >= 1", fn, NP, P_tok);
+  if (P_tok % 64 != 0) return fail(HSA_ERR_UNSUPPORTED, "%s: P_tok = %d is not a multiple of 64", fn, P_tok);
+  if (Kp < 1 || Kp > NP) return fail(HSA_ERR_INVALID_ARG, "%s: Kp = %d must be in [1, NP]", fn, Kp);
+  REQUIRE_PTR(sums64_pages);
+  REQUIRE_PTR(kbar128);
+  if (!sel) return fail(HSA_ERR_INVALID_ARG, "%s: sel is NULL", fn);
+  TRY(check_ws(fn, ws, ws_bytes, 256));
+  HSA_LAUNCH("kc128_from_pages", hsa::launch_kc128_from_pages(sums64_pages, NP, P_tok, sel, Kp, H * d, kbar128,
+                                                              status_of(ws), stream));
+  return HSA_OK;
+}
+
 // ------------------------------------------------------------------ tiered page store
 
 static hsa_status_t store_desc(const char* fn, const hkv_store_t* st, hsa::StoreDesc* out) {
@@ -566,8 +596,9 @@ static hsa_status_t run_block_select(const hsa_config_t* cfg, const Layout& L, c
   HSA_LAUNCH("pool", hsa::launch_pool(Q, Kq, Kc, cfg->H, cfg->d, cfg->Lq, cfg->Lc, q128, q64, kq64,
                                       kbar128 ? nullptr : kc128, stream));
   HSA_LAUNCH("block_select", hsa::launch_block_select(q128, kc128, q64, kq64, tau, cfg->H, cfg->d, cfg->Lq, cfg->Lc,
-                                                      scale_of(cfg), sel.inter_idx, sel.inter_cnt, sel.intra_idx,
-                                                      sel.intra_cnt, stream));
+                                                      scale_of(cfg), cfg->select_mode == HSA_SELECT_JOINT,
+                                                      sel.inter_idx, sel.inter_cnt, sel.intra_idx, sel.intra_cnt,
+                                                      stream));
   return HSA_OK;
 }
 
@@ -578,6 +609,7 @@ static hsa::AttnArgs attn_args(const hsa_config_t* cfg, const Layout& L, void* w
   a.Q = Q; a.Kc = Kc; a.Vc = Vc; a.Kq = Kq; a.Vq = Vq;
   a.H = cfg->H; a.d = cfg->d; a.Lq = cfg->Lq; a.Lc = cfg->Lc;
   a.scale = scale_of(cfg);
+  a.joint = cfg->select_mode == HSA_SELECT_JOINT;
   a.r = cfg->rank;
   a.status = status_of(ws);
   a.max_units = L.max_units;
@@ -730,11 +762,12 @@ static hsa_status_t forward_impl(const char* fn, const hsa_config_t* cfg, const 
                                  const float* tau, const float* gate_logit, const hsa_bf16* E, const hsa_bf16* F,
                                  long long ef_head_stride, void* out, int out_is_bf16,
                                  const hsa_selection_t* sel_out, void* ws, size_t ws_bytes, int which_part,
-                                 hsa_stream_t stream) {
+                                 bool selected, hsa_stream_t stream) {
   TRY(check_cfg(fn, cfg, true));
   TRY(check_tensors(fn, cfg, Q, Kc, Vc, Kq, Vq, true));
   OPTIONAL_PTR(kbar128);
-  if (!tau || !gate_logit) return fail(HSA_ERR_INVALID_ARG, "%s: tau / gate_logit is NULL", fn);
+  if ((!selected && !tau) || !gate_logit) return fail(HSA_ERR_INVALID_ARG, "%s: tau / gate_logit is NULL", fn);
+  if (selected && !sel_out) return fail(HSA_ERR_INVALID_ARG, "%s: the selection is NULL", fn);
   REQUIRE_PTR(E);
   REQUIRE_PTR(F);
   REQUIRE_PTR(out);
@@ -765,7 +798,7 @@ static hsa_status_t forward_impl(const char* fn, const hsa_config_t* cfg, const 
   TRY(run_projection(cfg, L, Kc, Vc, Kq, Vq, E, F, ef_head_stride, ws, a, which_part, side->s));
   if ((e = cudaEventRecord(side->join, side->s)) != cudaSuccess)
     return fail(HSA_ERR_CUDA, "%s: side stream: %s", fn, cudaGetErrorString(e));
-  TRY(run_block_select(cfg, L, Q, Kc, Kq, kbar128, tau, sel, ws, stream));
+  if (!selected) TRY(run_block_select(cfg, L, Q, Kc, Kq, kbar128, tau, sel, ws, stream));
   TRY(run_plan(L, sel, ws, a, stream));
   if ((e = cudaStreamWaitEvent(stream, side->join, 0)) != cudaSuccess)
     return fail(HSA_ERR_CUDA, "%s: side stream: %s", fn, cudaGetErrorString(e));
@@ -782,7 +815,15 @@ hsa_status_t hsa_forward(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_b
                          void* out, int out_is_bf16, const hsa_selection_t* sel_out, void* ws, size_t ws_bytes,
                          hsa_stream_t stream) {
   return forward_impl(__func__, cfg, Q, Kc, Vc, Kq, Vq, kbar128, tau, gate_logit, E, F, ef_head_stride, out,
-                      out_is_bf16, sel_out, ws, ws_bytes, hsa::kProjAll, stream);
+                      out_is_bf16, sel_out, ws, ws_bytes, hsa::kProjAll, false, stream);
+}
+
+hsa_status_t hsa_forward_selected(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc, const hsa_bf16* Vc,
+                                  const hsa_bf16* Kq, const hsa_bf16* Vq, const float* gate_logit, const hsa_bf16* E,
+                                  const hsa_bf16* F, long long ef_head_stride, const hsa_selection_t* sel, void* out,
+                                  int out_is_bf16, void* ws, size_t ws_bytes, hsa_stream_t stream) {
+  return forward_impl(__func__, cfg, Q, Kc, Vc, Kq, Vq, nullptr, nullptr, gate_logit, E, F, ef_head_stride, out,
+                      out_is_bf16, sel, ws, ws_bytes, hsa::kProjAll, true, stream);
 }
 
 hsa_status_t hsa_prepare_history(const hsa_config_t* cfg, const hsa_bf16* Kc, const hsa_bf16* Vc, const hsa_bf16* E,
@@ -821,7 +862,7 @@ hsa_status_t hsa_forward_reuse(const hsa_config_t* cfg, const hsa_bf16* Q, const
                                long long ef_head_stride, void* out, int out_is_bf16, const hsa_selection_t* sel_out,
                                void* ws, size_t ws_bytes, hsa_stream_t stream) {
   return forward_impl(__func__, cfg, Q, Kc, Vc, Kq, Vq, kbar128, tau, gate_logit, E, F, ef_head_stride, out,
-                      out_is_bf16, sel_out, ws, ws_bytes, hsa::kProjChunk, stream);
+                      out_is_bf16, sel_out, ws, ws_bytes, hsa::kProjChunk, false, stream);
 }
 
 }  // extern "C"

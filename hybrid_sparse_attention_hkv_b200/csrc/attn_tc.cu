@@ -8,7 +8,9 @@
 // 128-query tile).  The list, in order:
 //   linear tiles  64 rows of EK / FV (split bf16 hi + lo), r / 64 of them, in
 //                 segment 0 only;
-//   cached tiles  one 128-row tile per kept inter block of the cached KV;
+//   cached tiles  one 128-row tile per kept inter block of the cached KV (with the
+//                 joint block selection, the union of the two 64-query halves'
+//                 inter lists, each tile tagged with the halves that keep it);
 //   chunk tiles   the union of the two 64-query halves' kept 64-row intra blocks,
 //                 each tagged with the halves that use it; blocks with the same tag
 //                 are paired into 128-row tiles (two 64-row boxes in one slot), so
@@ -264,10 +266,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   int* tiles = reinterpret_cast<int*>(smem + Lay::kBytes);  // [r/64 + nKc + nKq]
   int* flags = tiles + (a.EKhi ? a.r / 64 : 0) + nKc + nKq; // [nKq]
   int* scratch = flags + nKq;                                 // [nKq]
+  int* flagc = scratch + nKq;                                 // [nKc] (joint selection)
   __shared__ __align__(8) uint64_t bar_q, bar_k_full[kKStages], bar_k_empty[kKStages], bar_v_full[kVStages],
       bar_v_empty[kVStages], bar_s_full[2], bar_p_full[2], bar_o_done, bar_final;
   __shared__ uint32_t s_tmem;
-  __shared__ int s_ntiles, s_n2;
+  __shared__ int s_ntiles, s_n2, s_ninter;
 
   __shared__ int s_last;
 
@@ -318,19 +321,35 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const bool do_lin = any_lin && seg == 0;  // the linear tiles belong to segment 0
   const bool do_sparse = a.inter_cnt != nullptr;
   const int n_lin = do_lin ? a.r / 64 : 0;
-  const int n_inter = do_sparse ? min(max(a.inter_cnt[(long long)h * nQ128 + qb], 0), nKc) : 0;
+  const int n_inter0 = (do_sparse && !a.joint) ? min(max(a.inter_cnt[(long long)h * nQ128 + qb], 0), nKc) : 0;
   for (int t = tid; t < n_lin; t += kTcThreads) tiles[t] = tc_tile_code((long long)t * 64, kTileLinear, 3);
   if (do_sparse) {
     const int32_t* ilist = a.inter_idx + ((long long)h * nQ128 + qb) * nKc;
-    for (int m = tid; m < n_inter; m += kTcThreads) {
+    for (int m = tid; m < n_inter0; m += kTcThreads) {
       const long long j = ilist[m];
       const bool ok = j >= 0 && j < nKc;
       if (!ok) set_status(status, HSA_ERR_DEVICE);
       tiles[n_lin + m] = ok ? tc_tile_code(j * 128, kTileCached, 3) : tc_tile_code(0, kTileCached, 0);
     }
     for (int j = tid; j < nKq; j += kTcThreads) flags[j] = 0;
+    if (a.joint)
+      for (int j = tid; j < nKc; j += kTcThreads) flagc[j] = 0;
   }
   __syncthreads();
+  if (do_sparse && a.joint) {  // the two 64-query halves' inter lists
+    for (int half = 0; half < 2; ++half) {
+      const int i64 = 2 * qb + half;
+      if (i64 < nQ64) {
+        const int cnt = min(max(a.inter_cnt[(long long)h * nQ64 + i64], 0), nKc);
+        const int32_t* lst = a.inter_idx + ((long long)h * nQ64 + i64) * nKc;
+        for (int m = tid; m < cnt; m += kTcThreads) {
+          const int j = lst[m];
+          if (j >= 0 && j < nKc) atomicOr(&flagc[j], 1 << half);
+          else set_status(status, HSA_ERR_DEVICE);
+        }
+      }
+    }
+  }
   if (do_sparse) {
     for (int half = 0; half < 2; ++half) {
       const int i64 = 2 * qb + half;
@@ -347,6 +366,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
   __syncthreads();
   if (warp == 0) {
+    int n_inter = n_inter0;
+    if (do_sparse && a.joint) {  // cached blocks kept by either half, ascending, tagged
+      n_inter = 0;
+      for (int b = 0; b < nKc; b += 32) {
+        const int j = b + lane;
+        const int f = j < nKc ? flagc[j] : 0;
+        const unsigned bal = __ballot_sync(0xffffffffu, f != 0);
+        if (f) tiles[n_lin + n_inter + __popc(bal & ((1u << lane) - 1u))] = tc_tile_code((long long)j * 128, kTileCached, f);
+        n_inter += __popc(bal);
+      }
+    }
     // chunk blocks by tag (both halves, half 0 only, half 1 only), ascending within a
     // tag, paired; a tag's odd block out stays a 64-row tile at the end of the list.
     // The partial last block (the largest id) is always the second of its pair.
@@ -380,6 +410,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0) {
       s_ntiles = base;
       s_n2 = n2;
+      s_ninter = n_inter;
     }
   }
   tc_fence_before();
@@ -388,6 +419,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // this segment's share of the sparse tiles, by cost (a 128-row tile costs 2, a lone
   // 64-row chunk tile 1; the 128-row tiles come first)
   const int n2 = s_n2;
+  const int n_inter = s_ninter;
   const int n1 = s_ntiles - n_lin - n2;
   const long long cost = 2LL * n2 + n1;
   auto cut = [&](long long x) -> int {  // sparse tiles whose cumulative cost before them is < x
@@ -786,7 +818,7 @@ cudaError_t launch_tc(const AttnArgs& a, cudaStream_t s) {
   if ((e = make_map(&maps.fvhi, lin ? a.FVhi : a.Vq, lin ? pr : a.Lq, lin ? D : HD, 64)) != cudaSuccess) return e;
   if ((e = make_map(&maps.fvlo, lin ? a.FVlo : a.Vq, lin ? pr : a.Lq, lin ? D : HD, 64)) != cudaSuccess) return e;
   const int n_lin = lin ? a.r / 64 : 0;
-  const size_t smem = 1024 + TcLayout<D>::kBytes + (size_t)(n_lin + nKc + 3 * nKq) * 4;
+  const size_t smem = 1024 + TcLayout<D>::kBytes + (size_t)(n_lin + 2 * nKc + 3 * nKq) * 4;
   if (smem > 232448) return cudaErrorInvalidConfiguration;
   e = cudaFuncSetAttribute(sparse_attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -354,6 +354,82 @@ cudaError_t launch_select_prompt(const float* e_cur, const float* e_seg, int n_s
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ 64-row key sums of a page
+// sums[b][c] = sum over the rows [64 b, min(64 b + 64, n)) of X[row][c], fp32 in row
+// order (a page's keys, once when it is sealed).  Thread = 16-byte column chunk.
+constexpr int kSumThreads = 128;
+
+__global__ void __launch_bounds__(kSumThreads) block_sums64_kernel(const uint16_t* __restrict__ X, long long n, int C,
+                                                                  float* __restrict__ sums) {
+  const long long b = blockIdx.x;
+  const int cc = blockIdx.y * kSumThreads + threadIdx.x;
+  if (cc * 8 >= C) return;
+  const long long r0 = b * 64, r1 = min(n, r0 + 64);
+  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  long long r = r0;
+  for (; r + 8 <= r1; r += 8) {
+    uint4 w[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) w[u] = ld_nc_v4(X + (r + u) * C + cc * 8);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) add8(acc, w[u]);
+  }
+  for (; r < r1; ++r) add8(acc, ld_nc_v4(X + r * C + cc * 8));
+  float4* out = reinterpret_cast<float4*>(sums + b * C + cc * 8);
+  out[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+  out[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+}
+
+cudaError_t launch_block_sums64(const uint16_t* X, long long n, int C, float* sums, cudaStream_t s) {
+  const long long nb = (n + 63) / 64;
+  const int cols = (C / 8 + kSumThreads - 1) / kSumThreads;
+  block_sums64_kernel<<<dim3((unsigned)nb, cols), kSumThreads, 0, s>>>(X, n, C, sums);
+  return cudaGetLastError();
+}
+
+// kbar128[j] of the active cache gathered from pages sel[0..Kp) (P_tok a multiple of
+// 64, so each 64-row half of a 128-row block lies in one page): the two halves'
+// stored sums, added in order, over the block's rows.  Needs only the selection,
+// not the gathered copy.
+__global__ void __launch_bounds__(kSumThreads) kc128_from_pages_kernel(const float* __restrict__ sums, int NP,
+                                                                      long long nb64_page,
+                                                                      const int32_t* __restrict__ sel, long long Lc,
+                                                                      int C, float* __restrict__ kbar128,
+                                                                      int* status) {
+  const long long j = blockIdx.x;
+  const int cc = blockIdx.y * kSumThreads + threadIdx.x;
+  if (cc * 8 >= C) return;
+  const long long P_tok = nb64_page * 64;
+  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int u = 0; u < 2; ++u) {
+    const long long r = j * 128 + u * 64;  // first gathered row of this half
+    if (r >= Lc) break;
+    const int p = sel[r / P_tok];
+    if (p < 0 || p >= NP) {
+      set_status(status, HSA_ERR_DEVICE);
+      continue;
+    }
+    const float4* src = reinterpret_cast<const float4*>(sums + ((long long)p * nb64_page + (r % P_tok) / 64) * C + cc * 8);
+    const float4 a = src[0], b = src[1];
+    acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+    acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
+  }
+  const float inv = 1.f / (float)min(128LL, Lc - j * 128);
+  float4* out = reinterpret_cast<float4*>(kbar128 + j * C + cc * 8);
+  out[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+  out[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+}
+
+cudaError_t launch_kc128_from_pages(const float* sums, int NP, long long P_tok, const int32_t* sel, int Kp, int C,
+                                    float* kbar128, int* status, cudaStream_t s) {
+  const long long Lc = (long long)Kp * P_tok;
+  const long long nKc = (Lc + 127) / 128;
+  const int cols = (C / 8 + kSumThreads - 1) / kSumThreads;
+  kc128_from_pages_kernel<<<dim3((unsigned)nKc, cols), kSumThreads, 0, s>>>(sums, NP, P_tok / 64, sel, Lc, C,
+                                                                           kbar128, status);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ gather
 // Unit = (K or V, 128-row block j of the output): 128 full rows (all heads).
 // Row R of the output comes from page sel[R / P_tok], row R % P_tok; a row is

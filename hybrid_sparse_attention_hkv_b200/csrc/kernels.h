@@ -38,6 +38,11 @@ cudaError_t launch_policy_keys(int policy, const float* rand_keys, int NP, float
 cudaError_t launch_select_prompt(const float* e_cur, const float* e_seg, int n_seg, int dim,
                                  const int32_t* seg_begin, int32_t* seg_out, int32_t* cand_range_out,
                                  cudaStream_t s);
+// 64-row key sums of a page ([ceil(n/64)][C] fp32) and the active cache's 128-row
+// key means from them (P_tok % 64 == 0).
+cudaError_t launch_block_sums64(const uint16_t* X, long long n, int C, float* sums, cudaStream_t s);
+cudaError_t launch_kc128_from_pages(const float* sums, int NP, long long P_tok, const int32_t* sel, int Kp, int C,
+                                    float* kbar128, int* status, cudaStream_t s);
 cudaError_t launch_gather(const uint16_t* const* page_k, const uint16_t* const* page_v, int NP,
                           const int32_t* sel, int Kp, long long P_tok, int H, int d, uint16_t* Kc,
                           uint16_t* Vc, float* kbar128, int* status, cudaStream_t s);
@@ -67,8 +72,10 @@ constexpr int kMaxSelBlocks = 8192;  // blocks per selection row (inter: ceil(Lc
 
 cudaError_t launch_pool(const uint16_t* Q, const uint16_t* Kq, const uint16_t* Kc, int H, int d, int Lq,
                         long long Lc, float* q128, float* q64, float* kq64, float* kc128, cudaStream_t s);
+// joint: one softmax per 64-row query block over its Kc and Kq blocks (inter rows per
+// 64-row query block); else the two maps separately.
 cudaError_t launch_block_select(const float* q128, const float* kc128, const float* q64, const float* kq64,
-                                const float* tau, int H, int d, int Lq, long long Lc, float scale,
+                                const float* tau, int H, int d, int Lq, long long Lc, float scale, bool joint,
                                 int32_t* inter_idx, int32_t* inter_cnt, int32_t* intra_idx, int32_t* intra_cnt,
                                 cudaStream_t s);
 
@@ -90,6 +97,7 @@ struct AttnArgs {
   int H, d, Lq;
   long long Lc;
   float scale;
+  bool joint;  // inter lists per 64-row query block (joint block selection)
   // sparse branch (runs when inter_cnt != NULL)
   const int32_t* inter_idx;
   const int32_t* inter_cnt;

@@ -50,7 +50,16 @@ __device__ int block_exclusive_scan(int v, int* s_warp, int& total) {
 // Cost of (head, query tile) i in 128-row tile units (x2, to count chunk tiles exactly).
 __device__ __forceinline__ int cost2(const AttnArgs& a, int i, int nQ128, int nQ64, int nKc, int nKq) {
   const int h = i / nQ128, qb = i % nQ128;
-  const int ni = min(max(a.inter_cnt[i], 0), nKc);
+  int ni = 0;
+  if (a.joint) {  // inter lists per 64-query half: their sum bounds the union
+    for (int half = 0; half < 2; ++half) {
+      const int i64 = 2 * qb + half;
+      if (i64 < nQ64) ni += min(max(a.inter_cnt[(long long)h * nQ64 + i64], 0), nKc);
+    }
+    ni = min(ni, nKc);
+  } else {
+    ni = min(max(a.inter_cnt[i], 0), nKc);
+  }
   int nc = 0;
   for (int half = 0; half < 2; ++half) {
     const int i64 = 2 * qb + half;

@@ -96,7 +96,9 @@ cudaError_t launch_pool(const uint16_t* Q, const uint16_t* Kq, const uint16_t* K
 }
 
 // ------------------------------------------------------------------ block selection
-// One CTA per selection row (head h, query block i, map inter|intra):
+// One CTA per selection row (head h, query block i, map inter|intra; in joint mode
+// one row per (head, 64-row query block) over the Kc blocks followed by the Kq
+// blocks, whose kept ids are split into the row's inter and intra lists):
 //   s_j = qbar_i . kbar_j * scale                 (fp32, one warp per block)
 //   e_j = exp(s_j - max_j s_j);  total = sum_j e_j (fp64)
 //   rank by e descending (ties -> lower j)        (bitonic sort in shared memory)
@@ -141,8 +143,8 @@ template <int D>
 __global__ void __launch_bounds__(kSelThreads) block_select_kernel(
     const float* __restrict__ q128, const float* __restrict__ kc128, const float* __restrict__ q64,
     const float* __restrict__ kq64, const float* __restrict__ tau, int H, int nQ128, int nKc, int nQ64, int nKq,
-    float scale, int32_t* __restrict__ inter_idx, int32_t* __restrict__ inter_cnt, int32_t* __restrict__ intra_idx,
-    int32_t* __restrict__ intra_cnt) {
+    float scale, bool joint, int32_t* __restrict__ inter_idx, int32_t* __restrict__ inter_cnt,
+    int32_t* __restrict__ intra_idx, int32_t* __restrict__ intra_cnt) {
   extern __shared__ __align__(16) unsigned char smraw[];
   __shared__ float qv[D];
   __shared__ double dred[40];
@@ -152,38 +154,63 @@ __global__ void __launch_bounds__(kSelThreads) block_select_kernel(
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   int row = blockIdx.x;
-  const bool inter = row < H * nQ128;
-  int h, i, nK;
+  // the row's keys are kbA[0 .. nA) followed by kbB[0 .. nK - nA); kept ids < nA go
+  // to idx_out / cnt_out, the others (minus nA) to idx_out2 / cnt_out2
+  int h, i, nK, nA;
   const float* qb;
-  const float* kb;
+  const float* kbA;
+  const float* kbB = nullptr;
   int32_t* idx_out;
   int32_t* cnt_out;
-  if (inter) {
+  int32_t* idx_out2 = nullptr;
+  int32_t* cnt_out2 = nullptr;
+  if (joint) {
+    h = row / nQ64;
+    i = row % nQ64;
+    nA = nKc;
+    nK = nKc + nKq;
+    qb = q64 + ((long long)i * H + h) * D;
+    kbA = kc128;
+    kbB = kq64;
+    idx_out = inter_idx + ((long long)h * nQ64 + i) * nKc;
+    cnt_out = inter_cnt + (long long)h * nQ64 + i;
+    idx_out2 = intra_idx + ((long long)h * nQ64 + i) * nKq;
+    cnt_out2 = intra_cnt + (long long)h * nQ64 + i;
+  } else if (row < H * nQ128) {
     h = row / nQ128;
     i = row % nQ128;
-    nK = nKc;
+    nK = nA = nKc;
     qb = q128 + ((long long)i * H + h) * D;
-    kb = kc128;
+    kbA = kc128;
     idx_out = inter_idx + ((long long)h * nQ128 + i) * nKc;
     cnt_out = inter_cnt + (long long)h * nQ128 + i;
   } else {
     row -= H * nQ128;
     h = row / nQ64;
     i = row % nQ64;
-    nK = nKq;
+    nK = nA = nKq;
     qb = q64 + ((long long)i * H + h) * D;
-    kb = kq64;
+    kbA = kq64;
     idx_out = intra_idx + ((long long)h * nQ64 + i) * nKq;
     cnt_out = intra_cnt + (long long)h * nQ64 + i;
   }
   if (nK == 0) {
-    if (tid == 0) *cnt_out = 0;
+    if (tid == 0) {
+      *cnt_out = 0;
+      if (cnt_out2) *cnt_out2 = 0;
+    }
     return;
   }
   const float t = tau[h];
   if (t >= 1.0f) {
-    for (int j = tid; j < nK; j += kSelThreads) idx_out[j] = j;
-    if (tid == 0) *cnt_out = nK;
+    for (int j = tid; j < nK; j += kSelThreads) {
+      if (j < nA) idx_out[j] = j;
+      else idx_out2[j - nA] = j - nA;
+    }
+    if (tid == 0) {
+      *cnt_out = nA;
+      if (cnt_out2) *cnt_out2 = nK - nA;
+    }
     return;
   }
   int NB2 = 1;
@@ -203,7 +230,7 @@ __global__ void __launch_bounds__(kSelThreads) block_select_kernel(
       acc[u] = 0.f;
       const int j = j0 + u;
       if (j < nK) {
-        const float* k = kb + ((long long)j * H + h) * D;
+        const float* k = j < nA ? kbA + ((long long)j * H + h) * D : kbB + ((long long)(j - nA) * H + h) * D;
 #pragma unroll
         for (int c = lane; c < D; c += 32) acc[u] = fmaf(qv[c], __ldg(k + c), acc[u]);
       }
@@ -291,40 +318,50 @@ __global__ void __launch_bounds__(kSelThreads) block_select_kernel(
   const int kstar = s_kstar;
   for (int x = tid; x < kstar; x += kSelThreads) flag[id[x]] = 1;
   __syncthreads();
-  // ordered compaction of the kept ids
-  int cnt = 0;
-  for (int x = b0; x < b1; ++x) cnt += flag[x];
-  int total_kept;
+  // ordered compaction of the kept ids (ids >= nA into the second list, minus nA)
+  int cnt = 0, cnt2 = 0;
+  for (int x = b0; x < b1; ++x) {
+    if (x < nA) cnt += flag[x];
+    else cnt2 += flag[x];
+  }
+  int total_kept, total_kept2;
   int pos = block_excl_scan<int>(cnt, ired, &total_kept);
-  for (int x = b0; x < b1; ++x)
-    if (flag[x]) idx_out[pos++] = x;
-  if (tid == 0) *cnt_out = kstar;
+  int pos2 = block_excl_scan<int>(cnt2, ired, &total_kept2);
+  for (int x = b0; x < b1; ++x) {
+    if (!flag[x]) continue;
+    if (x < nA) idx_out[pos++] = x;
+    else idx_out2[pos2++] = x - nA;
+  }
+  if (tid == 0) {
+    *cnt_out = total_kept;
+    if (cnt_out2) *cnt_out2 = total_kept2;
+  }
 }
 
 cudaError_t launch_block_select(const float* q128, const float* kc128, const float* q64, const float* kq64,
-                                const float* tau, int H, int d, int Lq, long long Lc, float scale,
+                                const float* tau, int H, int d, int Lq, long long Lc, float scale, bool joint,
                                 int32_t* inter_idx, int32_t* inter_cnt, int32_t* intra_idx, int32_t* intra_cnt,
                                 cudaStream_t s) {
   const int nQ128 = (Lq + 127) / 128, nQ64 = (Lq + 63) / 64;
   const int nKc = (int)((Lc + 127) / 128), nKq = nQ64;
-  int nmax = nKc > nKq ? nKc : nKq, NB2 = 1;
+  int nmax = joint ? nKc + nKq : (nKc > nKq ? nKc : nKq), NB2 = 1;
   while (NB2 < nmax) NB2 <<= 1;
   const size_t smem = (size_t)NB2 * 12;
-  const int grid = H * (nQ128 + nQ64);
+  const int grid = joint ? H * nQ64 : H * (nQ128 + nQ64);
   if (d == 128) {
     if (smem > 48 * 1024) {
       cudaError_t e = cudaFuncSetAttribute(block_select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
     }
     block_select_kernel<128><<<grid, kSelThreads, smem, s>>>(q128, kc128, q64, kq64, tau, H, nQ128, nKc, nQ64, nKq,
-                                                              scale, inter_idx, inter_cnt, intra_idx, intra_cnt);
+                                                              scale, joint, inter_idx, inter_cnt, intra_idx, intra_cnt);
   } else {
     if (smem > 48 * 1024) {
       cudaError_t e = cudaFuncSetAttribute(block_select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
     }
     block_select_kernel<64><<<grid, kSelThreads, smem, s>>>(q128, kc128, q64, kq64, tau, H, nQ128, nKc, nQ64, nKq,
-                                                             scale, inter_idx, inter_cnt, intra_idx, intra_cnt);
+                                                             scale, joint, inter_idx, inter_cnt, intra_idx, intra_cnt);
   }
   return cudaGetLastError();
 }

@@ -11,8 +11,9 @@ from __future__ import annotations
 
 import torch
 
-from . import (SelectionBuffers, hkv_gather, hkv_page_summary, hkv_select_pages, hkv_select_prompt,
-               hsa_forward, hsa_forward_reuse, hsa_prepare_history, hsa_workspace_size, make_config)
+from . import (SelectionBuffers, hkv_block_means_from_pages, hkv_gather, hkv_page_block_sums, hkv_page_summary,
+               hkv_select_pages, hkv_select_prompt, hsa_block_select, hsa_forward, hsa_forward_reuse,
+               hsa_forward_selected, hsa_prepare_history, hsa_workspace_size, make_config)
 
 
 def page_pointers(pages: torch.Tensor) -> torch.Tensor:
@@ -47,11 +48,21 @@ class HkvHsaStep:
         self.selection = SelectionBuffers.empty(self.cfg, dev)
         self.ws = torch.zeros(hsa_workspace_size(self.cfg, NP, P_tok), dtype=torch.uint8, device=dev)
         self.out = torch.empty(Lq, H, d, dtype=out_dtype, device=dev)
+        # Pages of a multiple of 64 rows keep their 64-row key sums (from the seal): the
+        # block selection then runs from them while the gather copies, on its own stream.
+        self.early = P_tok % 64 == 0
+        self.sums64 = torch.zeros(NP, P_tok // 64, H, d, dtype=torch.float32, device=dev) if self.early else None
+        self.gather_stream = torch.cuda.Stream(device=dev) if self.early else None
+        self.ev_sel = torch.cuda.Event()
+        self.ev_gathered = torch.cuda.Event()
 
-    def seal_pages(self, pages_k: torch.Tensor):
-        """Page summaries (mean key per head) of every page, computed once."""
+    def seal_pages(self, pages_k):
+        """Page summaries (mean key per head) and, when kept, 64-row key sums of every
+        page, computed once.  pages_k: [NP, P_tok, H, d] tensor or a list of pages."""
         for p in range(self.NP):
             hkv_page_summary(pages_k[p], self.kbar_pages[p], self.ws)
+            if self.early:
+                hkv_page_block_sums(pages_k[p], self.sums64[p])
 
     def _retrieve(self, Q, cand):
         """Page-level retrieval into self.sel (self.scores: the page scores)."""
@@ -70,10 +81,25 @@ class HkvHsaStep:
         self._retrieve(Q, cand)
         if self.store is not None:
             self.store.fetch(self.sel, self.ws)
+        if not self.early:
+            hkv_gather(self.page_k_ptrs, self.page_v_ptrs, self.sel, self.Kp, self.P_tok, self.H, self.d,
+                       self.Kc, self.Vc, self.ws, self.kbar128)
+            hsa_forward(self.cfg, Q, self.Kc, self.Vc, Kq, Vq, tau, gate_logit, E, F, dst, self.ws,
+                        self.kbar128, self.selection, ef_head_stride)
+            return dst
+        # the cache's block means from the pages' sums, then the gather on its own stream
+        # while this stream pools the chunk and selects blocks
+        main = torch.cuda.current_stream()
+        hkv_block_means_from_pages(self.sums64, self.sel, self.Kp, self.P_tok, self.H, self.d, self.kbar128, self.ws)
+        self.ev_sel.record(main)
+        self.gather_stream.wait_event(self.ev_sel)
         hkv_gather(self.page_k_ptrs, self.page_v_ptrs, self.sel, self.Kp, self.P_tok, self.H, self.d,
-                   self.Kc, self.Vc, self.ws, self.kbar128)
-        hsa_forward(self.cfg, Q, self.Kc, self.Vc, Kq, Vq, tau, gate_logit, E, F, dst, self.ws,
-                    self.kbar128, self.selection, ef_head_stride)
+                   self.Kc, self.Vc, self.ws, None, stream=self.gather_stream)
+        self.ev_gathered.record(self.gather_stream)
+        hsa_block_select(self.cfg, Q, self.Kc, Kq, tau, self.selection, self.ws, self.kbar128)
+        main.wait_event(self.ev_gathered)
+        hsa_forward_selected(self.cfg, Q, self.Kc, self.Vc, Kq, Vq, gate_logit, E, F, self.selection, dst, self.ws,
+                             ef_head_stride)
         return dst
 
     # ------------------------------------------------------------ multi-step reuse

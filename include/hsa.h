@@ -83,15 +83,30 @@ typedef struct {
   int block_intra;   /* must be 64 */
   int rank;          /* Linformer r */
   float scale;       /* softmax scale; 0 means 1/sqrt(d) */
+  int select_mode;   /* HSA_SELECT_SEPARATE (0) or HSA_SELECT_JOINT (1), see below */
 } hsa_config_t;
+
+/* Block-selection modes ([NEWS] HSA paragraph; the pages do not say whether the
+ * cached-KV and in-chunk block masses share one softmax):
+ *   HSA_SELECT_SEPARATE  the inter map (128-row query blocks x 128-row Kc blocks)
+ *                        and the intra map (64-row query blocks x 64-row Kq blocks)
+ *                        are softmaxed and thresholded separately (default);
+ *   HSA_SELECT_JOINT     per 64-row query block, its mean query against both the
+ *                        Kc 128-row block means and the Kq 64-row block means, one
+ *                        softmax and one tau_h threshold over the union; the kept
+ *                        Kc blocks then form an inter list per 64-row query block
+ *                        (inter_idx [H][nQ64][nKc], inter_cnt [H][nQ64]). */
+#define HSA_SELECT_SEPARATE 0
+#define HSA_SELECT_JOINT 1
 
 /* Per-head block selections (device buffers, written by hsa_block_select).
  * nQ128 = ceil(Lq/128), nKc = ceil(Lc/128), nQ64 = ceil(Lq/64), nKq = ceil(Lq/64).
  * Row (h, i) of inter_idx holds inter_cnt[h*nQ128+i] ascending block ids of Kc,
- * the rest of the row is unspecified; likewise for intra. */
+ * the rest of the row is unspecified; likewise for intra.  In HSA_SELECT_JOINT
+ * mode the inter rows are per 64-row query block (nQ64 rows per head). */
 typedef struct {
-  int32_t* inter_idx;   /* [H][nQ128][nKc] */
-  int32_t* inter_cnt;   /* [H][nQ128]      */
+  int32_t* inter_idx;   /* [H][nQ128][nKc] (joint: [H][nQ64][nKc]) */
+  int32_t* inter_cnt;   /* [H][nQ128]      (joint: [H][nQ64])      */
   int32_t* intra_idx;   /* [H][nQ64][nKq]  */
   int32_t* intra_cnt;   /* [H][nQ64]       */
 } hsa_selection_t;
@@ -136,6 +151,25 @@ hsa_status_t hsa_thread_release(void);
  * Deterministic (fixed reduction order).  Uses the workspace. */
 hsa_status_t hkv_page_summary(const hsa_bf16* K_page, int P_tok, int H, int d, float* kbar,
                               void* ws, size_t ws_bytes, hsa_stream_t stream);
+
+/* 64-row key sums of a page, computed once when it is sealed (reading: the block
+ * pooling of the cached KV in [NEWS] HSA paragraph, Binter = 128, can then be done
+ * from the page store before the active cache is gathered):
+ *   sums64[b * H*d + c] = sum over rows [64 b, min(64 b + 64, P_tok)) of K_page[row, c]
+ * K_page: [P_tok, H, d] bf16 (device or mapped pinned host); sums64: fp32
+ * [ceil(P_tok/64), H, d].  Fixed order. */
+hsa_status_t hkv_page_block_sums(const hsa_bf16* K_page, int P_tok, int H, int d, float* sums64, hsa_stream_t stream);
+
+/* The 128-row key block means of the active cache that the pages sel[0..Kp) would
+ * gather to, from their 64-row sums (sums64_pages: [NP, P_tok/64, H, d] fp32, from
+ * hkv_page_block_sums), without the gathered copy:
+ *   kbar128[j] = (sum of the two 64-row halves of rows [128 j, 128 j + 128)) / rows
+ * P_tok must be a multiple of 64 (each half then lies in one page), else
+ * HSA_ERR_UNSUPPORTED.  Pass kbar128 to hsa_block_select while hkv_gather copies.
+ * An out-of-range page id sets HSA_ERR_DEVICE.  Uses the workspace (status). */
+hsa_status_t hkv_block_means_from_pages(const float* sums64_pages, int NP, const int32_t* sel, int Kp, int P_tok,
+                                        int H, int d, float* kbar128, void* ws, size_t ws_bytes,
+                                        hsa_stream_t stream);
 
 /* Stage 1, prompt-level retrieval ([NEWS] HKV and open-questions paragraphs:
  * Top-1): s* = argmax_s cos(e_cur, e_seg[s]) (ties -> lowest s); then
@@ -387,6 +421,16 @@ hsa_status_t hsa_forward(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_b
                          const hsa_bf16* E, const hsa_bf16* F, long long ef_head_stride,
                          void* out, int out_is_bf16, const hsa_selection_t* sel_out,
                          void* ws, size_t ws_bytes, hsa_stream_t stream);
+
+/* hsa_forward with the block selection already made (sel, input: from
+ * hsa_block_select): the Linformer branch, the sparse branch and the gated merge.
+ * Lets a caller select blocks while the active cache is still being gathered
+ * (kbar128 from hkv_block_means_from_pages), then run the rest once it is. */
+hsa_status_t hsa_forward_selected(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc,
+                                  const hsa_bf16* Vc, const hsa_bf16* Kq, const hsa_bf16* Vq,
+                                  const float* gate_logit, const hsa_bf16* E, const hsa_bf16* F,
+                                  long long ef_head_stride, const hsa_selection_t* sel, void* out,
+                                  int out_is_bf16, void* ws, size_t ws_bytes, hsa_stream_t stream);
 
 /* Multi-step reuse ([NEWS] HKV paragraph: retrieval assembles the active cache of
  * the current chunk; kernel paragraph: KV reorganisation and copies dominate the

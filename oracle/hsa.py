@@ -196,14 +196,31 @@ class Selection:
     p_intra: np.ndarray  # [H, nQ64, nKq64]
 
 
-def block_select(Q, Kc, Kq, tau, scale=None, Binter=128, Bintra=64, dtype=np.float32) -> Selection:
+def block_select(Q, Kc, Kq, tau, scale=None, Binter=128, Bintra=64, dtype=np.float32, joint=False) -> Selection:
     """Head-adaptive block selection ([NEWS] HSA paragraph).
 
     Inter map: 128-row query blocks against 128-row blocks of the cached KV Kc.
     Intra map: 64-row query blocks against 64-row blocks of the chunk's own keys Kq.
-    Each map row is softmaxed and thresholded at tau_h separately."""
+    Each map row is softmaxed and thresholded at tau_h separately.
+
+    joint=True (the other reading of the pages): per 64-row query block, its mean
+    query scored against the Kc blocks followed by the Kq blocks, one softmax and one
+    threshold over that whole row; the kept ids below nKc form the row's inter list,
+    the others (minus nKc) its intra list.  p_inter then holds the joint masses
+    [H, nQ64, nKc + nKq] and p_intra is None."""
     H, d = Q.shape[1], Q.shape[2]
     scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if joint:
+        q64 = block_means(Q, Bintra, dtype)
+        kc, kq = block_means(Kc, Binter, dtype), block_means(Kq, Bintra, dtype)
+        nKc = kc.shape[0]
+        p = block_probs(q64, np.concatenate([kc, kq], axis=0), scale, dtype)
+        inter, intra = [], []
+        for h in range(H):
+            kept = [keep_blocks(p[h, i], float(tau[h])) for i in range(p.shape[1])]
+            inter.append([k[k < nKc].astype(np.int32) for k in kept])
+            intra.append([(k[k >= nKc] - nKc).astype(np.int32) for k in kept])
+        return Selection(inter, intra, p, None)
     p_inter = block_probs(block_means(Q, Binter, dtype), block_means(Kc, Binter, dtype), scale, dtype)
     p_intra = block_probs(block_means(Q, Bintra, dtype), block_means(Kq, Bintra, dtype), scale, dtype)
     inter = [[keep_blocks(p_inter[h, i], float(tau[h])) for i in range(p_inter.shape[1])] for h in range(H)]
@@ -217,21 +234,25 @@ def _block_rows(blocks, B, n) -> np.ndarray:
     return np.concatenate([np.arange(j * B, min((j + 1) * B, n)) for j in blocks]).astype(np.int64)
 
 
-def sparse_attention(Q, Kc, Vc, Kq, Vq, inter, intra, scale=None, Binter=128, Bintra=64, rows=None):
+def sparse_attention(Q, Kc, Vc, Kq, Vq, inter, intra, scale=None, Binter=128, Bintra=64, rows=None,
+                     inter_rows=None):
     """Exact attention over the selected blocks only ([NEWS] HSA paragraph).
 
-    For query t of head h the key set is the tokens of Kc blocks inter[h][t // Binter]
+    For query t of head h the key set is the tokens of Kc blocks inter[h][t // inter_rows]
     together with the tokens of Kq blocks intra[h][t // Bintra]; one softmax over
     that whole set:  o[t, h] = sum_k softmax_k(q_t . k * scale) v_k.
+    inter_rows = the query rows an inter list serves: Binter (default), or Bintra for
+    the joint selection's per-64-row inter lists.
     ``rows`` (optional) = query rows to compute; returns [len(rows), H, d] float64."""
     Lq, H, d = Q.shape
     Lc, Lk = Kc.shape[0], Kq.shape[0]
     scale = 1.0 / math.sqrt(d) if scale is None else scale
+    inter_rows = Binter if inter_rows is None else inter_rows
     rows = np.arange(Lq) if rows is None else np.asarray(rows)
     out = np.zeros((len(rows), H, d), dtype=np.float64)
     groups = {}
     for n, t in enumerate(rows):
-        groups.setdefault((int(t) // Binter, int(t) // Bintra), []).append(n)
+        groups.setdefault((int(t) // inter_rows, int(t) // Bintra), []).append(n)
     for h in range(H):
         for (i128, i64), ns in groups.items():
             kc = _block_rows(inter[h][i128], Binter, Lc)
@@ -335,12 +356,14 @@ def gated_merge(o_s, o_l, z) -> np.ndarray:
 
 
 def hsa_step(Q, Kc, Vc, Kq, Vq, tau, z, E, F, scale=None, Binter=128, Bintra=64,
-             rows=None, selection=None, dtype=np.float32):
+             rows=None, selection=None, dtype=np.float32, joint=False):
     """HSA over the active cache plus the current chunk ([PROJ] overall architecture):
     block selection, sparse branch, linear branch, gated merge.  ``selection`` may be
-    passed in (e.g. a GPU selection already verified against this oracle)."""
-    sel = block_select(Q, Kc, Kq, tau, scale, Binter, Bintra, dtype) if selection is None else selection
-    o_s = sparse_attention(Q, Kc, Vc, Kq, Vq, sel.inter, sel.intra, scale, Binter, Bintra, rows)
+    passed in (e.g. a GPU selection already verified against this oracle); joint =
+    the joint block selection (inter lists per 64-row query block)."""
+    sel = block_select(Q, Kc, Kq, tau, scale, Binter, Bintra, dtype, joint) if selection is None else selection
+    o_s = sparse_attention(Q, Kc, Vc, Kq, Vq, sel.inter, sel.intra, scale, Binter, Bintra, rows,
+                           inter_rows=Bintra if joint else Binter)
     EK, FV = linear_projection(E, F, Kc, Kq, Vc, Vq)
     o_l = linear_attention(Q, EK, FV, scale, rows)
     return {"selection": sel, "o_s": o_s, "o_l": o_l, "out": gated_merge(o_s, o_l, z), "EK": EK, "FV": FV}

@@ -86,10 +86,7 @@ class DeviceStep:
         self.step = HkvHsaStep(H, d, shape.Lq, P, NP, shape.Kp, shape.r, kp, vp, out_dtype, store=self.store)
         if self.host:
             # summaries read the mapped host pages directly
-            from hybrid_sparse_attention_hkv_b200 import hkv_page_summary
-            for p in range(NP):
-                t = _HostPageView(self.host[0].dev_ptr + p * stride, P, H, d)
-                hkv_page_summary(t, self.step.kbar_pages[p], self.step.ws)
+            self.step.seal_pages([_HostPageView(self.host[0].dev_ptr + p * stride, P, H, d) for p in range(NP)])
         else:
             self.step.seal_pages(self.pages_k)
         self.e_cur = self.e_seg = self.seg_begin = None

@@ -543,3 +543,53 @@ def test_fidelity_report_matches_the_oracle(small):
     s = torch.einsum("thc,khc->htk", torch.from_numpy(oracle.widen(x.Q)), K) / math.sqrt(shape.d)
     want = torch.logsumexp(s, dim=2).T.numpy()
     np.testing.assert_allclose(lse.cpu().numpy(), want, atol=2e-3)
+
+
+def test_block_means_from_page_sums():
+    """64-row key sums kept per page give the active cache's 128-row block means without
+    the gathered copy: equal to the oracle's block means of the gathered cache."""
+    shape = SMALL[2]  # pages of 384 rows
+    ds = DeviceStep(shape, 19)
+    x, st = ds.x, ds.step
+    assert st.early
+    ds.run()
+    torch.cuda.synchronize()
+    for p in range(shape.NP):
+        want = oracle.block_means(x.pages_k[p], 64) * 64
+        np.testing.assert_allclose(st.sums64[p].cpu().numpy(), want, rtol=1e-5, atol=1e-4)
+    Kc = oracle.gather_pages(x.pages_k, st.sel.cpu().numpy())
+    np.testing.assert_allclose(st.kbar128.cpu().numpy(), oracle.block_means(Kc, 128), rtol=1e-5, atol=1e-6)
+    assert np.array_equal(bits_of(st.Kc), Kc)
+    assert hsa.hsa_status_read(st.ws) == 0
+
+
+# ----------------------------------------------------------------- joint block selection
+
+def test_joint_selection_and_output(small):
+    """HSA_SELECT_JOINT: one softmax per 64-row query block over its cached and chunk
+    blocks.  The GPU's kept blocks (inter and intra together) equal the oracle's, with
+    the same exemptions, and the output equals the oracle's HSA step on that selection
+    (inter lists per 64-row query block)."""
+    x, st, shape = small.x, small.step, small.shape
+    cfg = make_config(shape.H, shape.d, shape.Lq, shape.Lc, shape.r, select_mode=hsa.SELECT_JOINT)
+    sel = SelectionBuffers.empty(cfg)
+    out = torch.empty_like(st.out)
+    hsa.hsa_forward(cfg, small.Q, st.Kc, st.Vc, small.Kq, small.Vq, small.tau, small.z, small.E, small.F, out, st.ws,
+                    st.kbar128, sel=sel)
+    torch.cuda.synchronize()
+    assert hsa.hsa_status_read(st.ws) == 0
+    Kc, Vc = bits_of(st.Kc), bits_of(st.Vc)
+    nKc = -(-shape.Lc // 128)
+    gi = selection_lists(sel.inter_idx.cpu().numpy(), sel.inter_cnt.cpu().numpy())
+    gq = selection_lists(sel.intra_idx.cpu().numpy(), sel.intra_cnt.cpu().numpy())
+    assert len(gi[0]) == -(-shape.Lq // 64)
+    combined = [[np.concatenate([gi[h][i], gq[h][i] + nKc]) for i in range(len(gi[h]))] for h in range(shape.H)]
+    for dt in (np.float32, np.float64):
+        ref = oracle.block_select(x.Q, Kc, x.Kq, x.tau, dtype=dt, joint=True)
+        ref_c = [[np.concatenate([ref.inter[h][i], ref.intra[h][i] + nKc]) for i in range(len(ref.inter[h]))]
+                 for h in range(shape.H)]
+        n, e = check_selection(combined, ref_c, ref.p_inter, x.tau, f"joint {dt.__name__}")
+        assert e <= max(1, n // 100)
+    res = oracle.hsa_step(x.Q, Kc, Vc, x.Kq, x.Vq, x.tau, x.z, x.E, x.F, joint=True,
+                          selection=oracle.Selection(gi, gq, None, None))
+    assert_close(out.cpu().numpy(), res["out"], "joint selection output")

@@ -527,3 +527,48 @@ def test_fidelity_closed_forms():
             m.append(np.exp(logsumexp(s[t, kept]) - logsumexp(s[t])))
         assert abs(rep[h, 2] - np.mean(m)) < 1e-12
         assert 0 < rep[h, 2] < 1 and rep[h, 1] < 1 and rep[h, 4] > 0
+
+
+def test_block_select_joint_golden(golden_dir):
+    """The joint selection (one softmax per 64-row query block over the cached and the
+    chunk blocks) against hand-derived lists, some of them empty, on the separate
+    mode's fixture; the lists are also the minimum-cardinality subsets found by
+    enumeration over the joint masses computed here with numpy."""
+    g = load(golden_dir, "block_select.json")
+    Q = bf16(np.repeat(np.asarray(g["Q64_blocks"], np.float32).transpose(1, 0, 2), 64, axis=0))
+    Kc = bf16(np.repeat(np.asarray(g["Kc128_blocks"], np.float32).transpose(1, 0, 2), 128, axis=0))
+    Kq = bf16(np.repeat(np.asarray(g["Kq64_blocks"], np.float32).transpose(1, 0, 2), 64, axis=0))
+    tau = np.asarray(g["tau"], dtype=np.float32)
+    sel = oracle.block_select(Q, Kc, Kq, tau, scale=math.log(2.0), dtype=np.float64, joint=True)
+    assert [[r.tolist() for r in h] for h in sel.inter] == g["joint"]["keep_inter"]
+    assert [[r.tolist() for r in h] for h in sel.intra] == g["joint"]["keep_intra"]
+    q64 = np.asarray(g["Q64_blocks"], np.float64)
+    keys = np.concatenate([np.asarray(g["Kc128_blocks"], np.float64), np.asarray(g["Kq64_blocks"], np.float64)], axis=1)
+    for h in range(2):
+        for i in range(4):
+            w = 2.0 ** (keys[h] @ q64[h, i])
+            p = w / w.sum()
+            kept = g["joint"]["keep_inter"][h][i] + [4 + j for j in g["joint"]["keep_intra"][h][i]]
+            assert p[kept].sum() >= tau[h]
+            smaller = [sum(p[list(c)]) for c in itertools.combinations(range(8), len(kept) - 1)] if len(kept) > 1 else []
+            assert all(m < tau[h] for m in smaller)  # no fewer blocks reach tau
+
+
+def test_sparse_attention_joint_rows_use_64_row_inter_lists():
+    """With inter_rows = 64 each 64-row query block uses its own inter list: equal to
+    masked dense attention with the per-64-row key sets."""
+    H, d, Lq, Lc = 1, 8, 128, 256
+    Q, Kc, Vc = rand_bf16((Lq, H, d), 41, 1), rand_bf16((Lc, H, d), 41, 2), rand_bf16((Lc, H, d), 41, 3)
+    Kq, Vq = rand_bf16((Lq, H, d), 41, 4), rand_bf16((Lq, H, d), 41, 5)
+    inter = [[np.array([0]), np.array([1])]]
+    intra = [[np.array([1]), np.array([0])]]
+    got = oracle.sparse_attention(Q, Kc, Vc, Kq, Vq, inter, intra, inter_rows=64)
+    K = np.concatenate([oracle.widen(Kc), oracle.widen(Kq)])
+    V = np.concatenate([oracle.widen(Vc), oracle.widen(Vq)])
+    mask = np.full((1, Lq, Lc + Lq), -np.inf)
+    mask[0, :64, 0:128] = 0
+    mask[0, :64, Lc + 64:Lc + 128] = 0
+    mask[0, 64:, 128:256] = 0
+    mask[0, 64:, Lc:Lc + 64] = 0
+    want = sdpa(oracle.widen(Q), K, V, 1 / math.sqrt(d), mask)
+    np.testing.assert_allclose(got, want, rtol=1e-10, atol=1e-12)
