@@ -79,6 +79,8 @@ def step_work(shape):
     L = Lc + Lq
     return {
         "proj_flops": H * 4.0 * r * L * d,             # EK and FV: 2 * (2 r L d) per head
+        "proj_chunk_flops": H * 4.0 * r * Lq * d,      # the chunk's own rows only (history prepared)
+        "proj_hist_flops": H * 4.0 * r * Lc * d,       # the cached rows only
         "lin_attn_flops": H * 4.0 * Lq * r * d,        # Q EK^T and P FV
         "gather_bytes": 4.0 * Lc * H * d * 2,          # read + write of K and V pages
         "proj_bytes": 2.0 * L * H * d * 2 + 2.0 * r * L * 2,
@@ -536,11 +538,15 @@ def run_gpu(args, shape, rank, world, local):
     t_kind = "burst" if at_max else "sustained"
     t_peak = peaks["bf16_tflops"] if at_max else peaks["bf16_tflops_sustained"]
     host_gbs = measure_host_link(dev) if shape.host_pages else None
+    # pages of a multiple of 64 rows: the step gathers and projects the history in one
+    # pass (gather_project) and the step's own projection covers the chunk's rows only
+    early = shape.P_tok % 64 == 0
     kernel_work = {
         # the fused attention kernel: selected-block FLOPs of the sparse branch plus the
         # useful FLOPs of the linear branch (the split-precision extra products not counted)
         "attention_merge": ("tensor", f_sparse + w["lin_attn_flops"]),
-        "linformer_proj": ("tensor", w["proj_flops"]),
+        "linformer_proj": ("tensor", w["proj_chunk_flops"] if early else w["proj_flops"]),
+        "gather_project": ("tensor", w["proj_hist_flops"]),
         "gather": ("host-link", w["gather_bytes"] / 2) if shape.host_pages else ("hbm", w["gather_bytes"]),
         "pool": ("hbm", w["pool_bytes"]),
         "page_scores_partial": ("hbm", w["select_pages_bytes"]),
@@ -550,6 +556,10 @@ def run_gpu(args, shape, rank, world, local):
         avg_ms = d["ms"] / d["launches"]
         entry = {"launches_per_step": d["launches"] / args.steps, "ms_per_launch": avg_ms,
                  "share": d["ms"] / sum(v["ms"] for v in per_kernel.values())}
+        if name == "gather_project":  # also its bytes: the pages read once, Kc / Vc written, E / F read
+            gp_bytes = w["gather_bytes"] + 2.0 * shape.r * shape.Lc * 2
+            entry["hbm_GBps"] = gp_bytes / (avg_ms / 1e3) / 1e9
+            entry["hbm_frac"] = entry["hbm_GBps"] / peaks["hbm_gbs"]
         if name in kernel_work:
             bound, work = kernel_work[name]
             if bound == "tensor":

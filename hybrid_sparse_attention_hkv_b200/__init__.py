@@ -29,8 +29,10 @@ EXPORTED = [
     "hkv_store_state_size", "hkv_store_init", "hkv_store_tables", "hkv_store_seal", "hkv_store_fetch",
     "hkv_store_prefetch", "hkv_store_residency", "hkv_select_pages_policy", "hkv_page_scores", "hkv_select_top",
     "hsa_sparse_attn_lse", "hsa_fidelity", "hkv_page_block_sums", "hkv_block_means_from_pages",
-    "hsa_forward_selected",
+    "hsa_forward_selected", "hsa_forward_ex", "hkv_gather_project",
 ]
+
+FWD_SELECTED, FWD_HISTORY = 1, 2
 
 POLICY_SCORE, POLICY_RECENT, POLICY_RANDOM = 0, 1, 2
 
@@ -102,6 +104,9 @@ def load_library(path: str = LIB_PATH):
         "hkv_page_block_sums": (I, [P, I, I, I, P, P]),
         "hkv_block_means_from_pages": (I, [P, I, P, I, I, I, I, P, P, S, P]),
         "hsa_forward_selected": (I, [CP, P, P, P, P, P, P, P, P, L, ctypes.POINTER(_Selection), P, I, P, S, P]),
+        "hsa_forward_ex": (I, [CP, P, P, P, P, P, P, P, P, P, P, L, P, I, ctypes.POINTER(_Selection), ctypes.c_uint,
+                               P, S, P]),
+        "hkv_gather_project": (I, [CP, P, P, I, P, I, I, P, P, L, P, P, P, S, P]),
         "hsa_fidelity": (I, [CP, P, P, P, P, P, P, P, S, P]),
         "hkv_select_top": (I, [P, I, P, I, P, P, S, P]),
         "hkv_store_state_size": (S, [I, I]),
@@ -342,6 +347,24 @@ def hsa_forward_selected(cfg, Q, Kc, Vc, Kq, Vq, gate_logit, E, F, sel: Selectio
                                                _p(gate_logit), _p(E), _p(F), ef_head_stride, ctypes.byref(sel.c()),
                                                _p(out), 1 if out.dtype == torch.bfloat16 else 0, _p(ws), ws.numel(),
                                                _stream(stream)), "hsa_forward_selected")
+
+
+def hsa_forward_ex(cfg, Q, Kc, Vc, Kq, Vq, tau, gate_logit, E, F, out, ws, sel: SelectionBuffers, flags=0,
+                   kbar128=None, ef_head_stride=0, stream=None):
+    """hsa_forward with FWD_SELECTED (sel is an input) and/or FWD_HISTORY (prepared history)."""
+    _check(load_library().hsa_forward_ex(ctypes.byref(cfg), _p(Q), _p(Kc), _p(Vc), _p(Kq), _p(Vq), _p(kbar128),
+                                         _p(tau), _p(gate_logit), _p(E), _p(F), ef_head_stride, _p(out),
+                                         1 if out.dtype == torch.bfloat16 else 0, ctypes.byref(sel.c()), flags, _p(ws),
+                                         ws.numel(), _stream(stream)), "hsa_forward_ex")
+
+
+def hkv_gather_project(cfg, page_k_ptrs, page_v_ptrs, sel, Kp, P_tok, E, F, Kc, Vc, ws, ef_head_stride=0,
+                       stream=None):
+    """Gather of the selected pages + the history's Linformer products, one pass."""
+    NP = page_k_ptrs.numel()
+    _check(load_library().hkv_gather_project(ctypes.byref(cfg), _p(page_k_ptrs), _p(page_v_ptrs), NP, _p(sel), Kp,
+                                             P_tok, _p(E), _p(F), ef_head_stride, _p(Kc), _p(Vc), _p(ws), ws.numel(),
+                                             _stream(stream)), "hkv_gather_project")
 
 
 def hsa_prepare_history(cfg, Kc, Vc, E, F, ws, ef_head_stride=0, stream=None):

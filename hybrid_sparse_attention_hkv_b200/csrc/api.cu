@@ -79,7 +79,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 struct Layout {
   size_t status = 0, colpart = 0, q128 = 0, q64 = 0, kq64 = 0, kc128 = 0;
   size_t inter_idx = 0, inter_cnt = 0, intra_idx = 0, intra_cnt = 0;
-  size_t units = 0, n_units = 0, tile_done = 0, part_o = 0, part_ml = 0, part_lin = 0, attn_end = 0;
+  size_t units = 0, n_units = 0, tile_done = 0, part_o = 0, part_ml = 0, lin_buf = 0, attn_end = 0;
   int max_units = 0, max_slots = 0;
   size_t ekhi = 0, eklo = 0, fvhi = 0, fvlo = 0, projpart = 0, ekfv_hist = 0;
   size_t pages_end = 0;  // bytes needed by the page (HKV) calls
@@ -115,7 +115,7 @@ Layout make_layout(int H, int d, int Lq, long long Lc, int r) {
   L.tile_done = take((size_t)H * nQ128 * 4);
   L.part_o = take((size_t)L.max_slots * 128 * d * 4);
   L.part_ml = take((size_t)L.max_slots * 128 * 8);
-  L.part_lin = take((size_t)L.max_slots * 128 * d * 4);
+  L.lin_buf = take((size_t)Lq * H * d * 4);
   L.attn_end = off;
   const size_t hrd = (size_t)H * r * d;
   L.ekhi = take(hrd * 2);
@@ -614,6 +614,7 @@ static hsa::AttnArgs attn_args(const hsa_config_t* cfg, const Layout& L, void* w
   a.status = status_of(ws);
   a.max_units = L.max_units;
   a.max_slots = L.max_slots;
+  a.lin_buf = at<float>(ws, L.lin_buf);
   return a;
 }
 
@@ -626,7 +627,6 @@ static hsa_status_t run_plan(const Layout& L, const hsa_selection_t& sel, void* 
   a.tile_done = at<int>(ws, L.tile_done);
   a.part_o = at<float>(ws, L.part_o);
   a.part_ml = at<float2>(ws, L.part_ml);
-  a.part_lin = at<float>(ws, L.part_lin);
   HSA_LAUNCH("attn_plan", hsa::launch_attn_plan(a, stream));
   return HSA_OK;
 }
@@ -850,6 +850,60 @@ hsa_status_t hsa_prepare_history(const hsa_config_t* cfg, const hsa_bf16* Kc, co
   HSA_LAUNCH("linformer_proj_history",
              hsa::launch_proj_tc(E, F, ef_head_stride, Kc, Kq, Vc, Vq, cfg->H, cfg->d, cfg->rank, cfg->Lc, cfg->Lq,
                                  hsa::kProjCached, splits, part, status_of(ws), stream));
+  HSA_LAUNCH("linformer_reduce_history",
+             hsa::launch_proj_reduce(part, splits, cfg->H, cfg->d, cfg->rank, nullptr, at<float>(ws, L.ekfv_hist),
+                                     nullptr, nullptr, nullptr, nullptr, stream));
+  return HSA_OK;
+}
+
+hsa_status_t hsa_forward_ex(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc, const hsa_bf16* Vc,
+                            const hsa_bf16* Kq, const hsa_bf16* Vq, const float* kbar128, const float* tau,
+                            const float* gate_logit, const hsa_bf16* E, const hsa_bf16* F, long long ef_head_stride,
+                            void* out, int out_is_bf16, const hsa_selection_t* sel, unsigned flags, void* ws,
+                            size_t ws_bytes, hsa_stream_t stream) {
+  if (flags & ~(unsigned)(HSA_FWD_SELECTED | HSA_FWD_HISTORY))
+    return fail(HSA_ERR_INVALID_ARG, "hsa_forward_ex: unknown flags 0x%x", flags);
+  return forward_impl(__func__, cfg, Q, Kc, Vc, Kq, Vq, kbar128, tau, gate_logit, E, F, ef_head_stride, out,
+                      out_is_bf16, sel, ws, ws_bytes, (flags & HSA_FWD_HISTORY) ? hsa::kProjChunk : hsa::kProjAll,
+                      (flags & HSA_FWD_SELECTED) != 0, stream);
+}
+
+hsa_status_t hkv_gather_project(const hsa_config_t* cfg, const hsa_bf16* const* page_k, const hsa_bf16* const* page_v,
+                                int NP, const int32_t* sel, int Kp, int P_tok, const hsa_bf16* E, const hsa_bf16* F,
+                                long long ef_head_stride, hsa_bf16* Kc, hsa_bf16* Vc, void* ws, size_t ws_bytes,
+                                hsa_stream_t stream) {
+  const char* fn = __func__;
+  TRY(check_cfg(fn, cfg, true));
+  if (NP < 1 || P_tok < 1) return fail(HSA_ERR_INVALID_ARG, "%s: NP = %d, P_tok = %d must be >= 1", fn, NP, P_tok);
+  if (Kp < 1 || Kp > NP) return fail(HSA_ERR_INVALID_ARG, "%s: Kp = %d must be in [1, NP]", fn, Kp);
+  if (P_tok % 64 != 0) return fail(HSA_ERR_UNSUPPORTED, "%s: P_tok = %d is not a multiple of 64", fn, P_tok);
+  if ((long long)Kp * P_tok != cfg->Lc)
+    return fail(HSA_ERR_INVALID_ARG, "%s: Kp * P_tok = %lld differs from cfg->Lc = %d", fn, (long long)Kp * P_tok,
+                cfg->Lc);
+  if (!page_k || !page_v || !sel) return fail(HSA_ERR_INVALID_ARG, "%s: NULL page table or selection", fn);
+  REQUIRE_PTR(Kc);
+  REQUIRE_PTR(Vc);
+  REQUIRE_PTR(E);
+  REQUIRE_PTR(F);
+  if (ef_head_stride != 0 && ef_head_stride != (long long)cfg->rank * (cfg->Lc + cfg->Lq))
+    return fail(HSA_ERR_UNSUPPORTED, "%s: ef_head_stride must be 0 (shared) or r * (Lc + Lq) (stacked per head)", fn);
+  const Layout L = make_layout(cfg->H, cfg->d, cfg->Lq, cfg->Lc, cfg->rank);
+  TRY(check_ws(fn, ws, ws_bytes, L.total));
+  float* part = at<float>(ws, L.projpart);
+  int splits = hsa::proj_tc_splits(cfg->H, cfg->d, cfg->rank, cfg->Lc, cfg->Lq, hsa::kProjCached);
+  if (splits > L.splits) splits = L.splits;
+  hsa::ProjPages pg;
+  pg.page_k = reinterpret_cast<const uint16_t* const*>(page_k);
+  pg.page_v = reinterpret_cast<const uint16_t* const*>(page_v);
+  pg.sel = sel;
+  pg.NP = NP;
+  pg.P_tok = P_tok;
+  pg.Kc_out = Kc;
+  pg.Vc_out = Vc;
+  // the maps of Kc / Vc (and of the chunk tensors) are not read in this mode
+  HSA_LAUNCH("gather_project", hsa::launch_proj_tc(E, F, ef_head_stride, Kc, Kc, Vc, Vc, cfg->H, cfg->d, cfg->rank,
+                                                   cfg->Lc, cfg->Lq, hsa::kProjCached, splits, part, status_of(ws),
+                                                   stream, &pg));
   HSA_LAUNCH("linformer_reduce_history",
              hsa::launch_proj_reduce(part, splits, cfg->H, cfg->d, cfg->rank, nullptr, at<float>(ws, L.ekfv_hist),
                                      nullptr, nullptr, nullptr, nullptr, stream));

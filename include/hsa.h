@@ -432,6 +432,35 @@ hsa_status_t hsa_forward_selected(const hsa_config_t* cfg, const hsa_bf16* Q, co
                                   long long ef_head_stride, const hsa_selection_t* sel, void* out,
                                   int out_is_bf16, void* ws, size_t ws_bytes, hsa_stream_t stream);
 
+/* hsa_forward with options (flags, OR-ed):
+ *   HSA_FWD_SELECTED  sel is an input (the block selection already made); tau and
+ *                     kbar128 are not read
+ *   HSA_FWD_HISTORY   the cached KV's Linformer products are in the workspace
+ *                     (hsa_prepare_history or hkv_gather_project): only the chunk's
+ *                     own keys and values are projected, as hsa_forward_reuse
+ * flags = 0 is hsa_forward. */
+#define HSA_FWD_SELECTED 1u
+#define HSA_FWD_HISTORY 2u
+hsa_status_t hsa_forward_ex(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc, const hsa_bf16* Vc,
+                            const hsa_bf16* Kq, const hsa_bf16* Vq, const float* kbar128, const float* tau,
+                            const float* gate_logit, const hsa_bf16* E, const hsa_bf16* F, long long ef_head_stride,
+                            void* out, int out_is_bf16, const hsa_selection_t* sel, unsigned flags,
+                            void* ws, size_t ws_bytes, hsa_stream_t stream);
+
+/* The active-cache gather and the history's Linformer products in one pass over
+ * the selected pages ([NEWS] kernel paragraph: the KV copies dominate the
+ * preprocessing; the copy and the projection then read each cached row once):
+ *   Kc, Vc                as hkv_gather (bitwise copies of pages sel[0..Kp));
+ *   history products      as hsa_prepare_history (E_h[:, 0:Lc] Kc_h, F_h[:, 0:Lc] Vc_h,
+ *                         fp32 in the workspace), for hsa_forward_reuse /
+ *                         hsa_forward_ex(HSA_FWD_HISTORY).
+ * Requires P_tok a multiple of 64 and Kp * P_tok == cfg->Lc.  Page tables as
+ * hkv_gather; an out-of-range page id sets HSA_ERR_DEVICE.  Uses the workspace. */
+hsa_status_t hkv_gather_project(const hsa_config_t* cfg, const hsa_bf16* const* page_k, const hsa_bf16* const* page_v,
+                                int NP, const int32_t* sel, int Kp, int P_tok, const hsa_bf16* E, const hsa_bf16* F,
+                                long long ef_head_stride, hsa_bf16* Kc, hsa_bf16* Vc,
+                                void* ws, size_t ws_bytes, hsa_stream_t stream);
+
 /* Multi-step reuse ([NEWS] HKV paragraph: retrieval assembles the active cache of
  * the current chunk; kernel paragraph: KV reorganisation and copies dominate the
  * preprocessing; reading: a chunk is denoised over several steps against one

@@ -130,7 +130,10 @@ def test_branches_standalone(small):
     EK, FV = oracle.linear_projection(x.E, x.F, Kc, x.Kq, Vc, x.Vq)
     ref_l = oracle.linear_attention(x.Q, EK, FV)
     assert_close(o_l.cpu().numpy(), ref_l, "linear branch")
-    # the gates isolate each branch exactly (same kernels, g = 1 or 0 in the merge)
+    # the gates isolate each branch exactly (g = 1 or 0 in the merge).  With g = 0 the
+    # output is the linear branch bit for bit.  With g = 1 it is the sparse branch up
+    # to the order of fp32 sums: key tiles alternate between two softmax groups by
+    # their position in the unit's list, which the linear tiles ahead of them shift.
     H = small.shape.H
     for z, want in ((float("inf"), o_s), (float("-inf"), o_l)):
         zz = torch.full((H,), z, dtype=torch.float32, device="cuda")
@@ -138,7 +141,10 @@ def test_branches_standalone(small):
         hsa.hsa_forward(cfg, small.Q, st.Kc, st.Vc, small.Kq, small.Vq, small.tau, zz, small.E, small.F, out, st.ws,
                         st.kbar128)
         torch.cuda.synchronize()
-        assert torch.equal(out, want), z
+        if z < 0 or (small.shape.r // 64) % 2 == 0:
+            assert torch.equal(out, want), z
+        else:
+            assert float((out - want).abs().max()) <= 1e-5 * float(want.abs().max()), z
 
 
 def test_deterministic(small):
@@ -593,3 +599,27 @@ def test_joint_selection_and_output(small):
     res = oracle.hsa_step(x.Q, Kc, Vc, x.Kq, x.Vq, x.tau, x.z, x.E, x.F, joint=True,
                           selection=oracle.Selection(gi, gq, None, None))
     assert_close(out.cpu().numpy(), res["out"], "joint selection output")
+
+
+def test_gather_project_equals_gather_then_projection():
+    """One pass over the selected pages: the same Kc / Vc bits as hkv_gather, and
+    denoising steps on its history products equal to hsa_forward on the full KV."""
+    shape = SMALL[2]  # pages of 384 rows (a multiple of 64)
+    ds = DeviceStep(shape, 23)
+    x, st = ds.x, ds.step
+    hsa.hkv_select_pages(st.kbar_pages, ds.Q, shape.Kp, st.sel, st.ws, st.scores)
+    hsa.hkv_gather_project(st.cfg, st.page_k_ptrs, st.page_v_ptrs, st.sel, shape.Kp, shape.P_tok, ds.E, ds.F,
+                           st.Kc, st.Vc, st.ws)
+    torch.cuda.synchronize()
+    sel = st.sel.cpu().numpy()
+    assert np.array_equal(bits_of(st.Kc), oracle.gather_pages(x.pages_k, sel))
+    assert np.array_equal(bits_of(st.Vc), oracle.gather_pages(x.pages_v, sel))
+    out_r = torch.empty_like(st.out)
+    hsa.hsa_forward_reuse(st.cfg, ds.Q, st.Kc, st.Vc, ds.Kq, ds.Vq, ds.tau, ds.z, ds.E, ds.F, out_r, st.ws,
+                          sel=st.selection)
+    out_f = torch.empty_like(st.out)
+    sel_f = SelectionBuffers.empty(st.cfg)
+    hsa.hsa_forward(st.cfg, ds.Q, st.Kc, st.Vc, ds.Kq, ds.Vq, ds.tau, ds.z, ds.E, ds.F, out_f, st.ws, sel=sel_f)
+    torch.cuda.synchronize()
+    assert float((out_r - out_f).abs().max()) <= 1e-4
+    assert hsa.hsa_status_read(st.ws) == 0
