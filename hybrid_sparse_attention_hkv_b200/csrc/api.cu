@@ -79,7 +79,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 struct Layout {
   size_t status = 0, colpart = 0, q128 = 0, q64 = 0, kq64 = 0, kc128 = 0;
   size_t inter_idx = 0, inter_cnt = 0, intra_idx = 0, intra_cnt = 0;
-  size_t units = 0, n_units = 0, tile_done = 0, part_o = 0, part_ml = 0, lin_buf = 0, attn_end = 0;
+  size_t units = 0, n_units = 0, tile_done = 0, part_o = 0, part_ml = 0, part_lin = 0, attn_end = 0;
   int max_units = 0, max_slots = 0;
   size_t ekhi = 0, eklo = 0, fvhi = 0, fvlo = 0, projpart = 0, ekfv_hist = 0;
   size_t pages_end = 0;  // bytes needed by the page (HKV) calls
@@ -115,7 +115,7 @@ Layout make_layout(int H, int d, int Lq, long long Lc, int r) {
   L.tile_done = take((size_t)H * nQ128 * 4);
   L.part_o = take((size_t)L.max_slots * 128 * d * 4);
   L.part_ml = take((size_t)L.max_slots * 128 * 8);
-  L.lin_buf = take((size_t)Lq * H * d * 4);
+  L.part_lin = take((size_t)L.max_slots * 128 * d * 4);
   L.attn_end = off;
   const size_t hrd = (size_t)H * r * d;
   L.ekhi = take(hrd * 2);
@@ -262,7 +262,7 @@ hsa_status_t hsa_workspace_size(const hsa_config_t* cfg, int NP, int P_tok, size
 
 hsa_status_t hsa_status_clear(void* ws, hsa_stream_t stream) {
   if (!ws) return fail(HSA_ERR_WORKSPACE, "hsa_status_clear: workspace is NULL");
-  cudaError_t e = cudaMemsetAsync(ws, 0, sizeof(int), stream);
+  cudaError_t e = cudaMemsetAsync(ws, 0, 2 * sizeof(int), stream);  // status and the ran-out flag
   return e == cudaSuccess ? HSA_OK : fail(HSA_ERR_CUDA, "hsa_status_clear: %s", cudaGetErrorString(e));
 }
 
@@ -614,7 +614,6 @@ static hsa::AttnArgs attn_args(const hsa_config_t* cfg, const Layout& L, void* w
   a.status = status_of(ws);
   a.max_units = L.max_units;
   a.max_slots = L.max_slots;
-  a.lin_buf = at<float>(ws, L.lin_buf);
   return a;
 }
 
@@ -627,6 +626,7 @@ static hsa_status_t run_plan(const Layout& L, const hsa_selection_t& sel, void* 
   a.tile_done = at<int>(ws, L.tile_done);
   a.part_o = at<float>(ws, L.part_o);
   a.part_ml = at<float2>(ws, L.part_ml);
+  a.part_lin = at<float>(ws, L.part_lin);
   HSA_LAUNCH("attn_plan", hsa::launch_attn_plan(a, stream));
   return HSA_OK;
 }

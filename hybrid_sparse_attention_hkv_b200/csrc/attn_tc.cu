@@ -56,18 +56,7 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kTcThreads = 384;    // 12 warps = 3 warpgroups
-constexpr int kWarpV = 2;          // V producer
-constexpr int kSoftThreads = 256;  // warps 4-11: two softmax groups of 128 threads
-// Register split (setmaxnreg): the producer / MMA warpgroup gives registers to the two
-// softmax warpgroups.  The launch holds kTcThreads x (the kernel's register count);
-// the split needs 128 x kSideRegs + 256 x kSoftRegs of them, so the host refuses to
-// launch a build whose register count is below kMinLaunchRegs.
-constexpr int kSideRegs = 56;
-constexpr int kSoftRegs = 224;
-constexpr int kTailRegs = 168;  // the common tail (TMEM release, merge of split lists) runs balanced again
-constexpr int kSplitRegs = (128 * kSideRegs + 256 * kSoftRegs + kTcThreads - 1) / kTcThreads;
-constexpr int kMinLaunchRegs = kSplitRegs > kTailRegs ? kSplitRegs : kTailRegs;
+constexpr int kTcThreads = 224;  // 7 warps
 constexpr int kKStages = 3;      // K ring: a slot frees as soon as its S MMA completes
 constexpr int kVStages = 2;      // V ring: a slot frees when its P.V MMA completes
 constexpr int kRegionBytes = 128 * 128;  // one [128 rows x 64 bf16] swizzled region
@@ -239,23 +228,6 @@ __device__ __forceinline__ void softmax_tile_split(const uint32_t (&sr)[64], flo
   l = l * alpha + (st.x + st.y);
 }
 
-// Weights that combine the two softmax groups of a row: w_x = 2^(m_x - M) with M the
-// larger max (0 for a group that saw no key); returns the combined sum
-// 2^(m_0 - M) l_0 + 2^(m_1 - M) l_1.
-__device__ __forceinline__ float combine_groups(float m0, float l0, float m1, float l1, float& M, float& w0,
-                                                float& w1) {
-  M = fmaxf(m0, m1);
-  w0 = (m0 == -INFINITY) ? 0.f : exp2f(m0 - M);
-  w1 = (m1 == -INFINITY) ? 0.f : exp2f(m1 - M);
-  return w0 * l0 + w1 * l1;
-}
-
-// w0 x0 + w1 x1 where a zero weight drops its term: a group that saw no key tile in
-// a phase never wrote its accumulator, whose TMEM columns then hold anything.
-__device__ __forceinline__ float wsum(uint32_t x0, float w0, uint32_t x1, float w1) {
-  return (w0 != 0.f ? __uint_as_float(x0) * w0 : 0.f) + (w1 != 0.f ? __uint_as_float(x1) * w1 : 0.f);
-}
-
 // MMA issue by the whole MMA warp (one elected lane issues), every loop unrolled at
 // compile time: the descriptors of one tile are its base descriptor plus constant
 // address offsets (in 16-byte units, the descriptor's low field), so consecutive
@@ -296,11 +268,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   int* scratch = flags + nKq;                                 // [nKq]
   int* flagc = scratch + nKq;                                 // [nKc] (joint selection)
   __shared__ __align__(8) uint64_t bar_q, bar_k_full[kKStages], bar_k_empty[kKStages], bar_v_full[kVStages],
-      bar_v_empty[kVStages], bar_s_full[2], bar_p_full[2], bar_final, bar_lin_done, bar_lin_free, bar_ml_lin,
-      bar_ml_fin;
-  __shared__ float2 s_ml_lin[2][128], s_ml_fin[2][128];  // (max, sum) of each group of each row
+      bar_v_empty[kVStages], bar_s_full[2], bar_p_full[2], bar_o_done, bar_final;
   __shared__ uint32_t s_tmem;
   __shared__ int s_ntiles, s_n2, s_ninter;
+
   __shared__ int s_last;
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
@@ -337,13 +308,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bar_s_full[b], 1);
-      mbar_init(&bar_p_full[b], kSoftThreads / 2);  // the group that owns the buffer
+      mbar_init(&bar_p_full[b], 128);
     }
+    mbar_init(&bar_o_done, 1);
     mbar_init(&bar_final, 1);
-    mbar_init(&bar_lin_done, 1);
-    mbar_init(&bar_lin_free, kSoftThreads);
-    mbar_init(&bar_ml_lin, kSoftThreads);
-    mbar_init(&bar_ml_fin, kSoftThreads);
     fence_barrier_init();
   }
 
@@ -451,6 +419,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // this segment's share of the sparse tiles, by cost (a 128-row tile costs 2, a lone
   // 64-row chunk tile 1; the 128-row tiles come first)
   const int n2 = s_n2;
+  const int n_inter = s_ninter;
   const int n1 = s_ntiles - n_lin - n2;
   const long long cost = 2LL * n2 + n1;
   auto cut = [&](long long x) -> int {  // sparse tiles whose cumulative cost before them is < x
@@ -462,363 +431,284 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   auto tile_at = [&](int j) -> int { return j < n_lin ? tiles[j] : tiles[j + t0]; };
   if (T == 0 && nseg == 1 && tid == 0) set_status(status, HSA_ERR_DEVICE);  // no key tile: empty selection
   const uint32_t tmem = s_tmem;
-  // TMEM: S_0 | S_1 | O_0 | O_1 -- key tile j uses S_{j&1} and accumulates into O_{j&1}
-  const uint32_t tO0 = tmem + 256, tO1 = tmem + 256 + D;
+  const uint32_t tOs = tmem + 256, tOl = tmem + 256 + D;
   constexpr int kHalfSlot = (D / 64) * 64 * 128;  // 64 rows x D bf16: hi part / lo part of a slot
 
-  // Every role takes its register share at its start and gives it back at its end,
-  // so that the code before and after the roles runs with the launch's count.
-  if (warp < 4) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kSideRegs));
-    if (warp == 0) {
-      // ------------------------------------------------------------ Q + K producer
-      if (lane == 0) {
-        prefetch_tensormap(&maps.q);
-        mbar_arrive_expect_tx(&bar_q, Lay::kQBytes);
-  #pragma unroll
-        for (int c = 0; c < D / 64; ++c) tma_load_2d(sQ + c * kRegionBytes, &maps.q, &bar_q, h * D + c * 64, q0);
-      }
-      for (int j = 0; j < T; ++j) {
-        const int s = j % kKStages;
-        if (!mbar_wait(&bar_k_empty[s], ((j / kKStages) & 1) ^ 1, status, wlim)) break;
-        if (lane == 0) {
-          const int code = tile_at(j);
-          const int type = tile_type(code);
-          const int rows = tile_rows(code);
-          unsigned char* dK = sK + s * Lay::kKVBytes;
-          mbar_arrive_expect_tx(&bar_k_full[s], type == kTileLinear ? 2 * kHalfSlot : (D / 64) * rows * 128);
-          if (type == kTileLinear) {
-            const int y = h * a.r + tile_start(code);
-  #pragma unroll
-            for (int c = 0; c < D / 64; ++c) {
-              tma_load_2d(dK + c * 64 * 128, &maps.ekhi, &bar_k_full[s], c * 64, y);
-              tma_load_2d(dK + kHalfSlot + c * 64 * 128, &maps.eklo, &bar_k_full[s], c * 64, y);
-            }
-          } else if (type == kTilePair) {  // rows 0-63 and 64-127 of the slot from two blocks
-  #pragma unroll
-            for (int c = 0; c < D / 64; ++c) {
-              tma_load_2d(dK + c * 128 * 128, &maps.kq, &bar_k_full[s], h * D + c * 64, pair_first(code) * 64);
-              tma_load_2d(dK + c * 128 * 128 + 64 * 128, &maps.kq, &bar_k_full[s], h * D + c * 64,
-                          pair_second(code) * 64);
-            }
-          } else {
-            const CUtensorMap* mk = type == kTileChunk ? &maps.kq : &maps.kc;
-  #pragma unroll
-            for (int c = 0; c < D / 64; ++c)
-              tma_load_2d(dK + c * rows * 128, mk, &bar_k_full[s], h * D + c * 64, tile_start(code));
-          }
-        }
-        __syncwarp();
-      }
-    } else if (warp == kWarpV) {
-      // ------------------------------------------------------------ V producer
-      for (int j = 0; j < T; ++j) {
-        const int s = j % kVStages;
-        if (!mbar_wait(&bar_v_empty[s], ((j / kVStages) & 1) ^ 1, status, wlim)) break;
-        if (lane == 0) {
-          const int code = tile_at(j);
-          const int type = tile_type(code);
-          const int rows = tile_rows(code);
-          unsigned char* dV = sV + s * Lay::kKVBytes;
-          mbar_arrive_expect_tx(&bar_v_full[s], type == kTileLinear ? 2 * kHalfSlot : (D / 64) * rows * 128);
-          if (type == kTileLinear) {
-            const int y = h * a.r + tile_start(code);
-  #pragma unroll
-            for (int c = 0; c < D / 64; ++c) {
-              tma_load_2d(dV + c * 64 * 128, &maps.fvhi, &bar_v_full[s], c * 64, y);
-              tma_load_2d(dV + kHalfSlot + c * 64 * 128, &maps.fvlo, &bar_v_full[s], c * 64, y);
-            }
-          } else if (type == kTilePair) {
-  #pragma unroll
-            for (int c = 0; c < D / 64; ++c) {
-              tma_load_2d(dV + c * 128 * 128, &maps.vq, &bar_v_full[s], h * D + c * 64, pair_first(code) * 64);
-              tma_load_2d(dV + c * 128 * 128 + 64 * 128, &maps.vq, &bar_v_full[s], h * D + c * 64,
-                          pair_second(code) * 64);
-            }
-          } else {
-            const CUtensorMap* mv = type == kTileChunk ? &maps.vq : &maps.vc;
-  #pragma unroll
-            for (int c = 0; c < D / 64; ++c)
-              tma_load_2d(dV + c * rows * 128, mv, &bar_v_full[s], h * D + c * 64, tile_start(code));
-          }
-        }
-        __syncwarp();
-      }
-    } else if (warp == 3) {
-      // idle: its warpgroup's registers went to the softmax warps
-    } else if (warp == 1) {
-      // ------------------------------------------------------------ MMA issuer
-      bool ok = mbar_wait_warp(&bar_q, 0, status, wlim);
-      tc_fence_after();
-      const uint64_t qd = sdesc_sw128(smem_u32(sQ), 16, 1024);
-      // The warp stays converged: waits take the warp's common answer, tile codes and
-      // descriptors are warp-uniform, one elected lane issues each MMA and commit.
-      // K and V arrive by TMA on their mbarriers, which orders them for the tensor
-      // core; only P, written to TMEM by the softmax warps, needs the tcgen05 fence.
-      // Order: S_0, S_1, then per tile j: P_j V_j into O_{j&1}, then S_{j+2} into the
-      // buffer P_j has just been read from (the tensor core runs its MMAs in order).
-      auto issue_s = [&](int j) -> bool {
-        const int s = j % kKStages;
-        if (!mbar_wait_warp(&bar_k_full[s], (j / kKStages) & 1, status, wlim)) return false;
-        const int code = tile_at(j);
-        const uint64_t kd = sdesc_sw128(smem_u32(sK + s * Lay::kKVBytes), 16, 1024);
-        const uint32_t tS = tmem + (j & 1) * 128;
-        if (tile_type(code) == kTileLinear) {  // EK_hi then EK_lo, 64 rows each
-          issue_qk<D, 64>(tS, qd, kd, false);
-          issue_qk<D, 64>(tS, qd, kd + (uint64_t)(kHalfSlot >> 4), true);
-        } else if (tile_rows(code) == 128) {
-          issue_qk<D, 128>(tS, qd, kd, false);
-        } else {
-          issue_qk<D, 64>(tS, qd, kd, false);
-        }
-        mma_commit_elect(&bar_k_empty[s]);
-        mma_commit_elect(&bar_s_full[j & 1]);
-        return true;
-      };
-      if (ok && T > 0) ok = issue_s(0);
-      if (ok && T > 1) ok = issue_s(1);
-      for (int j = 0; ok && j < T; ++j) {
-        // the first sparse P.V overwrites the accumulators: the linear branch must have
-        // been read out of them first
-        if (j == n_lin && n_lin > 0 && !mbar_wait_warp(&bar_lin_free, 0, status, wlim)) break;
-        if (!mbar_wait_warp(&bar_p_full[j & 1], (j >> 1) & 1, status, wlim)) break;
-        const int sv = j % kVStages;
-        if (!mbar_wait_warp(&bar_v_full[sv], (j / kVStages) & 1, status, wlim)) break;
-        tc_fence_after();
-        const int code = tile_at(j);
-        const uint32_t v_base = smem_u32(sV + sv * Lay::kKVBytes);
-        const uint32_t tP = tmem + (j & 1) * 128;
-        const uint32_t tO = (j & 1) ? tO1 : tO0;
-        // the first tile of each phase in each accumulator starts it
-        const bool acc = !(j < 2 || j == n_lin || j == n_lin + 1);
-        if (tile_type(code) == kTileLinear) {
-          // O += P_hi FV_hi + P_lo FV_hi + P_hi FV_lo
-          const uint64_t vhi = sdesc_sw128(v_base, 64 * 128, 1024);
-          const uint64_t vlo = sdesc_sw128(v_base + kHalfSlot, 64 * 128, 1024);
-          issue_pv<D, 64>(tO, tP, vhi, acc);
-          issue_pv<D, 64>(tO, tP + 32, vhi, true);
-          issue_pv<D, 64>(tO, tP, vlo, true);
-        } else if (tile_rows(code) == 128) {
-          issue_pv<D, 128>(tO, tP, sdesc_sw128(v_base, 128 * 128, 1024), acc);
-        } else {
-          issue_pv<D, 64>(tO, tP, sdesc_sw128(v_base, 64 * 128, 1024), acc);
-        }
-        mma_commit_elect(&bar_v_empty[sv]);
-        // one-shot barriers: every MMA of the linear phase / of the unit has completed
-        if (j == n_lin - 1) mma_commit_elect(&bar_lin_done);
-        if (j == T - 1) mma_commit_elect(&bar_final);
-        if (j + 2 < T && !issue_s(j + 2)) break;
-      }
+  if (warp == 0) {
+    // ------------------------------------------------------------ Q + K producer
+    if (lane == 0) {
+      prefetch_tensormap(&maps.q);
+      mbar_arrive_expect_tx(&bar_q, Lay::kQBytes);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) tma_load_2d(sQ + c * kRegionBytes, &maps.q, &bar_q, h * D + c * 64, q0);
     }
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kTailRegs));
-  } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftRegs));
-    {
-      // ------------------------------------------------------------ softmax + epilogue (warps 4-11)
-      const int grp = warp >= 8 ? 1 : 0;  // key tiles j with j % 2 == grp
-      const int wq = warp & 3;
-      const int row = 32 * wq + lane;
-      const int half_bit = wq < 2 ? 1 : 2;  // warp-uniform: rows 0..63 are query half 0
-      const uint32_t loff = (uint32_t)(32 * wq) << 16;
-      const uint32_t tO = (grp ? tO1 : tO0) + loff;
-      const uint32_t tS = tmem + grp * 128 + loff;
-      const float sl2 = a.scale * 1.4426950408889634f;
-      const int grow = q0 + row;
-      const bool valid_row = grow < a.Lq;
-      // out = g o_s + (1 - g) o_l with g = sigmoid(gate logit) when both branches run
-      const float g = (do_sparse && any_lin && a.gate_logit) ? 1.f / (1.f + expf(-a.gate_logit[h])) : 1.f;
-      float ms = -INFINITY, ls = 0.f;  // sparse branch running max / sum of this group
-      float ml = -INFINITY, ll = 0.f;  // linear branch running max / sum of this group
-      bool ok = true;
-      bool stashed = !do_lin;
-      auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {  // bounded, warp-uniform answer
-        return mbar_wait_warp(bar, par, status, wlim);
-      };
-      // ---- end of the linear phase: combine the two groups, weight by 1 - g (or 1),
-      // and stash (or, without a sparse branch, store) this thread's half of the row's
-      // columns; then hand the accumulators back to the sparse tiles
-      auto stash_linear = [&]() -> bool {
-        s_ml_lin[grp][row] = make_float2(ml, ll);
-        mbar_arrive(&bar_ml_lin);
-        if (!wait_all(&bar_ml_lin, 0) || !wait_all(&bar_lin_done, 0)) return false;
-        tc_fence_after();
-        const float2 p0 = s_ml_lin[0][row], p1 = s_ml_lin[1][row];
-        float M, w0, w1;
-        const float L = combine_groups(p0.x, p0.y, p1.x, p1.y, M, w0, w1);
-        const float wl = (do_sparse ? 1.f - g : 1.f) / L;
-        w0 *= wl;
-        w1 *= wl;
-  #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          const int cc = grp * (D / 32) + c;  // 16-column group of the row
-          uint32_t r0[16], r1[16];
-          tmem_ld16_sync(tO0 + loff + cc * 16, r0);
-          tmem_ld16_sync(tO1 + loff + cc * 16, r1);
-          if (valid_row) {
-            float v[16];
-  #pragma unroll
-            for (int k = 0; k < 16; ++k) v[k] = wsum(r0[k], w0, r1[k], w1);
-            if (do_sparse) {
-              float* dst = a.lin_buf + ((long long)grow * a.H + h) * D + cc * 16;
-  #pragma unroll
-              for (int k = 0; k < 16; k += 4) *reinterpret_cast<float4*>(dst + k) = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
-            } else {
-              store_out16(a, grow, h, D, cc, v);
-            }
+    for (int j = 0; j < T; ++j) {
+      const int s = j % kKStages;
+      if (!mbar_wait(&bar_k_empty[s], ((j / kKStages) & 1) ^ 1, status, wlim)) break;
+      if (lane == 0) {
+        const int code = tile_at(j);
+        const int type = tile_type(code);
+        const int rows = tile_rows(code);
+        unsigned char* dK = sK + s * Lay::kKVBytes;
+        mbar_arrive_expect_tx(&bar_k_full[s], type == kTileLinear ? 2 * kHalfSlot : (D / 64) * rows * 128);
+        if (type == kTileLinear) {
+          const int y = h * a.r + tile_start(code);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_2d(dK + c * 64 * 128, &maps.ekhi, &bar_k_full[s], c * 64, y);
+            tma_load_2d(dK + kHalfSlot + c * 64 * 128, &maps.eklo, &bar_k_full[s], c * 64, y);
           }
-        }
-        if (do_sparse) __threadfence();  // a merging CTA may read the stash
-        tc_fence_before();
-        mbar_arrive(&bar_lin_free);
-        return true;
-      };
-      for (int j = grp; j < T; j += 2) {
-        if (!stashed && j >= n_lin) {
-          stashed = true;
-          if (!stash_linear()) {
-            ok = false;
-            break;
+        } else if (type == kTilePair) {  // rows 0-63 and 64-127 of the slot from two blocks
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_2d(dK + c * 128 * 128, &maps.kq, &bar_k_full[s], h * D + c * 64, pair_first(code) * 64);
+            tma_load_2d(dK + c * 128 * 128 + 64 * 128, &maps.kq, &bar_k_full[s], h * D + c * 64,
+                        pair_second(code) * 64);
           }
+        } else {
+          const CUtensorMap* mk = type == kTileChunk ? &maps.kq : &maps.kc;
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_2d(dK + c * rows * 128, mk, &bar_k_full[s], h * D + c * 64, tile_start(code));
         }
-        if (!mbar_wait(&bar_s_full[grp], (j >> 1) & 1, status, wlim)) {
+      }
+      __syncwarp();
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------ V producer
+    for (int j = 0; j < T; ++j) {
+      const int s = j % kVStages;
+      if (!mbar_wait(&bar_v_empty[s], ((j / kVStages) & 1) ^ 1, status, wlim)) break;
+      if (lane == 0) {
+        const int code = tile_at(j);
+        const int type = tile_type(code);
+        const int rows = tile_rows(code);
+        unsigned char* dV = sV + s * Lay::kKVBytes;
+        mbar_arrive_expect_tx(&bar_v_full[s], type == kTileLinear ? 2 * kHalfSlot : (D / 64) * rows * 128);
+        if (type == kTileLinear) {
+          const int y = h * a.r + tile_start(code);
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_2d(dV + c * 64 * 128, &maps.fvhi, &bar_v_full[s], c * 64, y);
+            tma_load_2d(dV + kHalfSlot + c * 64 * 128, &maps.fvlo, &bar_v_full[s], c * 64, y);
+          }
+        } else if (type == kTilePair) {
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_2d(dV + c * 128 * 128, &maps.vq, &bar_v_full[s], h * D + c * 64, pair_first(code) * 64);
+            tma_load_2d(dV + c * 128 * 128 + 64 * 128, &maps.vq, &bar_v_full[s], h * D + c * 64,
+                        pair_second(code) * 64);
+          }
+        } else {
+          const CUtensorMap* mv = type == kTileChunk ? &maps.vq : &maps.vc;
+#pragma unroll
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_2d(dV + c * rows * 128, mv, &bar_v_full[s], h * D + c * 64, tile_start(code));
+        }
+      }
+      __syncwarp();
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    bool ok = mbar_wait_warp(&bar_q, 0, status, wlim);
+    tc_fence_after();
+    const uint64_t qd = sdesc_sw128(smem_u32(sQ), 16, 1024);
+    // The warp stays converged: waits take the warp's common answer, tile codes and
+    // descriptors are warp-uniform, one elected lane issues each MMA and commit.
+    // K and V arrive by TMA on their mbarriers, which orders them for the tensor
+    // core; only P, written to TMEM by the softmax warps, needs the tcgen05 fence.
+    auto issue_s = [&](int j) -> bool {
+      const int s = j % kKStages;
+      if (!mbar_wait_warp(&bar_k_full[s], (j / kKStages) & 1, status, wlim)) return false;
+      const int code = tile_at(j);
+      const uint64_t kd = sdesc_sw128(smem_u32(sK + s * Lay::kKVBytes), 16, 1024);
+      const uint32_t tS = tmem + (j & 1) * 128;
+      if (tile_type(code) == kTileLinear) {  // EK_hi then EK_lo, 64 rows each
+        issue_qk<D, 64>(tS, qd, kd, false);
+        issue_qk<D, 64>(tS, qd, kd + (uint64_t)(kHalfSlot >> 4), true);
+      } else if (tile_rows(code) == 128) {
+        issue_qk<D, 128>(tS, qd, kd, false);
+      } else {
+        issue_qk<D, 64>(tS, qd, kd, false);
+      }
+      mma_commit_elect(&bar_k_empty[s]);
+      mma_commit_elect(&bar_s_full[j & 1]);
+      return true;
+    };
+    if (ok && T > 0) ok = issue_s(0);
+    for (int j = 0; ok && j < T; ++j) {
+      if (j + 1 < T && !issue_s(j + 1)) break;
+      if (!mbar_wait_warp(&bar_p_full[j & 1], (j >> 1) & 1, status, wlim)) break;
+      const int sv = j % kVStages;
+      if (!mbar_wait_warp(&bar_v_full[sv], (j / kVStages) & 1, status, wlim)) break;
+      tc_fence_after();
+      const int code = tile_at(j);
+      const uint32_t v_base = smem_u32(sV + sv * Lay::kKVBytes);
+      const uint32_t tP = tmem + (j & 1) * 128;
+      if (tile_type(code) == kTileLinear) {
+        // O_l += P_hi FV_hi + P_lo FV_hi + P_hi FV_lo; first linear tile initialises O_l
+        const uint64_t vhi = sdesc_sw128(v_base, 64 * 128, 1024);
+        const uint64_t vlo = sdesc_sw128(v_base + kHalfSlot, 64 * 128, 1024);
+        issue_pv<D, 64>(tOl, tP, vhi, j > 0);
+        issue_pv<D, 64>(tOl, tP + 32, vhi, true);
+        issue_pv<D, 64>(tOl, tP, vlo, true);
+      } else if (tile_rows(code) == 128) {  // the first sparse tile initialises O_s
+        issue_pv<D, 128>(tOs, tP, sdesc_sw128(v_base, 128 * 128, 1024), j > n_lin);
+      } else {
+        issue_pv<D, 64>(tOs, tP, sdesc_sw128(v_base, 64 * 128, 1024), j > n_lin);
+      }
+      mma_commit_elect(&bar_v_empty[sv]);
+      mma_commit_elect(&bar_o_done);
+      // one-shot: completes once every MMA of the unit has completed
+      if (j == T - 1) mma_commit_elect(&bar_final);
+    }
+  } else if (warp >= 2 && warp <= 5) {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int wq = warp & 3;
+    const int row = 32 * wq + lane;
+    const int half_bit = wq < 2 ? 1 : 2;  // warp-uniform: rows 0..63 are half 0
+    const uint32_t loff = (uint32_t)(32 * wq) << 16;
+    const float sl2 = a.scale * 1.4426950408889634f;
+    float ms = -INFINITY, ls = 0.f;  // sparse branch running max / sum
+    float ml = -INFINITY, ll = 0.f;  // linear branch running max / sum
+    bool ok = true;
+    for (int j = 0; j < T; ++j) {
+      const int b = j & 1;
+      if (!mbar_wait(&bar_s_full[b], (j >> 1) & 1, status, wlim)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int code = tile_at(j);
+      const int type = tile_type(code);
+      const int rows = tile_rows(code);
+      const long long nrows = (type == kTileChunk || type == kTilePair) ? (long long)a.Lq : a.Lc;
+      const int valid = type == kTileLinear ? 64
+                        : type == kTilePair ? 64 + (int)min(64LL, nrows - 64LL * pair_second(code))
+                                            : (int)min((long long)rows, nrows - tile_start(code));
+      const bool used = (code & half_bit) != 0;
+      const uint32_t tS = tmem + b * 128 + loff;
+      float alpha = 1.f;
+      bool rescale = false;
+      if (type == kTileLinear) {  // tile-uniform
+        uint32_t h64[64];
+        tmem_ld64_sync(tS, h64);
+        softmax_tile_split(h64, sl2, ml, ll, alpha, rescale, tS);
+      } else if (used) {  // warp-uniform (a warp's 32 rows lie in one 64-row half)
+        uint32_t sr[128];
+        if (rows == 128) {
+          tmem_ld128_sync(tS, sr);
+          if (valid == 128) softmax_tile<128, false>(sr, valid, sl2, ms, ls, alpha, rescale, tS);
+          else softmax_tile<128, true>(sr, valid, sl2, ms, ls, alpha, rescale, tS);
+        } else {
+          uint32_t h64[64];
+          tmem_ld64_sync(tS, h64);
+#pragma unroll
+          for (int k = 0; k < 64; ++k) sr[k] = h64[k];
+          if (valid == 64) softmax_tile<64, false>(sr, valid, sl2, ms, ls, alpha, rescale, tS);
+          else softmax_tile<64, true>(sr, valid, sl2, ms, ls, alpha, rescale, tS);
+        }
+      } else {
+        uint32_t zero[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) zero[k] = 0u;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (c * 32 < rows) tmem_st16(tS + c * 16, zero);
+      }
+      tmem_st_wait();
+      if (__any_sync(0xffffffffu, rescale)) {
+        // O holds the P.V products of tiles 0..j-1 once the last of them has completed
+        // (P.V of tile j cannot have started: it waits for this P).  Without a rescale
+        // nothing here touches O, and the wait is skipped.
+        if (j > 0 && !mbar_wait(&bar_o_done, (j - 1) & 1, status, wlim)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const int code = tile_at(j);
-        const int type = tile_type(code);
-        const int rows = tile_rows(code);
-        const long long nrows = (type == kTileChunk || type == kTilePair) ? (long long)a.Lq : a.Lc;
-        const int valid = type == kTileLinear ? 64
-                          : type == kTilePair ? 64 + (int)min(64LL, nrows - 64LL * pair_second(code))
-                                              : (int)min((long long)rows, nrows - tile_start(code));
-        const bool used = (code & half_bit) != 0;
-        float alpha = 1.f;
-        bool rescale = false;
-        if (type == kTileLinear) {  // tile-uniform
-          uint32_t h64[64];
-          tmem_ld64_sync(tS, h64);
-          softmax_tile_split(h64, sl2, ml, ll, alpha, rescale, tS);
-        } else if (used) {  // warp-uniform (a warp's 32 rows lie in one 64-row half)
-          uint32_t sr[128];
-          if (rows == 128) {
-            tmem_ld128_sync(tS, sr);
-            if (valid == 128) softmax_tile<128, false>(sr, valid, sl2, ms, ls, alpha, rescale, tS);
-            else softmax_tile<128, true>(sr, valid, sl2, ms, ls, alpha, rescale, tS);
-          } else {
-            uint32_t h64[64];
-            tmem_ld64_sync(tS, h64);
-  #pragma unroll
-            for (int k = 0; k < 64; ++k) sr[k] = h64[k];
-            if (valid == 64) softmax_tile<64, false>(sr, valid, sl2, ms, ls, alpha, rescale, tS);
-            else softmax_tile<64, true>(sr, valid, sl2, ms, ls, alpha, rescale, tS);
-          }
-        } else {
-          uint32_t zero[16];
-  #pragma unroll
-          for (int k = 0; k < 16; ++k) zero[k] = 0u;
-  #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            if (c * 32 < rows) tmem_st16(tS + c * 16, zero);
+        const uint32_t tO = type == kTileLinear ? tOl : tOs;
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t r[16];
+          tmem_ld16_sync(tO + loff + c * 16, r);
+#pragma unroll
+          for (int k = 0; k < 16; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
+          tmem_st16(tO + loff + c * 16, r);
         }
         tmem_st_wait();
-        if (__any_sync(0xffffffffu, rescale)) {
-          // O_grp holds the P.V products of this group's earlier tiles, all complete:
-          // S_j was issued after P.V of tile j - 2 (the group's previous tile) and the
-          // tensor core runs its MMAs in order; P.V of tile j waits for this P.
-          tc_fence_after();
-  #pragma unroll
-          for (int c = 0; c < D / 16; ++c) {
-            uint32_t r[16];
-            tmem_ld16_sync(tO + c * 16, r);
-  #pragma unroll
-            for (int k = 0; k < 16; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * alpha);
-            tmem_st16(tO + c * 16, r);
-          }
-          tmem_st_wait();
-        }
-        tc_fence_before();
-        mbar_arrive(&bar_p_full[grp]);
       }
-      if (ok && !stashed) {  // this group had no tile after the linear ones
-        stashed = true;
-        ok = stash_linear();
-      }
-      // ---- epilogue of the sparse branch: wait for every P.V product of the unit on
-      // the one-shot barrier the MMA warp commits after its last P.V (phase 0, so its
-      // parity names it unambiguously), combine the two groups of the row and store
-      if (ok && do_sparse && T > 0) ok = wait_all(&bar_final, 0);
-      if (ok && do_sparse) {
-        s_ml_fin[grp][row] = make_float2(ms, ls);
-        mbar_arrive(&bar_ml_fin);
-        ok = wait_all(&bar_ml_fin, 0);
-      }
-      if (ok && do_sparse) {
-        tc_fence_after();
-        const float2 p0 = s_ml_fin[0][row], p1 = s_ml_fin[1][row];
-        float M, w0, w1;
-        const float L = combine_groups(p0.x, p0.y, p1.x, p1.y, M, w0, w1);
-        const bool had_sparse = T > n_lin;
-        if (nseg == 1) {
-          if (valid_row && !(L > 0.f)) set_status(status, HSA_ERR_DEVICE);
-          if (valid_row && a.lse_out && grp == 0)  // ln sum_k exp(q.k * scale) = (M + log2 L) ln 2
-            a.lse_out[(long long)grow * a.H + h] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
-          const float ws = L > 0.f ? g / L : 0.f;
-  #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            const int cc = grp * (D / 32) + c;
-            uint32_t r0[16], r1[16];
-            tmem_ld16_sync(tO0 + loff + cc * 16, r0);
-            tmem_ld16_sync(tO1 + loff + cc * 16, r1);
-            if (valid_row) {
-              float v[16];
-  #pragma unroll
-              for (int k = 0; k < 16; ++k) v[k] = (wsum(r0[k], w0, r1[k], w1)) * ws;
-              if (do_lin) {
-                const float* src = a.lin_buf + ((long long)grow * a.H + h) * D + cc * 16;
-  #pragma unroll
-                for (int k = 0; k < 16; k += 4) {
-                  const float4 l4 = *reinterpret_cast<const float4*>(src + k);
-                  v[k] += l4.x; v[k + 1] += l4.y; v[k + 2] += l4.z; v[k + 3] += l4.w;
-                }
-              }
-              store_out16(a, grow, h, D, cc, v);
-            }
-          }
-        } else {
-          // one segment of a split list: the combined unnormalised O_s (relative to M)
-          // and (M, L); the linear branch, if any, is in the stash
-          const int slot = slot0 + seg;
-          float* po = a.part_o + ((long long)slot * 128 + row) * D;
-  #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            const int cc = grp * (D / 32) + c;
-            uint32_t r0[16], r1[16];
-            if (had_sparse) {
-              tmem_ld16_sync(tO0 + loff + cc * 16, r0);
-              tmem_ld16_sync(tO1 + loff + cc * 16, r1);
-            }
-            if (valid_row) {
-  #pragma unroll
-              for (int k = 0; k < 16; k += 4) {
-                float4 o4 = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (had_sparse)
-                  o4 = make_float4(wsum(r0[k], w0, r1[k], w1),
-                                   wsum(r0[k + 1], w0, r1[k + 1], w1),
-                                   wsum(r0[k + 2], w0, r1[k + 2], w1),
-                                   wsum(r0[k + 3], w0, r1[k + 3], w1));
-                *reinterpret_cast<float4*>(po + cc * 16 + k) = o4;
-              }
-            }
-          }
-          if (valid_row && grp == 0)
-            a.part_ml[(long long)slot * 128 + row] = make_float2(had_sparse && L > 0.f ? M : -INFINITY, L);
-          __threadfence();
-        }
-      }
-  
+      tc_fence_before();
+      mbar_arrive(&bar_p_full[b]);
     }
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kTailRegs));
+    // Wait for every P.V product of the unit on the one-shot barrier the MMA warp
+    // commits after its last P.V (phase 0, so the parity names it unambiguously; the
+    // per-tile barrier can be up to two phases ahead or behind here).  The wait polls
+    // (bounded): the softmax warps have no other work left, and sleeping waits here
+    // cost 1 % of the kernel's time.
+    auto wait_poll = [&](uint64_t* bar, uint32_t par) -> bool {
+      bool r = false;
+      for (uint32_t i = 0; i < kSpinLimit && !r; ++i) r = mbar_try_wait(bar, par);
+      if (!r) set_status(status, HSA_ERR_TIMEOUT);
+      return __all_sync(0xffffffffu, r);
+    };
+    if (ok && (T == 0 || wait_poll(&bar_final, 0))) {
+      tc_fence_after();
+      const int grow = q0 + row;
+      const bool valid_row = grow < a.Lq;
+      // out = g o_s + (1 - g) o_l with g = sigmoid(gate logit) when both branches run
+      const float g = (do_sparse && any_lin && a.gate_logit) ? 1.f / (1.f + expf(-a.gate_logit[h])) : 1.f;
+      const float wl = do_lin ? (do_sparse ? 1.f - g : 1.f) / ll : 0.f;
+      if (nseg == 1) {
+        if (do_sparse && valid_row && !(ls > 0.f)) set_status(status, HSA_ERR_DEVICE);
+        const float ws = (do_sparse && ls > 0.f) ? g / ls : 0.f;
+        if (do_sparse && valid_row && a.lse_out)  // ln sum_k exp(q.k * scale) = (m + log2 l) ln 2
+          a.lse_out[(long long)grow * a.H + h] = ls > 0.f ? (ms + log2f(ls)) * 0.6931471805599453f : -INFINITY;
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t rs[16], rl[16];
+          if (do_sparse) tmem_ld16_sync(tOs + loff + c * 16, rs);
+          if (do_lin) tmem_ld16_sync(tOl + loff + c * 16, rl);
+          if (valid_row) {
+            float v[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              const float vs = do_sparse ? __uint_as_float(rs[k]) * ws : 0.f;
+              const float vl = do_lin ? __uint_as_float(rl[k]) * wl : 0.f;
+              v[k] = vs + vl;
+            }
+            store_out16(a, grow, h, D, c, v);
+          }
+        }
+      } else {
+        // one segment of a split list: unnormalised O_s and (max, sum); segment 0
+        // also leaves the weighted linear branch at the list's first slot
+        const int slot = slot0 + seg;
+        float* po = a.part_o + ((long long)slot * 128 + row) * D;
+        float* pl = a.part_lin + ((long long)slot0 * 128 + row) * D;
+        const bool had_sparse = T > n_lin;
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t rs[16], rl[16];
+          if (had_sparse) tmem_ld16_sync(tOs + loff + c * 16, rs);
+          if (do_lin) tmem_ld16_sync(tOl + loff + c * 16, rl);
+          if (valid_row) {
+#pragma unroll
+            for (int k = 0; k < 16; k += 4) {
+              *reinterpret_cast<float4*>(po + c * 16 + k) =
+                  had_sparse ? make_float4(__uint_as_float(rs[k]), __uint_as_float(rs[k + 1]),
+                                           __uint_as_float(rs[k + 2]), __uint_as_float(rs[k + 3]))
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+              if (do_lin)
+                *reinterpret_cast<float4*>(pl + c * 16 + k) =
+                    make_float4(__uint_as_float(rl[k]) * wl, __uint_as_float(rl[k + 1]) * wl,
+                                __uint_as_float(rl[k + 2]) * wl, __uint_as_float(rl[k + 3]) * wl);
+            }
+          }
+        }
+        if (valid_row) a.part_ml[(long long)slot * 128 + row] = make_float2(had_sparse && ls > 0.f ? ms : -INFINITY, ls);
+        __threadfence();
+      }
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -831,7 +721,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // segment order (which CTA that is does not change the result)
     if (tid == 0) s_last = atomicAdd(&a.tile_done[tq], 1) == nseg - 1;
     __syncthreads();
-    if (s_last && warp >= 4 && warp <= 7) {
+    if (s_last && warp >= 2 && warp <= 5) {
       __threadfence();
       const int row = 32 * (warp & 3) + lane, grow = q0 + row;
       if (grow < a.Lq) {
@@ -846,7 +736,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (a.lse_out) a.lse_out[(long long)grow * a.H + h] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
         const float g = (any_lin && a.gate_logit) ? 1.f / (1.f + expf(-a.gate_logit[h])) : 1.f;
         const float ws = L > 0.f ? g / L : 0.f;
-        const float* pl = a.lin_buf + ((long long)grow * a.H + h) * D;
+        const float* pl = a.part_lin + ((long long)slot0 * 128 + row) * D;
 #pragma unroll 1
         for (int c = 0; c < D / 16; ++c) {
           float v[16];
@@ -932,10 +822,6 @@ cudaError_t launch_tc(const AttnArgs& a, cudaStream_t s) {
   if (smem > 232448) return cudaErrorInvalidConfiguration;
   e = cudaFuncSetAttribute(sparse_attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  // the register split must fit in what the launch allocates (else setmaxnreg.inc waits)
-  cudaFuncAttributes fa;
-  if ((e = cudaFuncGetAttributes(&fa, sparse_attn_tc_kernel<D>)) != cudaSuccess) return e;
-  if (fa.numRegs < kMinLaunchRegs) return cudaErrorInvalidConfiguration;
   const int grid = a.units ? a.max_units : a.H * nQ128;
   sparse_attn_tc_kernel<D><<<grid, kTcThreads, smem, s>>>(maps, a, nQ128, nKc, nQ64, nKq);
   return cudaGetLastError();

@@ -15,7 +15,9 @@ constexpr int kBlockIntra = 64;
 // ------------------------------------------------------------------ status word
 // The first 256 bytes of every workspace are its header:
 //   int32 [0]  device status (an hsa_status_t); kernels record only the first failure
-//   int32 [1]  reserved
+//   int32 [1]  nonzero once a bounded wait has run out: every other wait of the same
+//              workspace then gives up at its next poll instead of running out on its
+//              own, so a protocol that stalls ends in one wait limit, not one per wait
 //   uint32[2]  kWaitTag when word 3 holds a limit set by hsa_set_wait_limit
 //   uint32[3]  limit of every bounded device wait, in microseconds
 constexpr uint32_t kWaitTag = 0x54494157u;  // "WAIT"

@@ -124,7 +124,7 @@ struct AttnArgs {
   int* tile_done;    // [H * nQ128] segments finished (zeroed by the plan)
   float* part_o;     // [max_slots][128][d] unnormalised O_s of a segment
   float2* part_ml;   // [max_slots][128] running max (log2 units) and sum of a segment
-  float* lin_buf;    // [Lq][H][d] the linear branch weighted by 1 - g, stashed between the two phases
+  float* part_lin;   // [max_slots][128][d] weighted linear branch of a split list (at its first slot)
 };
 // Sparse and/or linear branch with the gated merge, on tcgen05 / TMEM / TMA.
 cudaError_t launch_attn_tc(const AttnArgs& a, cudaStream_t s);

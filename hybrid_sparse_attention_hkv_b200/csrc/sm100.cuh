@@ -63,8 +63,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
   const uint64_t t0 = global_ns();
   do {
     if (mbar_try_wait_sleep(bar, parity)) return true;
+    // another wait of this workspace already ran out: give up now
+    if (status != nullptr && *reinterpret_cast<volatile int*>(status + 1) != 0) return false;
   } while (global_ns() - t0 < limit_ns);
   set_status(status, HSA_ERR_TIMEOUT);
+  if (status != nullptr) atomicExch(status + 1, 1);
   return false;
 }
 

@@ -37,6 +37,8 @@
  *     after the stream has reached the call.
  *   - Workspace: one caller-allocated device buffer of hsa_workspace_size()
  *     bytes (256-byte aligned) serves every entry point of a configuration.
+ *     Its 256-byte header (status word, ran-out flag, wait limit) must be zero
+ *     before first use: allocate it zeroed, or call hsa_status_clear.
  *     Calls that share a workspace must be ordered on one stream.
  *   - Supported shapes: d in {64, 128}; H >= 1; block_inter = 128;
  *     block_intra = 64; rank a multiple of 64 in [64, 1024]; Lc and Lq
@@ -116,7 +118,8 @@ typedef struct {
  * The size includes the 256-byte status header. */
 hsa_status_t hsa_workspace_size(const hsa_config_t* cfg, int NP, int P_tok, size_t* bytes);
 
-/* Clear the device status word of `ws` (enqueued on `stream`). */
+/* Clear the device status word of `ws` and its ran-out flag (enqueued on
+ * `stream`). */
 hsa_status_t hsa_status_clear(void* ws, hsa_stream_t stream);
 
 /* Synchronise `stream`, then copy the device status word of `ws` into *status
@@ -127,7 +130,10 @@ hsa_status_t hsa_status_read(const void* ws, hsa_stream_t stream, int* status);
  * waits of the tensor-core kernels), in microseconds; 0 restores the 2 s
  * default.  Enqueued on `stream`; kept in the workspace header until changed
  * (hsa_status_clear leaves it).  A wait that runs out records HSA_ERR_TIMEOUT in
- * the status word and its kernel drains its copies and MMAs and exits. */
+ * the status word, sets the workspace's ran-out flag, and its kernel drains its
+ * copies and MMAs and exits.  While the flag is set (until hsa_status_clear),
+ * every other wait of a kernel using `ws` gives up at its first unsuccessful
+ * poll, so a stalled launch ends after one wait limit rather than one per CTA. */
 hsa_status_t hsa_set_wait_limit(void* ws, unsigned int limit_us, hsa_stream_t stream);
 
 /* Self-test of the timeout path (failure detection; the paper has no
