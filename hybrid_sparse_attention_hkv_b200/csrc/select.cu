@@ -111,8 +111,11 @@ __device__ __forceinline__ bool ranks_before(float ea, int ia, float eb, int ib)
   return ea > eb || (ea == eb && ia < ib);
 }
 
+// Exclusive prefix sum of one value per thread over the block; `total` receives the
+// block's sum in every thread.  warp_tot: shared, kSelThreads / 32 + 1 entries.
 template <typename T>
-__device__ T block_excl_scan(T v, T* warp_tot, T* total) {
+__device__ T block_excl_scan(T v, T* warp_tot, T& total) {
+  constexpr int kWarps = kSelThreads / 32;
   const int lane = threadIdx.x % 32, warp = threadIdx.x / 32;
   T x = v;
 #pragma unroll
@@ -123,18 +126,19 @@ __device__ T block_excl_scan(T v, T* warp_tot, T* total) {
   if (lane == 31) warp_tot[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    T w = lane < kSelThreads / 32 ? warp_tot[lane] : T(0);
+    T w = lane < kWarps ? warp_tot[lane] : T(0);
     T wx = w;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       T y = __shfl_up_sync(0xffffffffu, wx, o);
       if (lane >= o) wx += y;
     }
-    if (lane < kSelThreads / 32) warp_tot[lane] = wx - w;  // exclusive warp offsets
-    if (lane == kSelThreads / 32 - 1) *total = wx;
+    if (lane < kWarps) warp_tot[lane] = wx - w;  // exclusive warp offsets
+    if (lane == kWarps - 1) warp_tot[kWarps] = wx;
   }
   __syncthreads();
   T r = warp_tot[warp] + x - v;
+  total = warp_tot[kWarps];
   __syncthreads();
   return r;
 }
@@ -302,7 +306,7 @@ __global__ void __launch_bounds__(kSelThreads) block_select_kernel(
   double local = 0.0;
   for (int x = b0; x < b1; ++x) local += (double)e[x];
   double tot_scan;
-  const double before = block_excl_scan<double>(local, dred, &tot_scan);
+  const double before = block_excl_scan<double>(local, dred, tot_scan);
   if (tid == 0) s_kstar = nK;
   __syncthreads();
   const double thr = (double)t * tot;
@@ -325,8 +329,8 @@ __global__ void __launch_bounds__(kSelThreads) block_select_kernel(
     else cnt2 += flag[x];
   }
   int total_kept, total_kept2;
-  int pos = block_excl_scan<int>(cnt, ired, &total_kept);
-  int pos2 = block_excl_scan<int>(cnt2, ired, &total_kept2);
+  int pos = block_excl_scan<int>(cnt, ired, total_kept);
+  int pos2 = block_excl_scan<int>(cnt2, ired, total_kept2);
   for (int x = b0; x < b1; ++x) {
     if (!flag[x]) continue;
     if (x < nA) idx_out[pos++] = x;
