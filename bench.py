@@ -538,14 +538,11 @@ def run_gpu(args, shape, rank, world, local):
     t_kind = "burst" if at_max else "sustained"
     t_peak = peaks["bf16_tflops"] if at_max else peaks["bf16_tflops_sustained"]
     host_gbs = measure_host_link(dev) if shape.host_pages else None
-    # pages of a multiple of 64 rows: the step gathers and projects the history in one
-    # pass (gather_project) and the step's own projection covers the chunk's rows only
-    early = shape.P_tok % 64 == 0
     kernel_work = {
         # the fused attention kernel: selected-block FLOPs of the sparse branch plus the
         # useful FLOPs of the linear branch (the split-precision extra products not counted)
         "attention_merge": ("tensor", f_sparse + w["lin_attn_flops"]),
-        "linformer_proj": ("tensor", w["proj_chunk_flops"] if early else w["proj_flops"]),
+        "linformer_proj": ("tensor", w["proj_flops"]),
         "gather_project": ("tensor", w["proj_hist_flops"]),
         "gather": ("host-link", w["gather_bytes"] / 2) if shape.host_pages else ("hbm", w["gather_bytes"]),
         "pool": ("hbm", w["pool_bytes"]),

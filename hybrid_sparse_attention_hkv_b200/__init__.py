@@ -162,6 +162,17 @@ def hsa_status_clear(ws, stream=None):
     _check(load_library().hsa_status_clear(_p(ws), _stream(stream)), "hsa_status_clear")
 
 
+def wait_report(ws) -> dict:
+    """The workspace header's record of a bounded wait that ran out: the status word,
+    the ran-out flag, and the site (kind << 24 | warp << 16 | tile, 0 if none) and CTA
+    of the first such wait.  Reads the header after synchronising the device."""
+    torch.cuda.synchronize(ws.device)
+    w = ws[:24].view(torch.int32).cpu().tolist()
+    site = w[4]
+    return {"status": w[0], "ran_out": w[1], "site": site, "kind": site >> 24, "warp": (site >> 16) & 0xFF,
+            "tile": site & 0xFFFF, "cta": w[5]}
+
+
 def hsa_status_read(ws, stream=None) -> int:
     st = ctypes.c_int(0)
     _check(load_library().hsa_status_read(_p(ws), _stream(stream), ctypes.byref(st)), "hsa_status_read")

@@ -77,7 +77,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Workspace layout shared by every entry point (offsets in bytes).
 struct Layout {
-  size_t status = 0, colpart = 0, q128 = 0, q64 = 0, kq64 = 0, kc128 = 0;
+  size_t status = 0, colpart = 0, q128 = 0, q64 = 0, kq64 = 0, kc128 = 0, bscores = 0;
   size_t inter_idx = 0, inter_cnt = 0, intra_idx = 0, intra_cnt = 0;
   size_t units = 0, n_units = 0, tile_done = 0, part_o = 0, part_ml = 0, part_lin = 0, attn_end = 0;
   int max_units = 0, max_slots = 0;
@@ -103,6 +103,7 @@ Layout make_layout(int H, int d, int Lq, long long Lc, int r) {
   L.q64 = take(nQ64 * hd * 4);
   L.kq64 = take(nQ64 * hd * 4);
   L.kc128 = take(nKc * hd * 4);
+  L.bscores = take(hsa::block_scores_floats(H, Lq, Lc) * 4);
   L.inter_idx = take((size_t)H * nQ64 * nKc * 4);  // nQ64 rows: room for the joint mode's per-64-row lists
   L.inter_cnt = take((size_t)H * nQ64 * 4);
   L.intra_idx = take((size_t)H * nQ64 * nQ64 * 4);
@@ -262,7 +263,9 @@ hsa_status_t hsa_workspace_size(const hsa_config_t* cfg, int NP, int P_tok, size
 
 hsa_status_t hsa_status_clear(void* ws, hsa_stream_t stream) {
   if (!ws) return fail(HSA_ERR_WORKSPACE, "hsa_status_clear: workspace is NULL");
-  cudaError_t e = cudaMemsetAsync(ws, 0, 2 * sizeof(int), stream);  // status and the ran-out flag
+  // the status, the ran-out flag and the first ran-out site (the wait limit stays)
+  cudaError_t e = cudaMemsetAsync(ws, 0, 2 * sizeof(int), stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(static_cast<char*>(ws) + 4 * sizeof(int), 0, 2 * sizeof(int), stream);
   return e == cudaSuccess ? HSA_OK : fail(HSA_ERR_CUDA, "hsa_status_clear: %s", cudaGetErrorString(e));
 }
 
@@ -597,8 +600,8 @@ static hsa_status_t run_block_select(const hsa_config_t* cfg, const Layout& L, c
                                       kbar128 ? nullptr : kc128, stream));
   HSA_LAUNCH("block_select", hsa::launch_block_select(q128, kc128, q64, kq64, tau, cfg->H, cfg->d, cfg->Lq, cfg->Lc,
                                                       scale_of(cfg), cfg->select_mode == HSA_SELECT_JOINT,
-                                                      sel.inter_idx, sel.inter_cnt, sel.intra_idx, sel.intra_cnt,
-                                                      stream));
+                                                      at<float>(ws, L.bscores), sel.inter_idx, sel.inter_cnt,
+                                                      sel.intra_idx, sel.intra_cnt, stream));
   return HSA_OK;
 }
 

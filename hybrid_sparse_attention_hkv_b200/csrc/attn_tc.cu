@@ -37,11 +37,13 @@
 //               when it grows by more than 2^8; finally o_s = O_s / l_s,
 //               o_l = O_l / l_l, out = g o_s + (1 - g) o_l, stored.
 // The tensor core computes S_{j+1} while the softmax warps work on S_j.
-// Every wait is bounded (HSA_ERR_TIMEOUT in the workspace status on expiry).  The
-// softmax warps' per-tile waits are per-lane (a warp-wide vote after each of them
-// cost 7% of the kernel's time); the MMA warp, which issues with elect.sync, and the
-// waits before the first and after the last tile, where the warps go on to
-// warp-collective TMEM access and teardown, take the warp's common answer.
+// Every wait is bounded (HSA_ERR_TIMEOUT in the workspace status on expiry) and names
+// its site (kind << 24 | warp << 16 | tile), recorded for the first wait of the
+// workspace that runs out.  The softmax warps' per-tile waits are per-lane (a
+// warp-wide vote after each of them cost 7% of the kernel's time); the producers, the
+// MMA warp, which issues with elect.sync, and the waits before the first and after the
+// last tile, where the warps go on to warp-collective TMEM access and teardown, take
+// the warp's common answer.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -60,6 +62,10 @@ constexpr int kTcThreads = 224;  // 7 warps
 constexpr int kKStages = 3;      // K ring: a slot frees as soon as its S MMA completes
 constexpr int kVStages = 2;      // V ring: a slot frees when its P.V MMA completes
 constexpr int kRegionBytes = 128 * 128;  // one [128 rows x 64 bf16] swizzled region
+// wait sites (header word 4 of the first wait that runs out: kind << 24 | warp << 16 | tile)
+constexpr int kSiteKEmpty = 1, kSiteVEmpty = 2, kSiteQ = 3, kSiteKFull = 4, kSitePFull = 6, kSiteVFull = 7,
+              kSiteSFull = 8, kSiteODone = 13;
+__device__ __forceinline__ int wait_site(int kind, int warp, int j) { return (kind << 24) | (warp << 16) | (j & 0xFFFF); }
 
 struct TcMaps {
   CUtensorMap q, kc, vc, kq, vq, ekhi, eklo, fvhi, fvlo;
@@ -444,7 +450,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     for (int j = 0; j < T; ++j) {
       const int s = j % kKStages;
-      if (!mbar_wait(&bar_k_empty[s], ((j / kKStages) & 1) ^ 1, status, wlim)) break;
+      if (!mbar_wait_warp(&bar_k_empty[s], ((j / kKStages) & 1) ^ 1, status, wlim, wait_site(kSiteKEmpty, warp, j)))
+        break;
       if (lane == 0) {
         const int code = tile_at(j);
         const int type = tile_type(code);
@@ -478,7 +485,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ------------------------------------------------------------ V producer
     for (int j = 0; j < T; ++j) {
       const int s = j % kVStages;
-      if (!mbar_wait(&bar_v_empty[s], ((j / kVStages) & 1) ^ 1, status, wlim)) break;
+      if (!mbar_wait_warp(&bar_v_empty[s], ((j / kVStages) & 1) ^ 1, status, wlim, wait_site(kSiteVEmpty, warp, j)))
+        break;
       if (lane == 0) {
         const int code = tile_at(j);
         const int type = tile_type(code);
@@ -510,7 +518,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    bool ok = mbar_wait_warp(&bar_q, 0, status, wlim);
+    bool ok = mbar_wait_warp(&bar_q, 0, status, wlim, wait_site(kSiteQ, warp, 0));
     tc_fence_after();
     const uint64_t qd = sdesc_sw128(smem_u32(sQ), 16, 1024);
     // The warp stays converged: waits take the warp's common answer, tile codes and
@@ -519,7 +527,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // core; only P, written to TMEM by the softmax warps, needs the tcgen05 fence.
     auto issue_s = [&](int j) -> bool {
       const int s = j % kKStages;
-      if (!mbar_wait_warp(&bar_k_full[s], (j / kKStages) & 1, status, wlim)) return false;
+      if (!mbar_wait_warp(&bar_k_full[s], (j / kKStages) & 1, status, wlim, wait_site(kSiteKFull, warp, j))) return false;
       const int code = tile_at(j);
       const uint64_t kd = sdesc_sw128(smem_u32(sK + s * Lay::kKVBytes), 16, 1024);
       const uint32_t tS = tmem + (j & 1) * 128;
@@ -538,9 +546,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (ok && T > 0) ok = issue_s(0);
     for (int j = 0; ok && j < T; ++j) {
       if (j + 1 < T && !issue_s(j + 1)) break;
-      if (!mbar_wait_warp(&bar_p_full[j & 1], (j >> 1) & 1, status, wlim)) break;
+      if (!mbar_wait_warp(&bar_p_full[j & 1], (j >> 1) & 1, status, wlim, wait_site(kSitePFull, warp, j))) break;
       const int sv = j % kVStages;
-      if (!mbar_wait_warp(&bar_v_full[sv], (j / kVStages) & 1, status, wlim)) break;
+      if (!mbar_wait_warp(&bar_v_full[sv], (j / kVStages) & 1, status, wlim, wait_site(kSiteVFull, warp, j))) break;
       tc_fence_after();
       const int code = tile_at(j);
       const uint32_t v_base = smem_u32(sV + sv * Lay::kKVBytes);
@@ -574,7 +582,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     bool ok = true;
     for (int j = 0; j < T; ++j) {
       const int b = j & 1;
-      if (!mbar_wait(&bar_s_full[b], (j >> 1) & 1, status, wlim)) {
+      if (!mbar_wait(&bar_s_full[b], (j >> 1) & 1, status, wlim, wait_site(kSiteSFull, warp, j))) {
         ok = false;
         break;
       }
@@ -621,7 +629,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // O holds the P.V products of tiles 0..j-1 once the last of them has completed
         // (P.V of tile j cannot have started: it waits for this P).  Without a rescale
         // nothing here touches O, and the wait is skipped.
-        if (j > 0 && !mbar_wait(&bar_o_done, (j - 1) & 1, status, wlim)) {
+        if (j > 0 && !mbar_wait(&bar_o_done, (j - 1) & 1, status, wlim, wait_site(kSiteODone, warp, j))) {
           ok = false;
           break;
         }

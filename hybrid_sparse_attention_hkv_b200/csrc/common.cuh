@@ -20,6 +20,8 @@ constexpr int kBlockIntra = 64;
 //              own, so a protocol that stalls ends in one wait limit, not one per wait
 //   uint32[2]  kWaitTag when word 3 holds a limit set by hsa_set_wait_limit
 //   uint32[3]  limit of every bounded device wait, in microseconds
+//   int32 [4]  site of the first wait that ran out (0: none, or a wait without a site)
+//   int32 [5]  CTA index of that wait
 constexpr uint32_t kWaitTag = 0x54494157u;  // "WAIT"
 constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
 

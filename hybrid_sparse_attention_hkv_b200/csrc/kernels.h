@@ -73,11 +73,13 @@ constexpr int kMaxSelBlocks = 8192;  // blocks per selection row (inter: ceil(Lc
 cudaError_t launch_pool(const uint16_t* Q, const uint16_t* Kq, const uint16_t* Kc, int H, int d, int Lq,
                         long long Lc, float* q128, float* q64, float* kq64, float* kc128, cudaStream_t s);
 // joint: one softmax per 64-row query block over its Kc and Kq blocks (inter rows per
-// 64-row query block); else the two maps separately.
+// 64-row query block); else the two maps separately.  scores: block_scores_floats()
+// floats of scratch for the rows' block scores.
+size_t block_scores_floats(int H, int Lq, long long Lc);
 cudaError_t launch_block_select(const float* q128, const float* kc128, const float* q64, const float* kq64,
                                 const float* tau, int H, int d, int Lq, long long Lc, float scale, bool joint,
-                                int32_t* inter_idx, int32_t* inter_cnt, int32_t* intra_idx, int32_t* intra_cnt,
-                                cudaStream_t s);
+                                float* scores, int32_t* inter_idx, int32_t* inter_cnt, int32_t* intra_idx,
+                                int32_t* intra_cnt, cudaStream_t s);
 
 // ---------------------------------------------------------------- attn_tc.cu / plan.cu
 // The attention kernel runs one CTA per work unit: a segment of the key-tile list

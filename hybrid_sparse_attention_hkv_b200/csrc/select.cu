@@ -5,6 +5,8 @@
 #include <float.h>
 #include <limits.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -95,6 +97,71 @@ cudaError_t launch_pool(const uint16_t* Q, const uint16_t* Kq, const uint16_t* K
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ block scores
+// s[h][i][j] = scale * qbar_i . kbar_j for every selection row i of one map and every
+// key block j (j < nA from kA, the rest from kB), fp32, summed over d in order.  One
+// CTA per (64 key blocks, 32 rows, head): both tiles pass through shared memory 32
+// dimensions at a time, so a key block's mean is read once per 32 rows rather than
+// once per row.
+constexpr int kScoreRows = 32, kScoreKeys = 64, kScoreChunk = 32;
+
+template <int D>
+__global__ void __launch_bounds__(256) block_scores_kernel(const float* __restrict__ q, int R,
+                                                           const float* __restrict__ kA, int nA,
+                                                           const float* __restrict__ kB, int K, int H, float scale,
+                                                           float* __restrict__ out) {
+  __shared__ float sq[kScoreRows][kScoreChunk + 1];
+  __shared__ float sk[kScoreKeys][kScoreChunk + 1];
+  const int h = blockIdx.z;
+  const int i0 = blockIdx.y * kScoreRows, j0 = blockIdx.x * kScoreKeys;
+  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;  // rows 2 ty, 2 ty + 1; keys tx + 16 u
+  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  for (int c0 = 0; c0 < D; c0 += kScoreChunk) {
+    for (int t = threadIdx.x; t < kScoreRows * kScoreChunk; t += 256) {
+      const int r = t / kScoreChunk, c = t % kScoreChunk, i = i0 + r;
+      sq[r][c] = i < R ? q[((long long)i * H + h) * D + c0 + c] : 0.f;
+    }
+    for (int t = threadIdx.x; t < kScoreKeys * kScoreChunk; t += 256) {
+      const int r = t / kScoreChunk, c = t % kScoreChunk, j = j0 + r;
+      float v = 0.f;
+      if (j < nA) v = kA[((long long)j * H + h) * D + c0 + c];
+      else if (j < K) v = kB[((long long)(j - nA) * H + h) * D + c0 + c];
+      sk[r][c] = v;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int c = 0; c < kScoreChunk; ++c) {
+      const float a0 = sq[2 * ty][c], a1 = sq[2 * ty + 1][c];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float b = sk[tx + 16 * u][c];
+        acc[0][u] = fmaf(a0, b, acc[0][u]);
+        acc[1][u] = fmaf(a1, b, acc[1][u]);
+      }
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int rr = 0; rr < 2; ++rr) {
+    const int i = i0 + 2 * ty + rr;
+    if (i >= R) continue;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = j0 + tx + 16 * u;
+      if (j < K) out[((long long)h * R + i) * K + j] = acc[rr][u] * scale;
+    }
+  }
+}
+
+template <int D>
+void launch_scores(const float* q, int R, const float* kA, int nA, const float* kB, int K, int H, float scale,
+                   float* out, cudaStream_t s) {
+  if (R == 0 || K == 0) return;
+  const dim3 grid((unsigned)((K + kScoreKeys - 1) / kScoreKeys), (unsigned)((R + kScoreRows - 1) / kScoreRows),
+                  (unsigned)H);
+  block_scores_kernel<D><<<grid, 256, 0, s>>>(q, R, kA, nA, kB, K, H, scale, out);
+}
+
 // ------------------------------------------------------------------ block selection
 // One CTA per selection row (head h, query block i, map inter|intra; in joint mode
 // one row per (head, 64-row query block) over the Kc blocks followed by the Kq
@@ -143,14 +210,11 @@ __device__ T block_excl_scan(T v, T* warp_tot, T& total) {
   return r;
 }
 
-template <int D>
 __global__ void __launch_bounds__(kSelThreads) block_select_kernel(
-    const float* __restrict__ q128, const float* __restrict__ kc128, const float* __restrict__ q64,
-    const float* __restrict__ kq64, const float* __restrict__ tau, int H, int nQ128, int nKc, int nQ64, int nKq,
-    float scale, bool joint, int32_t* __restrict__ inter_idx, int32_t* __restrict__ inter_cnt,
-    int32_t* __restrict__ intra_idx, int32_t* __restrict__ intra_cnt) {
+    const float* __restrict__ scores, const float* __restrict__ tau, int H, int nQ128, int nKc, int nQ64, int nKq,
+    bool joint, int32_t* __restrict__ inter_idx, int32_t* __restrict__ inter_cnt, int32_t* __restrict__ intra_idx,
+    int32_t* __restrict__ intra_cnt) {
   extern __shared__ __align__(16) unsigned char smraw[];
-  __shared__ float qv[D];
   __shared__ double dred[40];
   __shared__ int ired[40];
   __shared__ float fred[40];
@@ -158,12 +222,10 @@ __global__ void __launch_bounds__(kSelThreads) block_select_kernel(
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   int row = blockIdx.x;
-  // the row's keys are kbA[0 .. nA) followed by kbB[0 .. nK - nA); kept ids < nA go
-  // to idx_out / cnt_out, the others (minus nA) to idx_out2 / cnt_out2
+  // the row's keys: nK scores (block_scores_kernel); kept ids < nA go to idx_out /
+  // cnt_out, the others (minus nA) to idx_out2 / cnt_out2
   int h, i, nK, nA;
-  const float* qb;
-  const float* kbA;
-  const float* kbB = nullptr;
+  const float* srow;
   int32_t* idx_out;
   int32_t* cnt_out;
   int32_t* idx_out2 = nullptr;
@@ -173,9 +235,7 @@ __global__ void __launch_bounds__(kSelThreads) block_select_kernel(
     i = row % nQ64;
     nA = nKc;
     nK = nKc + nKq;
-    qb = q64 + ((long long)i * H + h) * D;
-    kbA = kc128;
-    kbB = kq64;
+    srow = scores + ((long long)h * nQ64 + i) * nK;
     idx_out = inter_idx + ((long long)h * nQ64 + i) * nKc;
     cnt_out = inter_cnt + (long long)h * nQ64 + i;
     idx_out2 = intra_idx + ((long long)h * nQ64 + i) * nKq;
@@ -184,8 +244,7 @@ __global__ void __launch_bounds__(kSelThreads) block_select_kernel(
     h = row / nQ128;
     i = row % nQ128;
     nK = nA = nKc;
-    qb = q128 + ((long long)i * H + h) * D;
-    kbA = kc128;
+    srow = scores + ((long long)h * nQ128 + i) * nKc;
     idx_out = inter_idx + ((long long)h * nQ128 + i) * nKc;
     cnt_out = inter_cnt + (long long)h * nQ128 + i;
   } else {
@@ -193,8 +252,7 @@ __global__ void __launch_bounds__(kSelThreads) block_select_kernel(
     h = row / nQ64;
     i = row % nQ64;
     nK = nA = nKq;
-    qb = q64 + ((long long)i * H + h) * D;
-    kbA = kq64;
+    srow = scores + (long long)H * nQ128 * nKc + ((long long)h * nQ64 + i) * nKq;
     idx_out = intra_idx + ((long long)h * nQ64 + i) * nKq;
     cnt_out = intra_cnt + (long long)h * nQ64 + i;
   }
@@ -223,28 +281,7 @@ __global__ void __launch_bounds__(kSelThreads) block_select_kernel(
   int* id = reinterpret_cast<int*>(e + NB2);    // [NB2]
   int* flag = id + NB2;                          // [NB2]
 
-  for (int c = tid; c < D; c += kSelThreads) qv[c] = qb[c];
-  __syncthreads();
-  // scores: each warp takes 8 blocks at a time so that their loads are in flight together
-  constexpr int kB = 8;
-  for (int j0 = warp * kB; j0 < nK; j0 += (kSelThreads / 32) * kB) {
-    float acc[kB];
-#pragma unroll
-    for (int u = 0; u < kB; ++u) {
-      acc[u] = 0.f;
-      const int j = j0 + u;
-      if (j < nK) {
-        const float* k = j < nA ? kbA + ((long long)j * H + h) * D : kbB + ((long long)(j - nA) * H + h) * D;
-#pragma unroll
-        for (int c = lane; c < D; c += 32) acc[u] = fmaf(qv[c], __ldg(k + c), acc[u]);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kB; ++u) {
-      const float s = warp_sum(acc[u]);
-      if (lane == 0 && j0 + u < nK) e[j0 + u] = s * scale;
-    }
-  }
+  for (int j = tid; j < nK; j += kSelThreads) e[j] = srow[j];
   __syncthreads();
   // row max
   float m = -INFINITY;
@@ -342,31 +379,43 @@ __global__ void __launch_bounds__(kSelThreads) block_select_kernel(
   }
 }
 
+size_t block_scores_floats(int H, int Lq, long long Lc) {
+  const long long nQ128 = (Lq + 127) / 128, nQ64 = (Lq + 63) / 64, nKc = (Lc + 127) / 128;
+  const long long separate = nQ128 * nKc + nQ64 * nQ64, joint = nQ64 * (nKc + nQ64);
+  return (size_t)H * (size_t)(separate > joint ? separate : joint);
+}
+
 cudaError_t launch_block_select(const float* q128, const float* kc128, const float* q64, const float* kq64,
                                 const float* tau, int H, int d, int Lq, long long Lc, float scale, bool joint,
-                                int32_t* inter_idx, int32_t* inter_cnt, int32_t* intra_idx, int32_t* intra_cnt,
-                                cudaStream_t s) {
+                                float* scores, int32_t* inter_idx, int32_t* inter_cnt, int32_t* intra_idx,
+                                int32_t* intra_cnt, cudaStream_t s) {
   const int nQ128 = (Lq + 127) / 128, nQ64 = (Lq + 63) / 64;
   const int nKc = (int)((Lc + 127) / 128), nKq = nQ64;
+  // the scores of every row: [H][nQ64][nKc + nKq] (joint), or [H][nQ128][nKc] followed
+  // by [H][nQ64][nKq] (separate)
+  auto scores_of = [&](auto tag) {
+    constexpr int D = decltype(tag)::value;
+    if (joint) {
+      launch_scores<D>(q64, nQ64, kc128, nKc, kq64, nKc + nKq, H, scale, scores, s);
+    } else {
+      launch_scores<D>(q128, nQ128, kc128, nKc, kc128, nKc, H, scale, scores, s);
+      launch_scores<D>(q64, nQ64, kq64, nKq, kq64, nKq, H, scale, scores + (long long)H * nQ128 * nKc, s);
+    }
+  };
+  if (d == 128) scores_of(std::integral_constant<int, 128>());
+  else scores_of(std::integral_constant<int, 64>());
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   int nmax = joint ? nKc + nKq : (nKc > nKq ? nKc : nKq), NB2 = 1;
   while (NB2 < nmax) NB2 <<= 1;
   const size_t smem = (size_t)NB2 * 12;
   const int grid = joint ? H * nQ64 : H * (nQ128 + nQ64);
-  if (d == 128) {
-    if (smem > 48 * 1024) {
-      cudaError_t e = cudaFuncSetAttribute(block_select_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-    }
-    block_select_kernel<128><<<grid, kSelThreads, smem, s>>>(q128, kc128, q64, kq64, tau, H, nQ128, nKc, nQ64, nKq,
-                                                              scale, joint, inter_idx, inter_cnt, intra_idx, intra_cnt);
-  } else {
-    if (smem > 48 * 1024) {
-      cudaError_t e = cudaFuncSetAttribute(block_select_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-    }
-    block_select_kernel<64><<<grid, kSelThreads, smem, s>>>(q128, kc128, q64, kq64, tau, H, nQ128, nKc, nQ64, nKq,
-                                                             scale, joint, inter_idx, inter_cnt, intra_idx, intra_cnt);
+  if (smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(block_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
   }
+  block_select_kernel<<<grid, kSelThreads, smem, s>>>(scores, tau, H, nQ128, nKc, nQ64, nKq, joint, inter_idx,
+                                                      inter_cnt, intra_idx, intra_cnt);
   return cudaGetLastError();
 }
 

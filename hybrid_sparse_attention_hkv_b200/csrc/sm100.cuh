@@ -57,8 +57,11 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
       : "memory");
   return ok != 0;
 }
-// Bounded wait for the phase with the given parity to complete.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status, uint64_t limit_ns) {
+// Bounded wait for the phase with the given parity to complete.  `site` (nonzero,
+// chosen by the caller) names the wait: the first wait of a workspace that runs out
+// records its site and CTA index in header words 4 and 5.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* status, uint64_t limit_ns,
+                                          int site = 0) {
   if (mbar_try_wait_sleep(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   do {
@@ -67,14 +70,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
     if (status != nullptr && *reinterpret_cast<volatile int*>(status + 1) != 0) return false;
   } while (global_ns() - t0 < limit_ns);
   set_status(status, HSA_ERR_TIMEOUT);
-  if (status != nullptr) atomicExch(status + 1, 1);
+  if (status != nullptr) {
+    if (site != 0 && atomicCAS(status + 4, 0, site) == 0) atomicExch(status + 5, (int)blockIdx.x);
+    atomicExch(status + 1, 1);
+  }
   return false;
 }
 
 // The same wait for a whole warp: every lane waits, and the warp agrees on the
 // outcome (one lane's timeout counts for all), so the lanes never diverge.
-__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int* status, uint64_t limit_ns) {
-  const bool ok = mbar_wait(bar, parity, status, limit_ns);
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int* status, uint64_t limit_ns,
+                                               int site = 0) {
+  const bool ok = mbar_wait(bar, parity, status, limit_ns, site);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -193,6 +200,12 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
       "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
+}
+// 8 consecutive columns.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
 }
 // Load 16 consecutive columns of this thread's lane and wait for them in the same
 // asm statement, so no use of r[] can be scheduled before the data has arrived.

@@ -14,6 +14,8 @@
 namespace hsa {
 namespace {
 
+constexpr int kSelftestSite = 0x7E << 24;
+
 __global__ void set_wait_limit_kernel(int* header, uint32_t limit_us) {
   uint32_t* w = reinterpret_cast<uint32_t*>(header);
   w[3] = limit_us;
@@ -26,8 +28,9 @@ __global__ void wait_selftest_kernel(int* status, unsigned long long* waited_ns)
   sm100::mbar_init(&bar, 1);
   sm100::fence_barrier_init();
   const uint64_t t0 = sm100::global_ns();
-  // phase 0 never completes: nothing arrives on the barrier
-  const bool ok = sm100::mbar_wait(&bar, 0, status, wait_limit_ns(status));
+  // phase 0 never completes: nothing arrives on the barrier.  The wait's site is
+  // kSelftestSite, so that the header's record of it can be checked.
+  const bool ok = sm100::mbar_wait(&bar, 0, status, wait_limit_ns(status), kSelftestSite);
   if (waited_ns) *waited_ns = sm100::global_ns() - t0;
   if (ok) set_status(status, HSA_ERR_DEVICE);  // cannot happen: the phase has no arrivals
 }

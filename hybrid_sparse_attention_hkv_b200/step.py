@@ -11,8 +11,8 @@ from __future__ import annotations
 
 import torch
 
-from . import (FWD_HISTORY, FWD_SELECTED, SelectionBuffers, hkv_block_means_from_pages, hkv_gather,
-               hkv_gather_project, hkv_page_block_sums, hkv_page_summary, hkv_select_pages, hkv_select_prompt,
+from . import (FWD_SELECTED, SelectionBuffers, hkv_block_means_from_pages, hkv_gather,
+               hkv_page_block_sums, hkv_page_summary, hkv_select_pages, hkv_select_prompt,
                hsa_block_select, hsa_forward, hsa_forward_ex, hsa_forward_reuse, hsa_prepare_history,
                hsa_workspace_size, make_config)
 
@@ -89,20 +89,19 @@ class HkvHsaStep:
                         self.kbar128, self.selection, ef_head_stride)
             return dst
         # the cache's block means from the pages' sums; then, on its own stream, the
-        # gather together with the history's Linformer products (one pass over the
-        # pages) while this stream pools the chunk and selects blocks; then the chunk's
-        # own projection, the plan and the attention
+        # gather (HBM-bound) while this stream pools the chunk and selects blocks; then
+        # the Linformer projection (beside the plan) and the attention
         main = torch.cuda.current_stream()
         hkv_block_means_from_pages(self.sums64, self.sel, self.Kp, self.P_tok, self.H, self.d, self.kbar128, self.ws)
         self.ev_sel.record(main)
         self.gather_stream.wait_event(self.ev_sel)
-        hkv_gather_project(self.cfg, self.page_k_ptrs, self.page_v_ptrs, self.sel, self.Kp, self.P_tok, E, F,
-                           self.Kc, self.Vc, self.ws, ef_head_stride, stream=self.gather_stream)
+        hkv_gather(self.page_k_ptrs, self.page_v_ptrs, self.sel, self.Kp, self.P_tok, self.H, self.d,
+                   self.Kc, self.Vc, self.ws, stream=self.gather_stream)
         self.ev_gathered.record(self.gather_stream)
         hsa_block_select(self.cfg, Q, self.Kc, Kq, tau, self.selection, self.ws, self.kbar128)
         main.wait_event(self.ev_gathered)
         hsa_forward_ex(self.cfg, Q, self.Kc, self.Vc, Kq, Vq, tau, gate_logit, E, F, dst, self.ws, self.selection,
-                       FWD_SELECTED | FWD_HISTORY, ef_head_stride=ef_head_stride)
+                       FWD_SELECTED, ef_head_stride=ef_head_stride)
         return dst
 
     # ------------------------------------------------------------ multi-step reuse
@@ -116,12 +115,6 @@ class HkvHsaStep:
         self._retrieve(Q, cand)
         if self.store is not None:
             self.store.fetch(self.sel, self.ws)
-        if self.early:
-            hkv_block_means_from_pages(self.sums64, self.sel, self.Kp, self.P_tok, self.H, self.d, self.kbar128,
-                                       self.ws)
-            hkv_gather_project(self.cfg, self.page_k_ptrs, self.page_v_ptrs, self.sel, self.Kp, self.P_tok, E, F,
-                               self.Kc, self.Vc, self.ws, ef_head_stride)
-            return
         hkv_gather(self.page_k_ptrs, self.page_v_ptrs, self.sel, self.Kp, self.P_tok, self.H, self.d,
                    self.Kc, self.Vc, self.ws, self.kbar128)
         hsa_prepare_history(self.cfg, self.Kc, self.Vc, E, F, self.ws, ef_head_stride)

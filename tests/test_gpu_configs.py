@@ -11,6 +11,7 @@ import numpy as np
 import pytest
 import torch
 
+import hybrid_sparse_attention_hkv_b200 as hsa
 import oracle
 import synth
 from hsa_testlib import (DeviceStep, assert_close, bits_of, check_pages, check_selection_both, sample_rows,
@@ -30,6 +31,7 @@ def run(request):
     ds = DeviceStep(shape, synth.seed_of(i))
     ds.run()
     torch.cuda.synchronize()
+    assert hsa.hsa_status_read(ds.step.ws) == 0, hsa.wait_report(ds.step.ws)
     yield i, ds
     ds.close()
     del ds

@@ -379,6 +379,8 @@ def test_bounded_wait_times_out_and_context_stays_usable():
     assert hsa.hsa_status_read(ws) == 5  # HSA_ERR_TIMEOUT
     ns = int(waited.item())
     assert 3_000_000 <= ns < 500_000_000, ns
+    rep = hsa.wait_report(ws)  # the self-test's wait names site kind 0x7E, CTA 0
+    assert rep["ran_out"] == 1 and rep["kind"] == 0x7E and rep["cta"] == 0, rep
     # the ran-out flag is now set: under a 1 s limit, the next wait gives up at its
     # first unsuccessful poll instead of running out on its own
     hsa.hsa_set_wait_limit(ws, 1_000_000)
@@ -388,6 +390,8 @@ def test_bounded_wait_times_out_and_context_stays_usable():
     assert ns < 100_000_000, ns
     # the context is usable: a fused forward under a generous limit completes with status 0
     hsa.hsa_status_clear(ws)
+    rep = hsa.wait_report(ws)
+    assert rep["status"] == 0 and rep["ran_out"] == 0 and rep["site"] == 0, rep
     hsa.hsa_set_wait_limit(ws, 200_000)  # 200 ms
     shape = synth.StepShape("wait", H=H, d=d, frames=1, F_tok=Lq, page_frames=1, page_tok=8, NP=1, Kp=1, r=64)
     x = synth.make_inputs(shape, 33)
