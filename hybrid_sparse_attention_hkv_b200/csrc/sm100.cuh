@@ -57,6 +57,8 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
       : "memory");
   return ok != 0;
 }
+constexpr uint64_t kFlagAfterNs = 50000;  // 50 us
+
 // Bounded wait for the phase with the given parity to complete.  `site` (nonzero,
 // chosen by the caller) names the wait: the first wait of a workspace that runs out
 // records its site and CTA index in header words 4 and 5.
@@ -64,11 +66,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
                                           int site = 0) {
   if (mbar_try_wait_sleep(bar, parity)) return true;
   const uint64_t t0 = global_ns();
+  uint64_t waited = 0;
   do {
     if (mbar_try_wait_sleep(bar, parity)) return true;
-    // another wait of this workspace already ran out: give up now
-    if (status != nullptr && *reinterpret_cast<volatile int*>(status + 1) != 0) return false;
-  } while (global_ns() - t0 < limit_ns);
+    waited = global_ns() - t0;
+    // another wait of this workspace already ran out: give up.  Checked only once this
+    // wait has lasted kFlagAfterNs, far longer than any hand-over of a running pipeline,
+    // so that the flag's load never delays a wait that is about to complete.
+    if (waited > kFlagAfterNs && status != nullptr && *reinterpret_cast<volatile int*>(status + 1) != 0)
+      return false;
+  } while (waited < limit_ns);
   set_status(status, HSA_ERR_TIMEOUT);
   if (status != nullptr) {
     if (site != 0 && atomicCAS(status + 4, 0, site) == 0) atomicExch(status + 5, (int)blockIdx.x);

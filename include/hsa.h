@@ -132,8 +132,8 @@ hsa_status_t hsa_status_read(const void* ws, hsa_stream_t stream, int* status);
  * (hsa_status_clear leaves it).  A wait that runs out records HSA_ERR_TIMEOUT in
  * the status word, sets the workspace's ran-out flag, and its kernel drains its
  * copies and MMAs and exits.  While the flag is set (until hsa_status_clear),
- * every other wait of a kernel using `ws` gives up at its first unsuccessful
- * poll, so a stalled launch ends after one wait limit rather than one per CTA. */
+ * every other wait of a kernel using `ws` gives up once it has waited 50 us,
+ * so a stalled launch ends after one wait limit rather than one per CTA. */
 hsa_status_t hsa_set_wait_limit(void* ws, unsigned int limit_us, hsa_stream_t stream);
 
 /* Self-test of the timeout path (failure detection; the paper has no

@@ -381,8 +381,8 @@ def test_bounded_wait_times_out_and_context_stays_usable():
     assert 3_000_000 <= ns < 500_000_000, ns
     rep = hsa.wait_report(ws)  # the self-test's wait names site kind 0x7E, CTA 0
     assert rep["ran_out"] == 1 and rep["kind"] == 0x7E and rep["cta"] == 0, rep
-    # the ran-out flag is now set: under a 1 s limit, the next wait gives up at its
-    # first unsuccessful poll instead of running out on its own
+    # the ran-out flag is now set: under a 1 s limit, the next wait gives up after
+    # 50 us instead of running out on its own
     hsa.hsa_set_wait_limit(ws, 1_000_000)
     hsa.hsa_selftest_wait(ws, waited)
     assert hsa.hsa_status_read(ws) == 5
