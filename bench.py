@@ -33,18 +33,35 @@ METRIC = "HSA layer query-tokens/s + eff. TFLOP/s on 1 B200; % tensor/HBM roofli
 UNIT = "query-tokens/s"
 DEFAULT_WORKLOAD = 3
 
-# DRAM traffic per launch from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum),
-# keyed by kernel; valid only while that kernel's section of its source file (from its
-# section marker to the next one) is unchanged (sha256 prefix of the section).
 TRAFFIC = {
-    # ncu capture of the gather and the projection at the Wan-1.3B 480p workload
-    "gather": {"file": "hkv.cu", "section": "gather", "sha": "ea6010aad5d6ab04", "bytes": 306732800 + 251682048},
-    "linformer_proj": {"file": "proj_tc.cu", "section": "kernel", "sha": "75f5b56741b141bd",
-                       "bytes": 392642816 + 3636480},
-    # ncu capture of the attention kernel at the Wan-1.3B 480p workload
-    "attention_merge": {"file": "attn_tc.cu", "section": "kernel", "sha": "4cb6ffdabc6aea75",
-                        "bytes": 278155264 + 20598528},
+    # dram__bytes_read.sum + dram__bytes_write.sum of one launch, from an ncu capture at
+    # TRAFFIC_WORKLOAD (the summaries under profiles/); valid while the kernel's source
+    # section is unchanged (sha).  Another workload scales them by the KV the kernel
+    # streams ("kv": cached rows x heads x d; "kvq": all KV rows x heads x d).
+    "gather": {"file": "hkv.cu", "section": "gather", "sha": "ea6010aad5d6ab04", "bytes": 306730752 + 248329984,
+               "scale": "kv"},
+    "linformer_proj": {"file": "proj_tc.cu", "section": "kernel", "sha": "58b967d1bbf135b5",
+                       "bytes": 392641024 + 6231040, "scale": "kvq"},
+    "attention_merge": {"file": "attn_tc.cu", "section": "kernel", "sha": "fd734552ee4b2c0f",
+                        "bytes": 279298560 + 19572224, "scale": "kv"},
 }
+TRAFFIC_WORKLOAD = 1  # synth.SHAPES index of the captured workload (Wan-1.3B 480p)
+
+
+def traffic_of(name, shape):
+    """Per-launch DRAM traffic of kernel `name` at `shape`, or None (no capture, or the
+    kernel's source changed since the capture)."""
+    tr = TRAFFIC.get(name)
+    if not tr or tr["sha"] != section_sha(os.path.join(ROOT, "hybrid_sparse_attention_hkv_b200", "csrc", tr["file"]),
+                                          tr["section"]):
+        return None
+    import synth
+    ref = synth.SHAPES[TRAFFIC_WORKLOAD]
+    if tr["scale"] == "kv":
+        f = (shape.Lc * shape.H * shape.d) / (ref.Lc * ref.H * ref.d)
+    else:
+        f = ((shape.Lc + shape.Lq) * shape.H * shape.d) / ((ref.Lc + ref.Lq) * ref.H * ref.d)
+    return int(round(tr["bytes"] * f))
 
 
 SECTION_MARK = "// ------------------------------------------------------------------ "
@@ -544,7 +561,9 @@ def run_gpu(args, shape, rank, world, local):
         "attention_merge": ("tensor", f_sparse + w["lin_attn_flops"]),
         "linformer_proj": ("tensor", w["proj_flops"]),
         "gather_project": ("tensor", w["proj_hist_flops"]),
-        "gather": ("host-link", w["gather_bytes"] / 2) if shape.host_pages else ("hbm", w["gather_bytes"]),
+        # with a host tier the timed steps gather from the HBM slots the store keeps the
+        # selected pages in (host_tier reports the cold fetch over the host link)
+        "gather": ("hbm", w["gather_bytes"]),
         "pool": ("hbm", w["pool_bytes"]),
         "page_scores_partial": ("hbm", w["select_pages_bytes"]),
     }
@@ -572,19 +591,14 @@ def run_gpu(args, shape, rank, world, local):
                 ach = work / (avg_ms / 1e3) / 1e9
                 entry.update({"bound": "hbm", "achieved": ach, "unit": "GB/s", "peak": peaks["hbm_gbs"],
                               "frac": ach / peaks["hbm_gbs"]})
-        tr = TRAFFIC.get(name)
-        if tr and tr["sha"] == section_sha(os.path.join(ROOT, "hybrid_sparse_attention_hkv_b200", "csrc", tr["file"]),
-                                           tr["section"]):
-            entry["traffic"] = tr["bytes"]
+        tr = traffic_of(name, shape)
+        if tr is not None:
+            entry["traffic"] = tr
         kernels[name] = entry
     dom = max(kernels, key=lambda k: kernels[k]["share"])
     de = kernels[dom]
     bound = de.get("bound", "hbm")
-    traffic = None
-    tr = TRAFFIC.get(dom)
-    if tr and tr["sha"] == section_sha(os.path.join(ROOT, "hybrid_sparse_attention_hkv_b200", "csrc", tr["file"]),
-                                       tr["section"]):
-        traffic = tr["bytes"]
+    traffic = traffic_of(dom, shape)
     peak_source = {"tensor": f"{peaks['source']} bf16 {t_kind} (median SM clock {sm} of {smax} MHz)",
                    "hbm": f"{peaks['source']} HBM copy",
                    "host-link": "pinned host-to-device copy measured in this run"}.get(bound, "")

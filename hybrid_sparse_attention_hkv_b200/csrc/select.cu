@@ -100,46 +100,48 @@ cudaError_t launch_pool(const uint16_t* Q, const uint16_t* Kq, const uint16_t* K
 // ------------------------------------------------------------------ block scores
 // s[h][i][j] = scale * qbar_i . kbar_j for every selection row i of one map and every
 // key block j (j < nA from kA, the rest from kB), fp32, summed over d in order.  One
-// CTA per (64 key blocks, 32 rows, head): both tiles pass through shared memory 32
-// dimensions at a time, so a key block's mean is read once per 32 rows rather than
-// once per row.
-constexpr int kScoreRows = 32, kScoreKeys = 64, kScoreChunk = 32;
+// CTA per (64 key blocks, 32 rows, head): both tiles are loaded whole into shared
+// memory (16-byte loads, all in flight at once), so a key block's mean is read once
+// per 32 rows rather than once per row, in one memory round trip.
+constexpr int kScoreRows = 32, kScoreKeys = 64;
 
 template <int D>
 __global__ void __launch_bounds__(256) block_scores_kernel(const float* __restrict__ q, int R,
                                                            const float* __restrict__ kA, int nA,
                                                            const float* __restrict__ kB, int K, int H, float scale,
                                                            float* __restrict__ out) {
-  __shared__ float sq[kScoreRows][kScoreChunk + 1];
-  __shared__ float sk[kScoreKeys][kScoreChunk + 1];
+  extern __shared__ __align__(16) float sm_scores[];
+  constexpr int P = D + 4;  // row pitch (floats): 16-byte rows, rows 4 banks apart
+  float* sq = sm_scores;                   // [kScoreRows][P]
+  float* sk = sm_scores + kScoreRows * P;  // [kScoreKeys][P]
   const int h = blockIdx.z;
   const int i0 = blockIdx.y * kScoreRows, j0 = blockIdx.x * kScoreKeys;
+  constexpr int V = D / 4;  // float4 per row
+  for (int t = threadIdx.x; t < kScoreRows * V; t += 256) {
+    const int r = t / V, c = t % V, i = i0 + r;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i < R) v = __ldg(reinterpret_cast<const float4*>(q + ((long long)i * H + h) * D) + c);
+    *reinterpret_cast<float4*>(sq + r * P + 4 * c) = v;
+  }
+  for (int t = threadIdx.x; t < kScoreKeys * V; t += 256) {
+    const int r = t / V, c = t % V, j = j0 + r;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (j < nA) v = __ldg(reinterpret_cast<const float4*>(kA + ((long long)j * H + h) * D) + c);
+    else if (j < K) v = __ldg(reinterpret_cast<const float4*>(kB + ((long long)(j - nA) * H + h) * D) + c);
+    *reinterpret_cast<float4*>(sk + r * P + 4 * c) = v;
+  }
+  __syncthreads();
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;  // rows 2 ty, 2 ty + 1; keys tx + 16 u
   float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-  for (int c0 = 0; c0 < D; c0 += kScoreChunk) {
-    for (int t = threadIdx.x; t < kScoreRows * kScoreChunk; t += 256) {
-      const int r = t / kScoreChunk, c = t % kScoreChunk, i = i0 + r;
-      sq[r][c] = i < R ? q[((long long)i * H + h) * D + c0 + c] : 0.f;
-    }
-    for (int t = threadIdx.x; t < kScoreKeys * kScoreChunk; t += 256) {
-      const int r = t / kScoreChunk, c = t % kScoreChunk, j = j0 + r;
-      float v = 0.f;
-      if (j < nA) v = kA[((long long)j * H + h) * D + c0 + c];
-      else if (j < K) v = kB[((long long)(j - nA) * H + h) * D + c0 + c];
-      sk[r][c] = v;
-    }
-    __syncthreads();
 #pragma unroll 8
-    for (int c = 0; c < kScoreChunk; ++c) {
-      const float a0 = sq[2 * ty][c], a1 = sq[2 * ty + 1][c];
+  for (int c = 0; c < D; ++c) {
+    const float a0 = sq[(2 * ty) * P + c], a1 = sq[(2 * ty + 1) * P + c];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float b = sk[tx + 16 * u][c];
-        acc[0][u] = fmaf(a0, b, acc[0][u]);
-        acc[1][u] = fmaf(a1, b, acc[1][u]);
-      }
+    for (int u = 0; u < 4; ++u) {
+      const float b = sk[(tx + 16 * u) * P + c];
+      acc[0][u] = fmaf(a0, b, acc[0][u]);
+      acc[1][u] = fmaf(a1, b, acc[1][u]);
     }
-    __syncthreads();
   }
 #pragma unroll
   for (int rr = 0; rr < 2; ++rr) {
@@ -154,12 +156,19 @@ __global__ void __launch_bounds__(256) block_scores_kernel(const float* __restri
 }
 
 template <int D>
-void launch_scores(const float* q, int R, const float* kA, int nA, const float* kB, int K, int H, float scale,
-                   float* out, cudaStream_t s) {
-  if (R == 0 || K == 0) return;
+cudaError_t launch_scores(const float* q, int R, const float* kA, int nA, const float* kB, int K, int H, float scale,
+                          float* out, cudaStream_t s) {
+  if (R == 0 || K == 0) return cudaSuccess;
+  const size_t smem = (size_t)(kScoreRows + kScoreKeys) * (D + 4) * sizeof(float);
+  if (smem > 48 * 1024) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(block_scores_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
   const dim3 grid((unsigned)((K + kScoreKeys - 1) / kScoreKeys), (unsigned)((R + kScoreRows - 1) / kScoreRows),
                   (unsigned)H);
-  block_scores_kernel<D><<<grid, 256, 0, s>>>(q, R, kA, nA, kB, K, H, scale, out);
+  block_scores_kernel<D><<<grid, 256, smem, s>>>(q, R, kA, nA, kB, K, H, scale, out);
+  return cudaGetLastError();
 }
 
 // ------------------------------------------------------------------ block selection
@@ -393,18 +402,14 @@ cudaError_t launch_block_select(const float* q128, const float* kc128, const flo
   const int nKc = (int)((Lc + 127) / 128), nKq = nQ64;
   // the scores of every row: [H][nQ64][nKc + nKq] (joint), or [H][nQ128][nKc] followed
   // by [H][nQ64][nKq] (separate)
-  auto scores_of = [&](auto tag) {
+  auto scores_of = [&](auto tag) -> cudaError_t {
     constexpr int D = decltype(tag)::value;
-    if (joint) {
-      launch_scores<D>(q64, nQ64, kc128, nKc, kq64, nKc + nKq, H, scale, scores, s);
-    } else {
-      launch_scores<D>(q128, nQ128, kc128, nKc, kc128, nKc, H, scale, scores, s);
-      launch_scores<D>(q64, nQ64, kq64, nKq, kq64, nKq, H, scale, scores + (long long)H * nQ128 * nKc, s);
-    }
+    if (joint) return launch_scores<D>(q64, nQ64, kc128, nKc, kq64, nKc + nKq, H, scale, scores, s);
+    const cudaError_t e = launch_scores<D>(q128, nQ128, kc128, nKc, kc128, nKc, H, scale, scores, s);
+    if (e != cudaSuccess) return e;
+    return launch_scores<D>(q64, nQ64, kq64, nKq, kq64, nKq, H, scale, scores + (long long)H * nQ128 * nKc, s);
   };
-  if (d == 128) scores_of(std::integral_constant<int, 128>());
-  else scores_of(std::integral_constant<int, 64>());
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = d == 128 ? scores_of(std::integral_constant<int, 128>()) : scores_of(std::integral_constant<int, 64>());
   if (e != cudaSuccess) return e;
   int nmax = joint ? nKc + nKq : (nKc > nKq ? nKc : nKq), NB2 = 1;
   while (NB2 < nmax) NB2 <<= 1;
