@@ -35,17 +35,18 @@ DEFAULT_WORKLOAD = 3
 
 TRAFFIC = {
     # dram__bytes_read.sum + dram__bytes_write.sum of one launch, from an ncu capture at
-    # TRAFFIC_WORKLOAD (the summaries under profiles/); valid while the kernel's source
-    # section is unchanged (sha).  Another workload scales them by the KV the kernel
-    # streams ("kv": cached rows x heads x d; "kvq": all KV rows x heads x d).
-    "gather": {"file": "hkv.cu", "section": "gather", "sha": "ea6010aad5d6ab04", "bytes": 306730752 + 248329984,
-               "scale": "kv"},
-    "linformer_proj": {"file": "proj_tc.cu", "section": "kernel", "sha": "58b967d1bbf135b5",
-                       "bytes": 392641024 + 6231040, "scale": "kvq"},
+    # TRAFFIC_WORKLOAD (the summaries under profiles/), with the rows x heads x d of KV
+    # that launch streamed; valid while the kernel's source section is unchanged (sha).
+    # Another workload scales the bytes by its own launch's rows x heads x d.
     "attention_merge": {"file": "attn_tc.cu", "section": "kernel", "sha": "fd734552ee4b2c0f",
-                        "bytes": 279298560 + 19572224, "scale": "kv"},
+                        "bytes": 279298560 + 19572224, "rows": "cached"},
 }
 TRAFFIC_WORKLOAD = 1  # synth.SHAPES index of the captured workload (Wan-1.3B 480p)
+
+
+def launch_rows(name, shape):
+    """KV rows one launch of kernel `name` streams."""
+    return shape.Lc
 
 
 def traffic_of(name, shape):
@@ -57,10 +58,7 @@ def traffic_of(name, shape):
         return None
     import synth
     ref = synth.SHAPES[TRAFFIC_WORKLOAD]
-    if tr["scale"] == "kv":
-        f = (shape.Lc * shape.H * shape.d) / (ref.Lc * ref.H * ref.d)
-    else:
-        f = ((shape.Lc + shape.Lq) * shape.H * shape.d) / ((ref.Lc + ref.Lq) * ref.H * ref.d)
+    f = (launch_rows(name, shape) * shape.H * shape.d) / (launch_rows(name, ref) * ref.H * ref.d)
     return int(round(tr["bytes"] * f))
 
 
@@ -459,7 +457,7 @@ def run_gpu(args, shape, rank, world, local):
         one_step()
     torch.cuda.synchronize()
 
-    trace = hsa.KernelTrace(max_kernels=16 * args.steps)
+    trace = hsa.KernelTrace(max_kernels=64 * args.steps)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     clocks = ClockSampler(local)
@@ -555,12 +553,13 @@ def run_gpu(args, shape, rank, world, local):
     t_kind = "burst" if at_max else "sustained"
     t_peak = peaks["bf16_tflops"] if at_max else peaks["bf16_tflops_sustained"]
     host_gbs = measure_host_link(dev) if shape.host_pages else None
+    # the work below is per step; a kernel launched several times a step would be rated
+    # on its summed time
     kernel_work = {
         # the fused attention kernel: selected-block FLOPs of the sparse branch plus the
         # useful FLOPs of the linear branch (the split-precision extra products not counted)
         "attention_merge": ("tensor", f_sparse + w["lin_attn_flops"]),
         "linformer_proj": ("tensor", w["proj_flops"]),
-        "gather_project": ("tensor", w["proj_hist_flops"]),
         # with a host tier the timed steps gather from the HBM slots the store keeps the
         # selected pages in (host_tier reports the cold fetch over the host link)
         "gather": ("hbm", w["gather_bytes"]),
@@ -570,25 +569,22 @@ def run_gpu(args, shape, rank, world, local):
     kernels = {}
     for name, d in per_kernel.items():
         avg_ms = d["ms"] / d["launches"]
+        step_ms = d["ms"] / args.steps  # the kernel's summed time a step
         entry = {"launches_per_step": d["launches"] / args.steps, "ms_per_launch": avg_ms,
                  "share": d["ms"] / sum(v["ms"] for v in per_kernel.values())}
-        if name == "gather_project":  # also its bytes: the pages read once, Kc / Vc written, E / F read
-            gp_bytes = w["gather_bytes"] + 2.0 * shape.r * shape.Lc * 2
-            entry["hbm_GBps"] = gp_bytes / (avg_ms / 1e3) / 1e9
-            entry["hbm_frac"] = entry["hbm_GBps"] / peaks["hbm_gbs"]
         if name in kernel_work:
             bound, work = kernel_work[name]
             if bound == "tensor":
-                ach = work / (avg_ms / 1e3) / 1e12
+                ach = work / (step_ms / 1e3) / 1e12
                 entry.update({"bound": "tensor", "achieved": ach, "unit": "TFLOP/s", "peak": t_peak,
                               "frac": ach / t_peak, "frac_burst": ach / peaks["bf16_tflops"],
                               "frac_sustained": ach / peaks["bf16_tflops_sustained"]})
             elif bound == "host-link":
-                ach = work / (avg_ms / 1e3) / 1e9  # bytes read over the host link (K and V pages)
+                ach = work / (step_ms / 1e3) / 1e9  # bytes read over the host link (K and V pages)
                 entry.update({"bound": "host-link", "achieved": ach, "unit": "GB/s", "peak": host_gbs,
                               "frac": ach / host_gbs if host_gbs else None})
             else:
-                ach = work / (avg_ms / 1e3) / 1e9
+                ach = work / (step_ms / 1e3) / 1e9
                 entry.update({"bound": "hbm", "achieved": ach, "unit": "GB/s", "peak": peaks["hbm_gbs"],
                               "frac": ach / peaks["hbm_gbs"]})
         tr = traffic_of(name, shape)

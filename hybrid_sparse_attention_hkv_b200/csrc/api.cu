@@ -871,6 +871,25 @@ hsa_status_t hsa_forward_ex(const hsa_config_t* cfg, const hsa_bf16* Q, const hs
                       (flags & HSA_FWD_SELECTED) != 0, stream);
 }
 
+// The Linformer products of the cached KV's rows [r0, r1) into the history products
+// (added to them when `add`), on `stream`.
+static hsa_status_t project_history_rows(const hsa_config_t* cfg, const Layout& L, const hsa_bf16* Kc,
+                                         const hsa_bf16* Vc, const hsa_bf16* E, const hsa_bf16* F,
+                                         long long ef_head_stride, void* ws, long long r0, long long r1, bool add,
+                                         hsa_stream_t stream) {
+  float* part = at<float>(ws, L.projpart);
+  float* hist = at<float>(ws, L.ekfv_hist);
+  int splits = hsa::proj_tc_splits(cfg->H, cfg->d, cfg->rank, r1 - r0, 0, hsa::kProjCached);
+  if (splits > L.splits) splits = L.splits;
+  HSA_LAUNCH("linformer_proj_history",
+             hsa::launch_proj_tc(E, F, ef_head_stride, Kc, Kc, Vc, Vc, cfg->H, cfg->d, cfg->rank, cfg->Lc, cfg->Lq,
+                                 hsa::kProjCached, splits, part, status_of(ws), stream, r0, r1));
+  HSA_LAUNCH("linformer_reduce_history",
+             hsa::launch_proj_reduce(part, splits, cfg->H, cfg->d, cfg->rank, add ? hist : nullptr, hist, nullptr,
+                                     nullptr, nullptr, nullptr, stream));
+  return HSA_OK;
+}
+
 hsa_status_t hkv_gather_project(const hsa_config_t* cfg, const hsa_bf16* const* page_k, const hsa_bf16* const* page_v,
                                 int NP, const int32_t* sel, int Kp, int P_tok, const hsa_bf16* E, const hsa_bf16* F,
                                 long long ef_head_stride, hsa_bf16* Kc, hsa_bf16* Vc, void* ws, size_t ws_bytes,
@@ -892,24 +911,14 @@ hsa_status_t hkv_gather_project(const hsa_config_t* cfg, const hsa_bf16* const* 
     return fail(HSA_ERR_UNSUPPORTED, "%s: ef_head_stride must be 0 (shared) or r * (Lc + Lq) (stacked per head)", fn);
   const Layout L = make_layout(cfg->H, cfg->d, cfg->Lq, cfg->Lc, cfg->rank);
   TRY(check_ws(fn, ws, ws_bytes, L.total));
-  float* part = at<float>(ws, L.projpart);
-  int splits = hsa::proj_tc_splits(cfg->H, cfg->d, cfg->rank, cfg->Lc, cfg->Lq, hsa::kProjCached);
-  if (splits > L.splits) splits = L.splits;
-  hsa::ProjPages pg;
-  pg.page_k = reinterpret_cast<const uint16_t* const*>(page_k);
-  pg.page_v = reinterpret_cast<const uint16_t* const*>(page_v);
-  pg.sel = sel;
-  pg.NP = NP;
-  pg.P_tok = P_tok;
-  pg.Kc_out = Kc;
-  pg.Vc_out = Vc;
-  // the maps of Kc / Vc (and of the chunk tensors) are not read in this mode
-  HSA_LAUNCH("gather_project", hsa::launch_proj_tc(E, F, ef_head_stride, Kc, Kc, Vc, Vc, cfg->H, cfg->d, cfg->rank,
-                                                   cfg->Lc, cfg->Lq, hsa::kProjCached, splits, part, status_of(ws),
-                                                   stream, &pg));
-  HSA_LAUNCH("linformer_reduce_history",
-             hsa::launch_proj_reduce(part, splits, cfg->H, cfg->d, cfg->rank, nullptr, at<float>(ws, L.ekfv_hist),
-                                     nullptr, nullptr, nullptr, nullptr, stream));
+  // The gather, then the history's products on the same stream.  (Two overlaps of
+  // the HBM-bound copy with the tensor-bound projection measured slower on B200: one
+  // kernel copying the pages into the projection's operand ring, and stages of whole
+  // pages gathered on this stream while a side stream projects the previous stage.)
+  HSA_LAUNCH("gather", hsa::launch_gather(reinterpret_cast<const uint16_t* const*>(page_k),
+                                          reinterpret_cast<const uint16_t* const*>(page_v), NP, sel, Kp, P_tok,
+                                          cfg->H, cfg->d, Kc, Vc, nullptr, status_of(ws), stream));
+  TRY(project_history_rows(cfg, L, Kc, Vc, E, F, ef_head_stride, ws, 0, cfg->Lc, false, stream));
   return HSA_OK;
 }
 

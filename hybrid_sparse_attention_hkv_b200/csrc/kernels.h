@@ -145,22 +145,13 @@ constexpr int kProjAll = 0;
 constexpr int kProjCached = 1;
 constexpr int kProjChunk = 2;
 int proj_tc_splits(int H, int d, int r, long long Lc, int Lq, int which_part);
-// With `pages` (kProjCached only): the cached KV's rows are read from the selected
-// pages and also written to Kc_out / Vc_out -- the gather and the history projection
-// in one pass (P_tok a multiple of 64).
-struct ProjPages {
-  const uint16_t* const* page_k;
-  const uint16_t* const* page_v;
-  const int32_t* sel;
-  int NP;
-  long long P_tok;
-  uint16_t* Kc_out;
-  uint16_t* Vc_out;
-};
+// rows_lo / rows_hi (>= 0, multiples of 64, within [0, Lc]; kProjCached only): the
+// launch covers only the cached KV's rows [rows_lo, rows_hi) (one stage of a pipeline
+// over the selected pages).
 cudaError_t launch_proj_tc(const uint16_t* E, const uint16_t* F, long long ef_head_stride, const uint16_t* Kc,
                            const uint16_t* Kq, const uint16_t* Vc, const uint16_t* Vq, int H, int d, int r,
                            long long Lc, int Lq, int which_part, int splits, float* part, int* status,
-                           cudaStream_t s, const ProjPages* pages = nullptr);
+                           cudaStream_t s, long long rows_lo = -1, long long rows_hi = -1);
 // Sum the split partials in a fixed order, plus `add` ([2][H][r][d] fp32, nullable):
 // into fp32 sums `sum_out` when it is given, else into the split-bf16 pairs.
 cudaError_t launch_proj_reduce(const float* part, int splits, int H, int d, int r, const float* add,

@@ -47,16 +47,6 @@ struct PjArgs {
   int chunks_per_split;
   float* part;       // [splits][2][H][r][D]
   int* status;
-  // pages mode (cached chunks only): the K / V rows come from the selected pages of a
-  // page table instead of Kc / Vc, and the first r group's CTAs also write them to
-  // Kc / Vc (the gather and the projection in one pass over the pages)
-  const uint16_t* const* page_k;
-  const uint16_t* const* page_v;
-  const int32_t* sel;
-  int NP;
-  long long P_tok;   // a multiple of 64: a 64-row chunk lies in one page
-  uint16_t* Kc_out;
-  uint16_t* Vc_out;
 };
 
 template <int NB, int MT>  // NB = HP x d accumulator columns per r tile
@@ -98,10 +88,9 @@ __global__ void __launch_bounds__(kPjThreads, 1) proj_tc_kernel(const __grid_con
     tmem_alloc(&s_tmem, Lay::kTmemCols);
     tmem_relinquish();
   }
-  const bool pages = a.page_k != nullptr;
   if (tid == 32) {
     for (int s = 0; s < NS; ++s) {
-      mbar_init(&bar_full[s], pages ? 1 + 128 : 1);  // + the 128 threads that copy the B chunk
+      mbar_init(&bar_full[s], 1);
       mbar_init(&bar_empty[s], 1);
     }
     mbar_init(&bar_acc, 1);
@@ -127,15 +116,13 @@ __global__ void __launch_bounds__(kPjThreads, 1) proj_tc_kernel(const __grid_con
         const int brow = cached ? c * kChunk : (c - a.n_chunks_c) * kChunk;
         const int ecol = cached ? c * kChunk : (int)a.Lc + (c - a.n_chunks_c) * kChunk;
         unsigned char* st = smem + s * Lay::kStageBytes;
-        mbar_arrive_expect_tx(&bar_full[s], pages ? MT * Lay::kEBytes : Lay::kStageBytes);
+        mbar_arrive_expect_tx(&bar_full[s], Lay::kStageBytes);
 #pragma unroll
         for (int t = 0; t < MT; ++t) tma_load_2d(st + t * Lay::kEBytes, mE, &bar_full[s], ecol, erow0 + t * 128);
-        if (!pages) {
 #pragma unroll
-          for (int c2 = 0; c2 < NB / 64; ++c2)
-            tma_load_2d(st + MT * Lay::kEBytes + c2 * (kChunk * 128), cached ? mBc : mBq, &bar_full[s],
-                        h0 * D + c2 * 64, brow);
-        }
+        for (int c2 = 0; c2 < NB / 64; ++c2)
+          tma_load_2d(st + MT * Lay::kEBytes + c2 * (kChunk * 128), cached ? mBc : mBq, &bar_full[s],
+                      h0 * D + c2 * 64, brow);
       }
       __syncwarp();
     }
@@ -168,44 +155,6 @@ __global__ void __launch_bounds__(kPjThreads, 1) proj_tc_kernel(const __grid_con
     if (lane == 0 && ok && nc > 0) mma_commit(&bar_acc);
     __syncwarp();
   } else {
-    if (pages) {
-      // ---- B chunks from the pages: 64 rows x NB columns per stage, 16-byte vectors
-      // into the 128-byte-swizzled layout a TMA box would produce (16-byte unit u of
-      // row r at unit u ^ (r & 7) of the row's 128 bytes), and, by the first r group,
-      // into Kc / Vc as well
-      const int t = tid - 64;  // 0..127
-      const uint16_t* const* table = which ? a.page_v : a.page_k;
-      uint16_t* gout = (rg == 0) ? (which ? a.Vc_out : a.Kc_out) : nullptr;
-      const long long C = (long long)a.H * D;
-      constexpr int kVecPerRow = NB / 8;                   // 16-byte vectors of a row's NB columns
-      constexpr int kVec = kChunk * kVecPerRow / 128;      // per thread per chunk
-      for (int i = 0; i < nc; ++i) {
-        const int s = i % NS;
-        if (!mbar_wait(&bar_empty[s], ((i / NS) & 1) ^ 1, a.status, wlim)) break;
-        const long long row0 = (long long)(c_begin + i) * kChunk;  // first row of the cached KV
-        const long long slot = row0 / a.P_tok;
-        const int p = a.sel[slot];
-        const bool okp = p >= 0 && p < a.NP;
-        if (!okp && t == 0) set_status(a.status, HSA_ERR_DEVICE);
-        const uint16_t* src = okp ? table[p] + (row0 - slot * a.P_tok) * C + (long long)h0 * D : nullptr;
-        unsigned char* bst = smem + s * Lay::kStageBytes + MT * Lay::kEBytes;
-        uint4 w[kVec];
-#pragma unroll
-        for (int u = 0; u < kVec; ++u) {
-          const int v = t + u * 128, r = v / kVecPerRow, cc = v % kVecPerRow;
-          w[u] = okp ? ld_nc_v4(src + (long long)r * C + cc * 8) : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int u = 0; u < kVec; ++u) {
-          const int v = t + u * 128, r = v / kVecPerRow, cc = v % kVecPerRow;
-          const int region = cc / 8, unit = cc % 8;
-          *reinterpret_cast<uint4*>(bst + region * (kChunk * 128) + r * 128 + ((unit ^ (r & 7)) << 4)) = w[u];
-          if (gout) *reinterpret_cast<uint4*>(gout + (row0 + r) * C + (long long)h0 * D + cc * 8) = w[u];
-        }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor core
-        mbar_arrive(&bar_full[s]);
-      }
-    }
     const int wq = warp & 3;
     const int row = 32 * wq + lane;
     const uint32_t loff = (uint32_t)(32 * wq) << 16;
@@ -324,7 +273,7 @@ int proj_tc_splits(int H, int d, int r, long long Lc, int Lq, int part) {
 cudaError_t launch_proj_tc(const uint16_t* E, const uint16_t* F, long long ef_head_stride, const uint16_t* Kc,
                            const uint16_t* Kq, const uint16_t* Vc, const uint16_t* Vq, int H, int d, int r,
                            long long Lc, int Lq, int which_part, int splits, float* part, int* status,
-                           cudaStream_t s, const ProjPages* pg) {
+                           cudaStream_t s, long long rows_lo, long long rows_hi) {
   cudaError_t e = encoder();
   if (e != cudaSuccess) return e;
   const long long L = Lc + Lq;
@@ -344,16 +293,13 @@ cudaError_t launch_proj_tc(const uint16_t* E, const uint16_t* F, long long ef_he
   a.n_chunks = a.n_chunks_c + (Lq + kChunk - 1) / kChunk;
   a.chunk_lo = which_part == kProjChunk ? a.n_chunks_c : 0;
   a.chunk_hi = which_part == kProjCached ? a.n_chunks_c : a.n_chunks;
+  if (which_part == kProjCached && rows_lo >= 0 && rows_hi > rows_lo && rows_hi <= Lc && rows_lo % kChunk == 0) {
+    a.chunk_lo = (int)(rows_lo / kChunk);
+    a.chunk_hi = (int)((rows_hi + kChunk - 1) / kChunk);
+  }
   a.chunks_per_split = (a.chunk_hi - a.chunk_lo + splits - 1) / splits;
   a.part = part;
   a.status = status;
-  a.page_k = pg ? pg->page_k : nullptr;
-  a.page_v = pg ? pg->page_v : nullptr;
-  a.sel = pg ? pg->sel : nullptr;
-  a.NP = pg ? pg->NP : 0;
-  a.P_tok = pg ? pg->P_tok : 0;
-  a.Kc_out = pg ? pg->Kc_out : nullptr;
-  a.Vc_out = pg ? pg->Vc_out : nullptr;
   const int hp = proj_heads_per_cta(H, a.per_head != 0);
   const int mt = proj_tiles_per_cta(r, d, hp);
   const int groups = ((r + 127) / 128 + mt - 1) / mt;

@@ -453,15 +453,15 @@ hsa_status_t hsa_forward_ex(const hsa_config_t* cfg, const hsa_bf16* Q, const hs
                             void* out, int out_is_bf16, const hsa_selection_t* sel, unsigned flags,
                             void* ws, size_t ws_bytes, hsa_stream_t stream);
 
-/* The active-cache gather and the history's Linformer products in one pass over
- * the selected pages ([NEWS] kernel paragraph: the KV copies dominate the
- * preprocessing; the copy and the projection then read each cached row once):
+/* The active-cache gather and the history's Linformer products in one call
+ * ([NEWS] kernel paragraph: the KV copies dominate the preprocessing):
  *   Kc, Vc                as hkv_gather (bitwise copies of pages sel[0..Kp));
  *   history products      as hsa_prepare_history (E_h[:, 0:Lc] Kc_h, F_h[:, 0:Lc] Vc_h,
  *                         fp32 in the workspace), for hsa_forward_reuse /
  *                         hsa_forward_ex(HSA_FWD_HISTORY).
- * Requires P_tok a multiple of 64 and Kp * P_tok == cfg->Lc.  Page tables as
- * hkv_gather; an out-of-range page id sets HSA_ERR_DEVICE.  Uses the workspace. */
+ * Enqueues the gather, then the projection, on `stream`.  Requires P_tok a multiple
+ * of 64 and Kp * P_tok == cfg->Lc.  Page tables as hkv_gather; an out-of-range page
+ * id sets HSA_ERR_DEVICE.  Uses the workspace. */
 hsa_status_t hkv_gather_project(const hsa_config_t* cfg, const hsa_bf16* const* page_k, const hsa_bf16* const* page_v,
                                 int NP, const int32_t* sel, int Kp, int P_tok, const hsa_bf16* E, const hsa_bf16* F,
                                 long long ef_head_stride, hsa_bf16* Kc, hsa_bf16* Vc,
