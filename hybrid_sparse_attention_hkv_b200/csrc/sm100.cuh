@@ -269,28 +269,6 @@ __device__ __forceinline__ void tmem_wait_ld_tied(uint32_t (&r)[128]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(r[0]),"+r"(r[1]),"+r"(r[2]),"+r"(r[3]),"+r"(r[4]),"+r"(r[5]),"+r"(r[6]),"+r"(r[7]),"+r"(r[8]),"+r"(r[9]),"+r"(r[10]),"+r"(r[11]),"+r"(r[12]),"+r"(r[13]),"+r"(r[14]),"+r"(r[15]),"+r"(r[16]),"+r"(r[17]),"+r"(r[18]),"+r"(r[19]),"+r"(r[20]),"+r"(r[21]),"+r"(r[22]),"+r"(r[23]),"+r"(r[24]),"+r"(r[25]),"+r"(r[26]),"+r"(r[27]),"+r"(r[28]),"+r"(r[29]),"+r"(r[30]),"+r"(r[31]),"+r"(r[32]),"+r"(r[33]),"+r"(r[34]),"+r"(r[35]),"+r"(r[36]),"+r"(r[37]),"+r"(r[38]),"+r"(r[39]),"+r"(r[40]),"+r"(r[41]),"+r"(r[42]),"+r"(r[43]),"+r"(r[44]),"+r"(r[45]),"+r"(r[46]),"+r"(r[47]),"+r"(r[48]),"+r"(r[49]),"+r"(r[50]),"+r"(r[51]),"+r"(r[52]),"+r"(r[53]),"+r"(r[54]),"+r"(r[55]),"+r"(r[56]),"+r"(r[57]),"+r"(r[58]),"+r"(r[59]),"+r"(r[60]),"+r"(r[61]),"+r"(r[62]),"+r"(r[63]),"+r"(r[64]),"+r"(r[65]),"+r"(r[66]),"+r"(r[67]),"+r"(r[68]),"+r"(r[69]),"+r"(r[70]),"+r"(r[71]),"+r"(r[72]),"+r"(r[73]),"+r"(r[74]),"+r"(r[75]),"+r"(r[76]),"+r"(r[77]),"+r"(r[78]),"+r"(r[79]),"+r"(r[80]),"+r"(r[81]),"+r"(r[82]),"+r"(r[83]),"+r"(r[84]),"+r"(r[85]),"+r"(r[86]),"+r"(r[87]),"+r"(r[88]),"+r"(r[89]),"+r"(r[90]),"+r"(r[91]),"+r"(r[92]),"+r"(r[93]),"+r"(r[94]),"+r"(r[95]),"+r"(r[96]),"+r"(r[97]),"+r"(r[98]),"+r"(r[99]),"+r"(r[100]),"+r"(r[101]),"+r"(r[102]),"+r"(r[103]),"+r"(r[104]),"+r"(r[105]),"+r"(r[106]),"+r"(r[107]),"+r"(r[108]),"+r"(r[109]),"+r"(r[110]),"+r"(r[111]),"+r"(r[112]),"+r"(r[113]),"+r"(r[114]),"+r"(r[115]),"+r"(r[116]),"+r"(r[117]),"+r"(r[118]),"+r"(r[119]),"+r"(r[120]),"+r"(r[121]),"+r"(r[122]),"+r"(r[123]),"+r"(r[124]),"+r"(r[125]),"+r"(r[126]),"+r"(r[127]) :: "memory");
 }
 
-// 2^x for a pair of arguments on the FMA and integer pipes, to take load off the
-// special-function unit.  Cody-Waite style range reduction (W. J. Cody, W. Waite,
-// "Software Manual for the Elementary Functions", 1980): x = n + f with n the nearest
-// integer (added and removed through the 1.5 * 2^23 rounding constant) and
-// f in [-1/2, 1/2]; 2^f from a degree-3 polynomial fitted to 2^f on that interval
-// (weighted least squares on the relative error; max relative error 7.6e-5 in fp32,
-// below the bf16 rounding of P); the exponent n is added to the result's bit pattern.
-// Arguments below -126 are clamped (results ~1e-38 instead of 0).
-__device__ __forceinline__ float2 ex2_poly2(float2 x) {
-  x.x = fmaxf(x.x, -126.f);
-  x.y = fmaxf(x.y, -126.f);
-  const float2 magic = make_float2(12582912.f, 12582912.f);  // 1.5 * 2^23
-  const float2 y = __fadd2_rn(x, magic);                      // round(x) in the low mantissa bits
-  const float2 n = __fadd2_rn(y, make_float2(-12582912.f, -12582912.f));
-  const float2 f = __fadd2_rn(x, make_float2(-n.x, -n.y));
-  float2 p = __ffma2_rn(make_float2(0.05516991f, 0.05516991f), f, make_float2(0.24260677f, 0.24260677f));
-  p = __ffma2_rn(p, f, make_float2(0.69326091f, 0.69326091f));
-  p = __ffma2_rn(p, f, make_float2(0.99992836f, 0.99992836f));
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(y.x) << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(y.y) << 23)));
-}
-
 // 2^x on the special-function unit (flushes denormal results to zero).
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
