@@ -38,8 +38,8 @@ TRAFFIC = {
     # TRAFFIC_WORKLOAD (the summaries under profiles/), with the rows x heads x d of KV
     # that launch streamed; valid while the kernel's source section is unchanged (sha).
     # Another workload scales the bytes by its own launch's rows x heads x d.
-    "attention_merge": {"file": "attn_tc.cu", "section": "kernel", "sha": "fd734552ee4b2c0f",
-                        "bytes": 279298560 + 19572224, "rows": "cached"},
+    "attention_merge": {"file": "attn_tc.cu", "section": "kernel", "sha": "2da5f949c952ab3f",
+                        "bytes": 277418240 + 18491136, "rows": "cached"},
 }
 TRAFFIC_WORKLOAD = 1  # synth.SHAPES index of the captured workload (Wan-1.3B 480p)
 
