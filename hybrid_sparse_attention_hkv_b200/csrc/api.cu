@@ -829,21 +829,10 @@ hsa_status_t hsa_forward_selected(const hsa_config_t* cfg, const hsa_bf16* Q, co
                       out_is_bf16, sel, ws, ws_bytes, hsa::kProjAll, true, stream);
 }
 
-hsa_status_t hsa_prepare_history(const hsa_config_t* cfg, const hsa_bf16* Kc, const hsa_bf16* Vc, const hsa_bf16* E,
-                                 const hsa_bf16* F, long long ef_head_stride, void* ws, size_t ws_bytes,
-                                 hsa_stream_t stream) {
-  const char* fn = __func__;
-  TRY(check_cfg(fn, cfg, true));
-  if (cfg->Lc > 0) {
-    REQUIRE_PTR(Kc);
-    REQUIRE_PTR(Vc);
-  }
-  REQUIRE_PTR(E);
-  REQUIRE_PTR(F);
-  if (ef_head_stride != 0 && ef_head_stride != (long long)cfg->rank * (cfg->Lc + cfg->Lq))
-    return fail(HSA_ERR_UNSUPPORTED, "%s: ef_head_stride must be 0 (shared) or r * (Lc + Lq) (stacked per head)", fn);
-  const Layout L = make_layout(cfg->H, cfg->d, cfg->Lq, cfg->Lc, cfg->rank);
-  TRY(check_ws(fn, ws, ws_bytes, L.total));
+// The cached KV's Linformer products (E Kc, F Vc; fp32) into the workspace, on `stream`.
+static hsa_status_t project_history(const hsa_config_t* cfg, const Layout& L, const hsa_bf16* Kc, const hsa_bf16* Vc,
+                                    const hsa_bf16* E, const hsa_bf16* F, long long ef_head_stride, void* ws,
+                                    hsa_stream_t stream) {
   float* part = at<float>(ws, L.projpart);
   int splits = hsa::proj_tc_splits(cfg->H, cfg->d, cfg->rank, cfg->Lc, cfg->Lq, hsa::kProjCached);
   if (splits > L.splits) splits = L.splits;
@@ -859,6 +848,24 @@ hsa_status_t hsa_prepare_history(const hsa_config_t* cfg, const hsa_bf16* Kc, co
   return HSA_OK;
 }
 
+hsa_status_t hsa_prepare_history(const hsa_config_t* cfg, const hsa_bf16* Kc, const hsa_bf16* Vc, const hsa_bf16* E,
+                                 const hsa_bf16* F, long long ef_head_stride, void* ws, size_t ws_bytes,
+                                 hsa_stream_t stream) {
+  const char* fn = __func__;
+  TRY(check_cfg(fn, cfg, true));
+  if (cfg->Lc > 0) {
+    REQUIRE_PTR(Kc);
+    REQUIRE_PTR(Vc);
+  }
+  REQUIRE_PTR(E);
+  REQUIRE_PTR(F);
+  if (ef_head_stride != 0 && ef_head_stride != (long long)cfg->rank * (cfg->Lc + cfg->Lq))
+    return fail(HSA_ERR_UNSUPPORTED, "%s: ef_head_stride must be 0 (shared) or r * (Lc + Lq) (stacked per head)", fn);
+  const Layout L = make_layout(cfg->H, cfg->d, cfg->Lq, cfg->Lc, cfg->rank);
+  TRY(check_ws(fn, ws, ws_bytes, L.total));
+  return project_history(cfg, L, Kc, Vc, E, F, ef_head_stride, ws, stream);
+}
+
 hsa_status_t hsa_forward_ex(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc, const hsa_bf16* Vc,
                             const hsa_bf16* Kq, const hsa_bf16* Vq, const float* kbar128, const float* tau,
                             const float* gate_logit, const hsa_bf16* E, const hsa_bf16* F, long long ef_head_stride,
@@ -871,25 +878,6 @@ hsa_status_t hsa_forward_ex(const hsa_config_t* cfg, const hsa_bf16* Q, const hs
                       (flags & HSA_FWD_SELECTED) != 0, stream);
 }
 
-// The Linformer products of the cached KV's rows [r0, r1) into the history products
-// (added to them when `add`), on `stream`.
-static hsa_status_t project_history_rows(const hsa_config_t* cfg, const Layout& L, const hsa_bf16* Kc,
-                                         const hsa_bf16* Vc, const hsa_bf16* E, const hsa_bf16* F,
-                                         long long ef_head_stride, void* ws, long long r0, long long r1, bool add,
-                                         hsa_stream_t stream) {
-  float* part = at<float>(ws, L.projpart);
-  float* hist = at<float>(ws, L.ekfv_hist);
-  int splits = hsa::proj_tc_splits(cfg->H, cfg->d, cfg->rank, r1 - r0, 0, hsa::kProjCached);
-  if (splits > L.splits) splits = L.splits;
-  HSA_LAUNCH("linformer_proj_history",
-             hsa::launch_proj_tc(E, F, ef_head_stride, Kc, Kc, Vc, Vc, cfg->H, cfg->d, cfg->rank, cfg->Lc, cfg->Lq,
-                                 hsa::kProjCached, splits, part, status_of(ws), stream, r0, r1));
-  HSA_LAUNCH("linformer_reduce_history",
-             hsa::launch_proj_reduce(part, splits, cfg->H, cfg->d, cfg->rank, add ? hist : nullptr, hist, nullptr,
-                                     nullptr, nullptr, nullptr, stream));
-  return HSA_OK;
-}
-
 hsa_status_t hkv_gather_project(const hsa_config_t* cfg, const hsa_bf16* const* page_k, const hsa_bf16* const* page_v,
                                 int NP, const int32_t* sel, int Kp, int P_tok, const hsa_bf16* E, const hsa_bf16* F,
                                 long long ef_head_stride, hsa_bf16* Kc, hsa_bf16* Vc, void* ws, size_t ws_bytes,
@@ -898,7 +886,6 @@ hsa_status_t hkv_gather_project(const hsa_config_t* cfg, const hsa_bf16* const* 
   TRY(check_cfg(fn, cfg, true));
   if (NP < 1 || P_tok < 1) return fail(HSA_ERR_INVALID_ARG, "%s: NP = %d, P_tok = %d must be >= 1", fn, NP, P_tok);
   if (Kp < 1 || Kp > NP) return fail(HSA_ERR_INVALID_ARG, "%s: Kp = %d must be in [1, NP]", fn, Kp);
-  if (P_tok % 64 != 0) return fail(HSA_ERR_UNSUPPORTED, "%s: P_tok = %d is not a multiple of 64", fn, P_tok);
   if ((long long)Kp * P_tok != cfg->Lc)
     return fail(HSA_ERR_INVALID_ARG, "%s: Kp * P_tok = %lld differs from cfg->Lc = %d", fn, (long long)Kp * P_tok,
                 cfg->Lc);
@@ -914,12 +901,11 @@ hsa_status_t hkv_gather_project(const hsa_config_t* cfg, const hsa_bf16* const* 
   // The gather, then the history's products on the same stream.  (Two overlaps of
   // the HBM-bound copy with the tensor-bound projection measured slower on B200: one
   // kernel copying the pages into the projection's operand ring, and stages of whole
-  // pages gathered on this stream while a side stream projects the previous stage.)
+  // pages gathered on this stream while a side stream projected the previous stage.)
   HSA_LAUNCH("gather", hsa::launch_gather(reinterpret_cast<const uint16_t* const*>(page_k),
                                           reinterpret_cast<const uint16_t* const*>(page_v), NP, sel, Kp, P_tok,
                                           cfg->H, cfg->d, Kc, Vc, nullptr, status_of(ws), stream));
-  TRY(project_history_rows(cfg, L, Kc, Vc, E, F, ef_head_stride, ws, 0, cfg->Lc, false, stream));
-  return HSA_OK;
+  return project_history(cfg, L, Kc, Vc, E, F, ef_head_stride, ws, stream);
 }
 
 hsa_status_t hsa_forward_reuse(const hsa_config_t* cfg, const hsa_bf16* Q, const hsa_bf16* Kc, const hsa_bf16* Vc,

@@ -145,13 +145,10 @@ constexpr int kProjAll = 0;
 constexpr int kProjCached = 1;
 constexpr int kProjChunk = 2;
 int proj_tc_splits(int H, int d, int r, long long Lc, int Lq, int which_part);
-// rows_lo / rows_hi (>= 0, multiples of 64, within [0, Lc]; kProjCached only): the
-// launch covers only the cached KV's rows [rows_lo, rows_hi) (one stage of a pipeline
-// over the selected pages).
 cudaError_t launch_proj_tc(const uint16_t* E, const uint16_t* F, long long ef_head_stride, const uint16_t* Kc,
                            const uint16_t* Kq, const uint16_t* Vc, const uint16_t* Vq, int H, int d, int r,
                            long long Lc, int Lq, int which_part, int splits, float* part, int* status,
-                           cudaStream_t s, long long rows_lo = -1, long long rows_hi = -1);
+                           cudaStream_t s);
 // Sum the split partials in a fixed order, plus `add` ([2][H][r][d] fp32, nullable):
 // into fp32 sums `sum_out` when it is given, else into the split-bf16 pairs.
 cudaError_t launch_proj_reduce(const float* part, int splits, int H, int d, int r, const float* add,

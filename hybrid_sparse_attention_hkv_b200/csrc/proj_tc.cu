@@ -273,7 +273,7 @@ int proj_tc_splits(int H, int d, int r, long long Lc, int Lq, int part) {
 cudaError_t launch_proj_tc(const uint16_t* E, const uint16_t* F, long long ef_head_stride, const uint16_t* Kc,
                            const uint16_t* Kq, const uint16_t* Vc, const uint16_t* Vq, int H, int d, int r,
                            long long Lc, int Lq, int which_part, int splits, float* part, int* status,
-                           cudaStream_t s, long long rows_lo, long long rows_hi) {
+                           cudaStream_t s) {
   cudaError_t e = encoder();
   if (e != cudaSuccess) return e;
   const long long L = Lc + Lq;
@@ -293,10 +293,6 @@ cudaError_t launch_proj_tc(const uint16_t* E, const uint16_t* F, long long ef_he
   a.n_chunks = a.n_chunks_c + (Lq + kChunk - 1) / kChunk;
   a.chunk_lo = which_part == kProjChunk ? a.n_chunks_c : 0;
   a.chunk_hi = which_part == kProjCached ? a.n_chunks_c : a.n_chunks;
-  if (which_part == kProjCached && rows_lo >= 0 && rows_hi > rows_lo && rows_hi <= Lc && rows_lo % kChunk == 0) {
-    a.chunk_lo = (int)(rows_lo / kChunk);
-    a.chunk_hi = (int)((rows_hi + kChunk - 1) / kChunk);
-  }
   a.chunks_per_split = (a.chunk_hi - a.chunk_lo + splits - 1) / splits;
   a.part = part;
   a.status = status;

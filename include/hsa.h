@@ -459,9 +459,9 @@ hsa_status_t hsa_forward_ex(const hsa_config_t* cfg, const hsa_bf16* Q, const hs
  *   history products      as hsa_prepare_history (E_h[:, 0:Lc] Kc_h, F_h[:, 0:Lc] Vc_h,
  *                         fp32 in the workspace), for hsa_forward_reuse /
  *                         hsa_forward_ex(HSA_FWD_HISTORY).
- * Enqueues the gather, then the projection, on `stream`.  Requires P_tok a multiple
- * of 64 and Kp * P_tok == cfg->Lc.  Page tables as hkv_gather; an out-of-range page
- * id sets HSA_ERR_DEVICE.  Uses the workspace. */
+ * Enqueues the gather, then the projection, on `stream`.  Requires Kp * P_tok ==
+ * cfg->Lc.  Page tables as hkv_gather; an out-of-range page id sets HSA_ERR_DEVICE.
+ * Uses the workspace. */
 hsa_status_t hkv_gather_project(const hsa_config_t* cfg, const hsa_bf16* const* page_k, const hsa_bf16* const* page_v,
                                 int NP, const int32_t* sel, int Kp, int P_tok, const hsa_bf16* E, const hsa_bf16* F,
                                 long long ef_head_stride, hsa_bf16* Kc, hsa_bf16* Vc,
