@@ -182,10 +182,8 @@ cudaError_t launch_scores(const float* q, int R, const float* kA, int nA, const 
 //   emit the k* kept ids ascending                (flag + ordered compaction)
 // tau >= 1 keeps every block.
 constexpr int kSelThreads = 256;
+constexpr int kMaxSortKeys = 16 * kSelThreads;  // blocks a selection row can rank
 
-__device__ __forceinline__ bool ranks_before(float ea, int ia, float eb, int ib) {
-  return ea > eb || (ea == eb && ia < ib);
-}
 
 // Exclusive prefix sum of one value per thread over the block; `total` receives the
 // block's sum in every thread.  warp_tot: shared, kSelThreads / 32 + 1 entries.
@@ -219,6 +217,82 @@ __device__ T block_excl_scan(T v, T* warp_tot, T& total) {
   return r;
 }
 
+// Rank a row's masses: e[0..nK) (>= 0) and their ids, into e / id in rank order
+// (masses descending, equal masses the lower id first), N = E x 256 >= nK a power of
+// two.  Keys mass bits << 32 | ~id order exactly so (the bits of non-negative floats
+// order as their values; padding keys are 0 and rank last).  Bitonic sort with each
+// thread holding E consecutive keys in registers: steps between a thread's own keys
+// swap registers, steps within a warp exchange by shuffles, and only the steps of
+// stride >= 32 E go through shared memory (`keys`, [N], over e and id): six
+// synchronised passes for any N, against log2(N) (log2(N) + 1) / 2 for a block-wide
+// network.
+template <int E>
+__device__ void rank_masses(float* e, int* id, int nK, unsigned long long* keys) {
+  constexpr int N = E * kSelThreads;
+  const int tid = threadIdx.x;
+  unsigned long long v[E];
+#pragma unroll
+  for (int r = 0; r < E; ++r) {
+    const int x = tid * E + r;
+    v[r] = x < nK ? ((unsigned long long)__float_as_uint(e[x]) << 32) | (unsigned)(0xFFFFFFFFu - (unsigned)x) : 0ull;
+  }
+  __syncthreads();  // e is read before any pass writes the keys over it
+  auto cas = [](unsigned long long a, unsigned long long b, bool keep_max) -> unsigned long long {
+    return keep_max ? (a > b ? a : b) : (a < b ? a : b);
+  };
+  // both loops unrolled: every register index below is a compile-time constant
+  constexpr int LOG2N = E == 1 ? 8 : E == 2 ? 9 : E == 4 ? 10 : E == 8 ? 11 : 12;
+  static_assert((1 << LOG2N) == N, "N = E x 256, a power of two");
+#pragma unroll
+  for (int ks = 1; ks <= LOG2N; ++ks) {
+    const int k = 1 << ks;
+#pragma unroll
+    for (int js = ks - 1; js >= 0; --js) {
+      const int j = 1 << js;
+      if (j < E) {  // partner in this thread's registers
+#pragma unroll
+        for (int r = 0; r < E; ++r) {
+          if ((r & j) == 0) {
+            const int x = tid * E + r;
+            const bool desc = (x & k) == 0;  // this block of k ends descending
+            const unsigned long long a = v[r], b = v[r + j];
+            v[r] = cas(a, b, desc);
+            v[r + j] = cas(a, b, !desc);
+          }
+        }
+      } else if (j < 32 * E) {  // partner in this warp: lane ^ (j / E)
+        const int m = j / E;
+#pragma unroll
+        for (int r = 0; r < E; ++r) {
+          const int x = tid * E + r;
+          const unsigned olo = __shfl_xor_sync(0xffffffffu, (unsigned)v[r], m);
+          const unsigned ohi = __shfl_xor_sync(0xffffffffu, (unsigned)(v[r] >> 32), m);
+          const unsigned long long o = ((unsigned long long)ohi << 32) | olo;
+          v[r] = cas(v[r], o, ((x & k) == 0) == ((x & j) == 0));  // the lower of the pair keeps the max in a descending block
+        }
+      } else {  // partner in another warp: through shared memory
+#pragma unroll
+        for (int r = 0; r < E; ++r) keys[tid * E + r] = v[r];
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < E; ++r) {
+          const int x = tid * E + r;
+          v[r] = cas(v[r], keys[x ^ j], ((x & k) == 0) == ((x & j) == 0));
+        }
+        __syncthreads();
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < E; ++r) {
+    const int x = tid * E + r;
+    e[x] = __uint_as_float((unsigned)(v[r] >> 32));
+    id[x] = (int)(0xFFFFFFFFu - (unsigned)v[r]);
+  }
+  __syncthreads();
+}
+
+template <int EMAX>  // the largest E = N / 256 of the launch's rows
 __global__ void __launch_bounds__(kSelThreads) block_select_kernel(
     const float* __restrict__ scores, const float* __restrict__ tau, int H, int nQ128, int nKc, int nQ64, int nKq,
     bool joint, int32_t* __restrict__ inter_idx, int32_t* __restrict__ inter_cnt, int32_t* __restrict__ intra_idx,
@@ -284,11 +358,12 @@ __global__ void __launch_bounds__(kSelThreads) block_select_kernel(
     }
     return;
   }
-  int NB2 = 1;
+  int NB2 = kSelThreads;  // sort size: a power of two >= nK, at least one key a thread
   while (NB2 < nK) NB2 <<= 1;
-  float* e = reinterpret_cast<float*>(smraw);   // [NB2]
-  int* id = reinterpret_cast<int*>(e + NB2);    // [NB2]
+  float* e = reinterpret_cast<float*>(smraw);   // [NB2] masses (rank order after the sort)
+  int* id = reinterpret_cast<int*>(e + NB2);    // [NB2] block ids (rank order after the sort)
   int* flag = id + NB2;                          // [NB2]
+  unsigned long long* keys = reinterpret_cast<unsigned long long*>(smraw);  // [NB2], over e and id
 
   for (int j = tid; j < nK; j += kSelThreads) e[j] = srow[j];
   __syncthreads();
@@ -306,13 +381,7 @@ __global__ void __launch_bounds__(kSelThreads) block_select_kernel(
   __syncthreads();
   m = fred[32];
   for (int j = tid; j < NB2; j += kSelThreads) {
-    if (j < nK) {
-      e[j] = expf(e[j] - m);
-      id[j] = j;
-    } else {
-      e[j] = -1.0f;  // sentinel ranks last
-      id[j] = INT_MAX;
-    }
+    if (j < nK) e[j] = expf(e[j] - m);
     flag[j] = 0;
   }
   __syncthreads();
@@ -329,21 +398,40 @@ __global__ void __launch_bounds__(kSelThreads) block_select_kernel(
   }
   __syncthreads();
   tot = dred[32];
-  // bitonic sort into rank order
-  for (int k = 2; k <= NB2; k <<= 1) {
-    for (int jj = k >> 1; jj > 0; jj >>= 1) {
-      for (int x = tid; x < NB2; x += kSelThreads) {
-        const int y = x ^ jj;
-        if (y > x) {
-          const bool first_half = (x & k) == 0;
-          const bool xb = ranks_before(e[x], id[x], e[y], id[y]);
-          if (first_half != xb) {
-            float te = e[x]; e[x] = e[y]; e[y] = te;
-            int ti = id[x]; id[x] = id[y]; id[y] = ti;
+  // NB2 <= EMAX x 256 (the launch's largest row); only the sizes up to it are built,
+  // so that a launch of short rows keeps few registers a thread.  Rows longer than the
+  // register network takes (kMaxSortKeys) rank with block-wide passes in shared memory.
+  const int E = NB2 / kSelThreads;
+  if (NB2 > kMaxSortKeys) {
+    for (int j = tid; j < NB2; j += kSelThreads) {
+      id[j] = j < nK ? j : INT_MAX;
+      if (j >= nK) e[j] = -1.0f;  // padding ranks last
+    }
+    __syncthreads();
+    for (int k = 2; k <= NB2; k <<= 1) {
+      for (int jj = k >> 1; jj > 0; jj >>= 1) {
+        for (int x = tid; x < NB2; x += kSelThreads) {
+          const int y = x ^ jj;
+          if (y > x) {
+            const bool before = e[x] > e[y] || (e[x] == e[y] && id[x] < id[y]);
+            if (((x & k) == 0) != before) {
+              const float te = e[x]; e[x] = e[y]; e[y] = te;
+              const int ti = id[x]; id[x] = id[y]; id[y] = ti;
+            }
           }
         }
+        __syncthreads();
       }
-      __syncthreads();
+    }
+  } else if (E == 1) rank_masses<1>(e, id, nK, keys);
+  else if constexpr (EMAX >= 2) {
+    if (E == 2) rank_masses<2>(e, id, nK, keys);
+    else if constexpr (EMAX >= 4) {
+      if (E == 4) rank_masses<4>(e, id, nK, keys);
+      else if constexpr (EMAX >= 8) {
+        if (E == 8) rank_masses<8>(e, id, nK, keys);
+        else if constexpr (EMAX >= 16) rank_masses<16>(e, id, nK, keys);
+      }
     }
   }
   // prefix sums over the ranked masses: each thread owns a contiguous chunk
@@ -411,17 +499,26 @@ cudaError_t launch_block_select(const float* q128, const float* kc128, const flo
   };
   cudaError_t e = d == 128 ? scores_of(std::integral_constant<int, 128>()) : scores_of(std::integral_constant<int, 64>());
   if (e != cudaSuccess) return e;
-  int nmax = joint ? nKc + nKq : (nKc > nKq ? nKc : nKq), NB2 = 1;
+  int nmax = joint ? nKc + nKq : (nKc > nKq ? nKc : nKq), NB2 = kSelThreads;
   while (NB2 < nmax) NB2 <<= 1;
   const size_t smem = (size_t)NB2 * 12;
   const int grid = joint ? H * nQ64 : H * (nQ128 + nQ64);
-  if (smem > 48 * 1024) {
-    e = cudaFuncSetAttribute(block_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
+  auto go = [&](auto kernel) -> cudaError_t {
+    if (smem > 48 * 1024) {
+      const cudaError_t r = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (r != cudaSuccess) return r;
+    }
+    kernel<<<grid, kSelThreads, smem, s>>>(scores, tau, H, nQ128, nKc, nQ64, nKq, joint, inter_idx, inter_cnt,
+                                           intra_idx, intra_cnt);
+    return cudaGetLastError();
+  };
+  switch (NB2 / kSelThreads) {
+    case 1: return go(block_select_kernel<1>);
+    case 2: return go(block_select_kernel<2>);
+    case 4: return go(block_select_kernel<4>);
+    case 8: return go(block_select_kernel<8>);
+    default: return go(block_select_kernel<16>);
   }
-  block_select_kernel<<<grid, kSelThreads, smem, s>>>(scores, tau, H, nQ128, nKc, nQ64, nKq, joint, inter_idx,
-                                                      inter_cnt, intra_idx, intra_cnt);
-  return cudaGetLastError();
 }
 
 }  // namespace hsa
