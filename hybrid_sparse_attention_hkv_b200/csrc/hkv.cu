@@ -259,7 +259,7 @@ cudaError_t launch_page_scores_partial(const uint16_t* Q, long long Lq, int C, c
   const int splits = page_score_splits(Lq);
   const long long rps = (Lq + splits - 1) / splits;
   const size_t smem = (size_t)C * 4;
-  if (smem > 48 * 1024) {
+  if (smem > kDefaultSmemOptIn) {
     cudaError_t e = cudaFuncSetAttribute(page_scores_partial_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
@@ -271,7 +271,7 @@ cudaError_t launch_page_scores_partial(const uint16_t* Q, long long Lq, int C, c
 cudaError_t launch_select_pages_final(const float* part, long long Lq, int NP, const int32_t* cand_range, int Kp,
                                       int32_t* sel_out, float* scores_out, int* status, cudaStream_t s) {
   const size_t smem = (size_t)NP * 4;
-  if (smem > 48 * 1024) {
+  if (smem > kDefaultSmemOptIn) {
     cudaError_t e = cudaFuncSetAttribute(select_pages_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;

@@ -9,6 +9,11 @@
 
 namespace hsa {
 
+// Dynamic shared memory above this asks for the opt-in attribute first: a launch may
+// use 48 KB without it, and the kernel's static shared memory (under 1 KB in every
+// kernel that checks this) counts toward the same 48 KB.
+constexpr size_t kDefaultSmemOptIn = 47 * 1024;
+
 // ---------------------------------------------------------------- api.cu
 // Record the text returned by hsa_last_error_detail() and return `code`.
 hsa_status_t api_fail(hsa_status_t code, const char* fmt, ...);

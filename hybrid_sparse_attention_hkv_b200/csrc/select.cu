@@ -160,7 +160,7 @@ cudaError_t launch_scores(const float* q, int R, const float* kA, int nA, const 
                           float* out, cudaStream_t s) {
   if (R == 0 || K == 0) return cudaSuccess;
   const size_t smem = (size_t)(kScoreRows + kScoreKeys) * (D + 4) * sizeof(float);
-  if (smem > 48 * 1024) {
+  if (smem > kDefaultSmemOptIn) {
     const cudaError_t e =
         cudaFuncSetAttribute(block_scores_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -504,7 +504,7 @@ cudaError_t launch_block_select(const float* q128, const float* kc128, const flo
   const size_t smem = (size_t)NB2 * 12;
   const int grid = joint ? H * nQ64 : H * (nQ128 + nQ64);
   auto go = [&](auto kernel) -> cudaError_t {
-    if (smem > 48 * 1024) {
+    if (smem > kDefaultSmemOptIn) {
       const cudaError_t r = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (r != cudaSuccess) return r;
     }

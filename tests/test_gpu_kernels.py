@@ -647,3 +647,26 @@ def test_thread_release_and_recreate():
     torch.cuda.synchronize()
     assert torch.equal(first, second)
     assert hsa.hsa_status_read(ds.step.ws) == 0
+
+
+@pytest.mark.parametrize("nKc", [300, 1000, 2000, 3000, 4200])
+def test_block_selection_row_lengths(nKc):
+    """Selection rows of every length the ranking takes (register networks of 256 to
+    4096 keys, and the shared-memory passes beyond) against the oracle."""
+    H, d, Lq = 2, 64, 128
+    Lc = nKc * 128 - 40  # a partial last block
+    Lc -= Lc % 8
+    cfg = make_config(H, d, Lq, Lc, 0)
+    g = torch.Generator(device="cuda").manual_seed(nKc)
+    Q = torch.randn(Lq, H, d, device="cuda", generator=g).to(torch.bfloat16)
+    Kc = torch.randn(Lc, H, d, device="cuda", generator=g).to(torch.bfloat16)
+    Kq = torch.randn(Lq, H, d, device="cuda", generator=g).to(torch.bfloat16)
+    tau = torch.tensor([0.5, 0.8], dtype=torch.float32, device="cuda")
+    sel = SelectionBuffers.empty(cfg)
+    ws = hsa.workspace(cfg)
+    hsa.hsa_block_select(cfg, Q, Kc, Kq, tau, sel, ws)
+    torch.cuda.synchronize()
+    assert hsa.hsa_status_read(ws) == 0
+    gi = selection_lists(sel.inter_idx.cpu().numpy(), sel.inter_cnt.cpu().numpy())
+    gq = selection_lists(sel.intra_idx.cpu().numpy(), sel.intra_cnt.cpu().numpy())
+    check_selection_both(gi, gq, bits_of(Q), bits_of(Kc), bits_of(Kq), tau.cpu().numpy(), f"nKc {nKc}")
