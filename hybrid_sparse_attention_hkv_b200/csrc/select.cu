@@ -175,14 +175,14 @@ cudaError_t launch_scores(const float* q, int R, const float* kA, int nA, const 
 // One CTA per selection row (head h, query block i, map inter|intra; in joint mode
 // one row per (head, 64-row query block) over the Kc blocks followed by the Kq
 // blocks, whose kept ids are split into the row's inter and intra lists):
-//   s_j = qbar_i . kbar_j * scale                 (fp32, one warp per block)
+//   s_j = qbar_i . kbar_j * scale                 (fp32, block_scores_kernel)
 //   e_j = exp(s_j - max_j s_j);  total = sum_j e_j (fp64)
-//   rank by e descending (ties -> lower j)        (bitonic sort in shared memory)
+//   rank by e descending (ties -> lower j)        (bitonic sort, rank_masses)
 //   k* = first k with sum_{m<k} e_(m) >= tau * total   (fp64 prefix sums)
 //   emit the k* kept ids ascending                (flag + ordered compaction)
 // tau >= 1 keeps every block.
 constexpr int kSelThreads = 256;
-constexpr int kMaxSortKeys = 16 * kSelThreads;  // blocks a selection row can rank
+constexpr int kMaxSortKeys = 16 * kSelThreads;  // longest row ranked in registers; longer rows sort block-wide
 
 
 // Exclusive prefix sum of one value per thread over the block; `total` receives the
