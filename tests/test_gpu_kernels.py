@@ -670,3 +670,40 @@ def test_block_selection_row_lengths(nKc):
     gi = selection_lists(sel.inter_idx.cpu().numpy(), sel.inter_cnt.cpu().numpy())
     gq = selection_lists(sel.intra_idx.cpu().numpy(), sel.intra_cnt.cpu().numpy())
     check_selection_both(gi, gq, bits_of(Q), bits_of(Kc), bits_of(Kq), tau.cpu().numpy(), f"nKc {nKc}")
+
+
+@pytest.mark.parametrize("joint", [False, True], ids=["separate", "joint"])
+def test_block_selection_longest_rows(joint):
+    """The longest selection rows the boundary accepts: 8192 cached blocks (the per-row
+    maximum of a separate map), and in joint mode those plus the chunk's blocks in one
+    row (16384 sort slots, the block-wide ranking), against the oracle."""
+    H, d, Lq = 2, 64, 128
+    nKc = 8192
+    Lc = nKc * 128 - 40
+    Lc -= Lc % 8
+    cfg = make_config(H, d, Lq, Lc, 0, select_mode=hsa.SELECT_JOINT if joint else hsa.SELECT_SEPARATE)
+    g = torch.Generator(device="cuda").manual_seed(8192 + joint)
+    Q = torch.randn(Lq, H, d, device="cuda", generator=g).to(torch.bfloat16)
+    Kc = torch.randn(Lc, H, d, device="cuda", generator=g).to(torch.bfloat16)
+    Kq = torch.randn(Lq, H, d, device="cuda", generator=g).to(torch.bfloat16)
+    tau = torch.tensor([0.5, 0.8], dtype=torch.float32, device="cuda")
+    sel = SelectionBuffers.empty(cfg)
+    ws = hsa.workspace(cfg)
+    hsa.hsa_block_select(cfg, Q, Kc, Kq, tau, sel, ws)
+    torch.cuda.synchronize()
+    assert hsa.hsa_status_read(ws) == 0
+    gi = selection_lists(sel.inter_idx.cpu().numpy(), sel.inter_cnt.cpu().numpy())
+    gq = selection_lists(sel.intra_idx.cpu().numpy(), sel.intra_cnt.cpu().numpy())
+    Qh, Kch, Kqh, t = bits_of(Q), bits_of(Kc), bits_of(Kq), tau.cpu().numpy()
+    del Kc
+    if not joint:
+        check_selection_both(gi, gq, Qh, Kch, Kqh, t, "longest rows")
+        return
+    assert len(gi[0]) == Lq // 64
+    combined = [[np.concatenate([gi[h][i], gq[h][i] + nKc]) for i in range(len(gi[h]))] for h in range(H)]
+    for dt in (np.float32, np.float64):
+        ref = oracle.block_select(Qh, Kch, Kqh, t, dtype=dt, joint=True)
+        ref_c = [[np.concatenate([ref.inter[h][i], ref.intra[h][i] + nKc]) for i in range(len(ref.inter[h]))]
+                 for h in range(H)]
+        n, e = check_selection(combined, ref_c, ref.p_inter, t, f"longest joint rows {dt.__name__}")
+        assert e <= max(1, n // 100)
