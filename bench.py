@@ -104,6 +104,20 @@ def step_work(shape):
     }
 
 
+def kernels_in_scope(name, shape, joint=False):
+    """Kernels one traced library call launches inside a step.  The block selection
+    runs its scores kernel once per map (the inter map only when there is a cached
+    KV; one map in joint mode) and then its ranking kernel; the page store's fetch
+    updates the residency on the device and then launches its copy kernel.  Every
+    other call of the step launches one kernel."""
+    if name == "block_select":
+        maps = 1 if joint else (1 if shape.Lc > 0 else 0) + 1
+        return maps + 1
+    if name == "store_fetch":
+        return 2
+    return 1
+
+
 def exact_pairs(shape, sel_bufs):
     """Selected query-key pairs counted from the selection lists (partial blocks exact)."""
     import numpy as np
@@ -481,7 +495,7 @@ def run_gpu(args, shape, rank, world, local):
     per_kernel = {}
     launches = 0
     for name, ms in trace.results():
-        launches += 1
+        launches += kernels_in_scope(name, shape)
         d = per_kernel.setdefault(name, {"launches": 0, "ms": 0.0})
         d["launches"] += 1
         d["ms"] += ms

@@ -6,6 +6,7 @@ import os
 import socket
 import subprocess
 import sys
+import types
 
 import numpy as np
 import pytest
@@ -165,3 +166,20 @@ def test_head_ranges_cover_every_head_once():
             assert r[0][0] == 0 and r[-1][1] == H
             assert all(a[1] == b[0] for a, b in zip(r, r[1:]))
             assert max(b - a for a, b in r) - min(b - a for a, b in r) <= 1
+
+
+def test_kernel_count_of_a_step():
+    """The bench's launch count: the traced calls of one step and the kernels each
+    launches add up to the per-step launches of the ncu launch list (14B 720p: 12
+    kernels a step, the block selection's scores kernel twice)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    c3 = synth.SHAPES[3]
+    step = ["page_scores_partial", "select_pages_final", "kc128_from_pages", "gather", "pool", "block_select",
+            "linformer_proj", "linformer_reduce", "attn_plan", "attention_merge"]
+    assert bench.kernels_in_scope("block_select", c3) == 3
+    assert sum(bench.kernels_in_scope(n, c3) for n in step) == 12
+    assert bench.kernels_in_scope("block_select", c3, joint=True) == 2
+    no_history = types.SimpleNamespace(Lc=0)  # no cached KV: the intra map alone
+    assert bench.kernels_in_scope("block_select", no_history) == 2
+    assert bench.kernels_in_scope("store_fetch", synth.SHAPES[4]) == 2
