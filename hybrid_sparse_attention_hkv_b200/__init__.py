@@ -10,6 +10,7 @@ from __future__ import annotations
 
 import ctypes
 import os
+from contextlib import contextmanager
 from dataclasses import dataclass
 
 import torch
@@ -29,7 +30,7 @@ EXPORTED = [
     "hkv_store_state_size", "hkv_store_init", "hkv_store_tables", "hkv_store_seal", "hkv_store_fetch",
     "hkv_store_prefetch", "hkv_store_residency", "hkv_select_pages_policy", "hkv_page_scores", "hkv_select_top",
     "hsa_sparse_attn_lse", "hsa_fidelity", "hkv_page_block_sums", "hkv_block_means_from_pages",
-    "hsa_forward_selected", "hsa_forward_ex", "hkv_gather_project",
+    "hsa_forward_selected", "hsa_forward_ex", "hkv_gather_project", "hsa_inject_fault",
 ]
 
 FWD_SELECTED, FWD_HISTORY = 1, 2
@@ -119,6 +120,7 @@ def load_library(path: str = LIB_PATH):
         "hsa_set_wait_limit": (I, [P, ctypes.c_uint, P]),
         "hsa_selftest_wait": (I, [P, P, P]),
         "hsa_thread_release": (I, []),
+        "hsa_inject_fault": (I, [I]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -191,6 +193,26 @@ def hsa_selftest_wait(ws, waited_ns=None, stream=None):
 
 def hsa_thread_release():
     _check(load_library().hsa_thread_release(), "hsa_thread_release")
+
+
+FAULT_NONE, FAULT_ARG, FAULT_WORKSPACE, FAULT_LAUNCH = 0, 1, 2, 3
+
+
+def hsa_inject_fault(kind: int):
+    """Make this thread's library calls fail at their configuration check
+    (FAULT_ARG), workspace check (FAULT_WORKSPACE) or first kernel launch
+    (FAULT_LAUNCH) until FAULT_NONE is set again."""
+    _check(load_library().hsa_inject_fault(int(kind)), "hsa_inject_fault")
+
+
+@contextmanager
+def injected_fault(kind: int):
+    """hsa_inject_fault(kind) for the duration of a with-block."""
+    hsa_inject_fault(kind)
+    try:
+        yield
+    finally:
+        hsa_inject_fault(FAULT_NONE)
 
 
 @dataclass

@@ -19,6 +19,7 @@ thread_local cudaEvent_t* t_events = nullptr;
 thread_local const char** t_names = nullptr;
 thread_local int t_pairs = 0;
 thread_local int t_count = 0;
+thread_local int t_fault = HSA_FAULT_NONE;  // hsa_inject_fault
 
 hsa_status_t fail(hsa_status_t code, const char* fmt, ...) {
   va_list ap;
@@ -46,6 +47,7 @@ struct TraceScope {
 
 #define HSA_LAUNCH(name, call)                                                   \
   do {                                                                           \
+    if (t_fault == HSA_FAULT_LAUNCH) return fail(HSA_ERR_CUDA, "%s: injected launch failure", name); \
     cudaError_t _e;                                                              \
     {                                                                            \
       TraceScope _tr(name, stream);                                              \
@@ -144,6 +146,7 @@ hsa_status_t check_heads(const char* fn, int H, int d) {
 }
 
 hsa_status_t check_cfg(const char* fn, const hsa_config_t* c, bool need_rank) {
+  if (t_fault == HSA_FAULT_ARG) return fail(HSA_ERR_INVALID_ARG, "%s: injected argument failure", fn);
   if (!c) return fail(HSA_ERR_INVALID_ARG, "%s: cfg is NULL", fn);
   hsa_status_t st = check_heads(fn, c->H, c->d);
   if (st != HSA_OK) return st;
@@ -203,6 +206,7 @@ cudaError_t side_stream(SideStream** out) {
 }
 
 hsa_status_t check_ws(const char* fn, const void* ws, size_t ws_bytes, size_t need) {
+  if (t_fault == HSA_FAULT_WORKSPACE) return fail(HSA_ERR_WORKSPACE, "%s: injected workspace failure", fn);
   if (!ws) return fail(HSA_ERR_WORKSPACE, "%s: workspace is NULL", fn);
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return fail(HSA_ERR_WORKSPACE, "%s: workspace not 256-byte aligned", fn);
   if (ws_bytes < need) return fail(HSA_ERR_WORKSPACE, "%s: workspace %zu bytes < %zu needed", fn, ws_bytes, need);
@@ -226,6 +230,8 @@ hsa_status_t check_sel(const char* fn, const hsa_selection_t& s) {
 }  // namespace
 
 namespace hsa {
+int injected_fault() { return t_fault; }
+
 hsa_status_t api_fail(hsa_status_t code, const char* fmt, ...) {
   va_list ap;
   va_start(ap, fmt);
@@ -236,6 +242,12 @@ hsa_status_t api_fail(hsa_status_t code, const char* fmt, ...) {
 }  // namespace hsa
 
 extern "C" {
+
+hsa_status_t hsa_inject_fault(int kind) {
+  if (kind < HSA_FAULT_NONE || kind > HSA_FAULT_LAUNCH) return fail(HSA_ERR_INVALID_ARG, "hsa_inject_fault: kind = %d", kind);
+  t_fault = kind;
+  return HSA_OK;
+}
 
 const char* hsa_status_string(hsa_status_t s) {
   switch (s) {
@@ -273,6 +285,7 @@ hsa_status_t hsa_set_wait_limit(void* ws, unsigned int limit_us, hsa_stream_t st
   if (!ws) return fail(HSA_ERR_WORKSPACE, "hsa_set_wait_limit: workspace is NULL");
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
     return fail(HSA_ERR_WORKSPACE, "hsa_set_wait_limit: workspace not 256-byte aligned");
+  if (t_fault == HSA_FAULT_LAUNCH) return fail(HSA_ERR_CUDA, "hsa_set_wait_limit: injected launch failure");
   cudaError_t e = hsa::launch_set_wait_limit(status_of(ws), limit_us, stream);
   return e == cudaSuccess ? HSA_OK : fail(HSA_ERR_CUDA, "hsa_set_wait_limit: %s", cudaGetErrorString(e));
 }
@@ -282,6 +295,7 @@ hsa_status_t hsa_selftest_wait(void* ws, unsigned long long* waited_ns, hsa_stre
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
     return fail(HSA_ERR_WORKSPACE, "hsa_selftest_wait: workspace not 256-byte aligned");
   OPTIONAL_PTR8(waited_ns);
+  if (t_fault == HSA_FAULT_LAUNCH) return fail(HSA_ERR_CUDA, "hsa_selftest_wait: injected launch failure");
   cudaError_t e = hsa::launch_wait_selftest(status_of(ws), waited_ns, stream);
   return e == cudaSuccess ? HSA_OK : fail(HSA_ERR_CUDA, "hsa_selftest_wait: %s", cudaGetErrorString(e));
 }

@@ -17,6 +17,8 @@ constexpr size_t kDefaultSmemOptIn = 47 * 1024;
 // ---------------------------------------------------------------- api.cu
 // Record the text returned by hsa_last_error_detail() and return `code`.
 hsa_status_t api_fail(hsa_status_t code, const char* fmt, ...);
+// The calling thread's injected fault kind (HSA_FAULT_*; hsa_inject_fault).
+int injected_fault();
 
 // ---------------------------------------------------------------- hkv.cu
 constexpr int kColMaxSplits = 296;  // 2 CTAs per SM for the column-sum partial pass

@@ -106,6 +106,7 @@ extern "C" hsa_status_t hkv_select_pages_noalloc(const float* kbar_pages, int NP
       return hsa::api_fail(HSA_ERR_INVALID_ARG, "%s: kbar_pages and Q must be non-NULL and 16-byte aligned", fn);
   if (!sel_out) return hsa::api_fail(HSA_ERR_INVALID_ARG, "%s: sel_out is NULL", fn);
 
+  if (hsa::injected_fault() == HSA_FAULT_LAUNCH) return hsa::api_fail(HSA_ERR_CUDA, "%s: injected launch failure", fn);
   void* base = nullptr;
   hsa_status_t st = scratch_address(&base);
   if (st != HSA_OK) return st;

@@ -148,6 +148,25 @@ hsa_status_t hsa_selftest_wait(void* ws, unsigned long long* waited_ns, hsa_stre
  * it before a thread that used hsa_forward exits, or to release the handles. */
 hsa_status_t hsa_thread_release(void);
 
+/* Host-side fault injection, for tests of a caller's error handling that fault no
+ * GPU (failure detection; the pages have no counterpart).  Sets the calling
+ * thread's fault kind until it is set back to HSA_FAULT_NONE:
+ *   HSA_FAULT_ARG        the configuration check of every entry point that takes
+ *                        an hsa_config_t fails: HSA_ERR_INVALID_ARG;
+ *   HSA_FAULT_WORKSPACE  the workspace check of every entry point that takes a
+ *                        workspace fails: HSA_ERR_WORKSPACE;
+ *   HSA_FAULT_LAUNCH     every entry point that launches kernels fails at its
+ *                        first launch, before it: HSA_ERR_CUDA.
+ * A failing call enqueues no kernel (hsa_forward may already have ordered its
+ * side stream after `stream`) and leaves its outputs and the workspace as they
+ * were; hsa_last_error_detail() says "injected".  Other threads are not affected.
+ * HSA_ERR_INVALID_ARG for an unknown kind. */
+#define HSA_FAULT_NONE 0
+#define HSA_FAULT_ARG 1
+#define HSA_FAULT_WORKSPACE 2
+#define HSA_FAULT_LAUNCH 3
+hsa_status_t hsa_inject_fault(int kind);
+
 /* ---------------------------------------------------------------- HKV ---- */
 
 /* Page descriptor ([NEWS] HKV paragraph; reading: the mean key of the page per

@@ -89,6 +89,58 @@ def test_null_and_misaligned_pointers_rejected(lib):
     assert code == 1
 
 
+def test_injected_faults_fail_before_any_launch(lib):
+    """Host-side fault injection: each kind fails its check with its code and an
+    "injected" detail, before anything is launched; setting it back restores the
+    ordinary checks; the kind belongs to the calling thread."""
+    import threading
+    cfg = hsa.make_config(2, 64, 256, 512, 64)
+    P = ctypes.c_void_p
+    a = P(0x10000)
+    ws = P(0x100000)
+    sel = hsa._Selection(0x20000, 0x30000, 0x40000, 0x50000)
+
+    def block_select(ws_bytes):
+        return lib.hsa_block_select(ctypes.byref(cfg), a, a, a, None, a, sel, ws, ws_bytes, None)
+
+    def detail():
+        return lib.hsa_last_error_detail().decode()
+
+    with hsa.injected_fault(hsa.FAULT_ARG):
+        with pytest.raises(hsa.HsaError) as e:
+            hsa.hsa_workspace_size(cfg)
+        assert e.value.code == 1 and "injected" in str(e.value)
+    with hsa.injected_fault(hsa.FAULT_WORKSPACE):
+        assert block_select(1 << 30) == 3 and "injected workspace" in detail()
+    with hsa.injected_fault(hsa.FAULT_LAUNCH):
+        # every check passes; the first launch (the pooling) fails before it is made
+        assert block_select(1 << 30) == 4 and "pool: injected launch" in detail()
+        code = lib.hkv_select_pages_noalloc(a, 4, None, a, 256, 2, 64, 2, a, None, None, None)
+        assert code == 4 and "injected launch" in detail()
+    # back to the ordinary checks
+    assert hsa.hsa_workspace_size(cfg) > 0
+    assert block_select(1024) == 3 and "injected" not in detail()
+    with pytest.raises(hsa.HsaError) as e:
+        hsa.hsa_inject_fault(7)
+    assert e.value.code == 1
+    # another thread's fault does not reach this one
+    seen = {}
+
+    def other():
+        with hsa.injected_fault(hsa.FAULT_ARG):
+            try:
+                hsa.hsa_workspace_size(cfg)
+                seen["other"] = 0
+            except hsa.HsaError as err:
+                seen["other"] = err.code
+
+    t = threading.Thread(target=other)
+    t.start()
+    t.join()
+    assert seen["other"] == 1
+    assert hsa.hsa_workspace_size(cfg) > 0
+
+
 def test_product_path_never_imports_the_oracle():
     """The package and its native sources carry no reference to the oracle."""
     pkg = os.path.join(ROOT, "hybrid_sparse_attention_hkv_b200")
