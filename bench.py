@@ -137,6 +137,18 @@ def exact_pairs(shape, sel_bufs):
     return pairs, float(ic.sum()) / max(1, ic.size * len(kc_size)), float(qc.sum()) / max(1, qc.size * len(kq_size))
 
 
+def kept_fraction_per_head(shape, sel_bufs):
+    """Per head, the fraction of (query block, key block) pairs kept in the inter and
+    in the intra map (the head-adaptive threshold keeps more blocks at larger tau_h)."""
+    H, Lq, Lc = shape.H, shape.Lq, shape.Lc
+    nkc, nkq = -(-Lc // 128), -(-Lq // 64)
+    ic = sel_bufs.inter_cnt.cpu().double().reshape(H, -1)
+    qc = sel_bufs.intra_cnt.cpu().double().reshape(H, -1)
+    inter = (ic.sum(1) / max(1, ic.shape[1] * nkc)).tolist()
+    intra = (qc.sum(1) / max(1, qc.shape[1] * nkq)).tolist()
+    return [round(v, 4) for v in inter], [round(v, 4) for v in intra]
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples; mark() brackets the timed region."""
@@ -556,6 +568,7 @@ def run_gpu(args, shape, rank, world, local):
     # work and rooflines
     peaks = load_peaks()
     pairs, inter_frac, intra_frac = exact_pairs(shape, st.selection)
+    inter_h, intra_h = kept_fraction_per_head(shape, st.selection)
     w = step_work(shape)
     f_sparse = 4.0 * shape.d * pairs
     f_total = f_sparse + w["proj_flops"] + w["lin_attn_flops"]
@@ -623,7 +636,8 @@ def run_gpu(args, shape, rank, world, local):
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded)",
         "config": workload_config(shape, args),
         "eff_tflops": eff_tflops,
-        "selected_fraction": {"inter": inter_frac, "intra": intra_frac},
+        "selected_fraction": {"inter": inter_frac, "intra": intra_frac,
+                              "inter_per_head": inter_h, "intra_per_head": intra_h},
         "roofline": roofline,
         "kernels": kernels,
         "gpu_launches": launches,

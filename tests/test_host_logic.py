@@ -183,3 +183,44 @@ def test_kernel_count_of_a_step():
     no_history = types.SimpleNamespace(Lc=0)  # no cached KV: the intra map alone
     assert bench.kernels_in_scope("block_select", no_history) == 2
     assert bench.kernels_in_scope("store_fetch", synth.SHAPES[4]) == 2
+
+
+def test_bench_pair_count_and_kept_fractions():
+    """The FLOP count behind the attention roofline: selected query-key pairs from
+    the selection lists, partial query and key blocks at their real sizes.  A
+    hand-worked selection (H = 2, Lq = 200, Lc = 300: query blocks of 128 + 72 and
+    4 x 64 - 56, cached blocks 128 + 128 + 44) gives 103072 pairs, and a token-level
+    mask built from the same lists counts the same."""
+    import torch
+    sys.path.insert(0, ROOT)
+    import bench
+    H, Lq, Lc = 2, 200, 300
+    shape = types.SimpleNamespace(H=H, Lq=Lq, Lc=Lc)
+    inter = [[[0, 2], [1]], [[0, 1, 2], [2]]]            # [h][128-row query block] -> cached blocks
+    intra = [[[0], [3], [0, 1, 2, 3], [2]], [[0], [1], [2], [3]]]  # [h][64-row query block] -> chunk blocks
+
+    def buffers(lists, n_blocks):
+        idx = torch.full((H, len(lists[0]), n_blocks), -1, dtype=torch.int32)
+        cnt = torch.zeros(H, len(lists[0]), dtype=torch.int32)
+        for h, rows in enumerate(lists):
+            for i, kept in enumerate(rows):
+                idx[h, i, :len(kept)] = torch.tensor(kept, dtype=torch.int32)
+                cnt[h, i] = len(kept)
+        return idx, cnt
+
+    ii, ic = buffers(inter, 3)
+    qi, qc = buffers(intra, 4)
+    sel = types.SimpleNamespace(inter_idx=ii, inter_cnt=ic, intra_idx=qi, intra_cnt=qc)
+    pairs, f_inter, f_intra = bench.exact_pairs(shape, sel)
+    assert pairs == 103072
+    mask = np.zeros((H, Lq, Lc + Lq), dtype=bool)
+    for h in range(H):
+        for t in range(Lq):
+            for j in inter[h][t // 128]:
+                mask[h, t, 128 * j:min(Lc, 128 * j + 128)] = True
+            for j in intra[h][t // 64]:
+                mask[h, t, Lc + 64 * j:Lc + min(Lq, 64 * j + 64)] = True
+    assert int(mask.sum()) == pairs
+    assert f_inter == 7 / 12 and f_intra == 11 / 32
+    per_inter, per_intra = bench.kept_fraction_per_head(shape, sel)
+    assert per_inter == [0.5, 0.6667] and per_intra == [0.4375, 0.25]
