@@ -224,3 +224,18 @@ def test_bench_pair_count_and_kept_fractions():
     assert f_inter == 7 / 12 and f_intra == 11 / 32
     per_inter, per_intra = bench.kept_fraction_per_head(shape, sel)
     assert per_inter == [0.5, 0.6667] and per_intra == [0.4375, 0.25]
+
+
+def test_bench_work_model_closed_forms():
+    """The algorithmic work the bench divides by: Linformer FLOPs
+    H (4 r L d + 4 Lq r d) (93.2 GFLOP at the 1.3B 480p workload) and gather bytes
+    4 Lc H d x 2 (613 MB at 1.3B 480p, 2.04 GB at 14B 480p, 4.72 GB at 14B 720p)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    c1, c2, c3 = synth.SHAPES[1], synth.SHAPES[2], synth.SHAPES[3]
+    w1 = bench.step_work(c1)
+    assert abs(w1["proj_flops"] + w1["lin_attn_flops"] - 93.2e9) < 0.05e9
+    assert w1["proj_flops"] == w1["proj_hist_flops"] + w1["proj_chunk_flops"]
+    assert round(w1["gather_bytes"] / 1e6) == 613
+    assert round(bench.step_work(c2)["gather_bytes"] / 1e7) == 204
+    assert round(bench.step_work(c3)["gather_bytes"] / 1e7) == 472
